@@ -1,0 +1,258 @@
+/*
+ * sq_oracle.c -- plain, slow CPU oracle for the SmoothQuant smoothed W8A8 linear layer.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the smoke check and the benchmark's CPU-baseline
+ * leg may load or run this code. It shares nothing with the CUDA library: no header, no helper,
+ * no table. Every step is written the way the pages state it, in plain loops, so that a reader
+ * can check it against them by eye.
+ *
+ * Pages cited (title, then section / equation / figure):
+ *   [MIGRATE] "06 -- SmoothQuant: Migrating Difficulty from Activations to Weights"
+ *   [TAMING]  "Taming the Outliers: A Deep Dive into SmoothQuant for LLM Quantization"
+ *   [W8A8]    "SmoothQuant and W8A8: Quantizing Activations Too"
+ *   [WOVS]    "SmoothQuant: Weight-Only vs W8A8"
+ *
+ * Readings where the pages are silent or disagree (each is also listed in the design notes):
+ *   - Quantiser: symmetric, delta = max|v| / 127, code = round-half-away-from-zero(v * (127/max|v|)),
+ *     clamped to [-127, 127]. The pages leave the tie rule open ([TAMING], "Why Outliers Break
+ *     Quantization") or use half-to-even in a listing; half-away is the fixed reading. The
+ *     reciprocal-multiply form (v * fl32(127/m)) is the fixed reading of "v / delta".
+ *   - All per-element arithmetic is binary32 with each operation rounded (compile with
+ *     -ffp-contract=off, no fast-math); the RMSNorm sum of squares is accumulated in binary64.
+ *   - RMSNorm is the standard x / sqrt(mean(x^2) + eps) * gamma (the pages name RMSNorm but do not
+ *     print it).
+ *   - Scale floors: both abs-maxima and s itself are floored at 1e-5 (binary32 constant).
+ *
+ * bf16 tensors are passed as uint16_t bit patterns.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORC_FLOOR 1e-5f
+#define ORC_QMAX 127
+
+/* bf16 -> binary32 is exact: the bf16 bits are the high half of the binary32 pattern. */
+static float bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* binary32 -> bf16, round to nearest, ties to even. The 16 dropped bits are the remainder:
+ * more than half an ulp rounds the magnitude up, exactly half rounds to the even neighbour.
+ * A carry out of the mantissa moves into the exponent, which is the correct next value. */
+static uint16_t f32_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu) != 0u)
+        return (uint16_t)((u >> 16) | 0x0040u); /* NaN stays a quiet NaN */
+    uint32_t kept = u & 0xFFFF0000u;
+    uint32_t rem = u & 0x0000FFFFu;
+    if (rem > 0x8000u || (rem == 0x8000u && (kept & 0x00010000u) != 0u))
+        kept += 0x00010000u;
+    return (uint16_t)(kept >> 16);
+}
+
+uint16_t orc_f32_to_bf16(float f) { return f32_to_bf16_rne(f); }
+float orc_bf16_to_f32(uint16_t h) { return bf16_to_f32(h); }
+
+/* Symmetric INT8 code of one value, [TAMING] "Why Outliers Break Quantization" (quantisation
+ * equation): v / delta rounded to the nearest integer. roundf is C99's round-half-away-from-zero. */
+static int8_t quantize_one(float v, float inv_delta)
+{
+    float t = v * inv_delta;
+    float r = roundf(t);
+    if (r > (float)ORC_QMAX) r = (float)ORC_QMAX;
+    if (r < -(float)ORC_QMAX) r = -(float)ORC_QMAX;
+    return (int8_t)r;
+}
+
+/* Quantise one row of already-smoothed binary32 values with one symmetric scale:
+ * m = max|v|, delta = m / 127, codes = round(v * (127 / m)). A zero row gives delta 0, codes 0.
+ * [MIGRATE] section 7 (one scale per output row / per token), [W8A8] "One layer, measured". */
+static void quantize_row(const float *v, int64_t n, int8_t *q, float *delta_out)
+{
+    float m = 0.0f;
+    for (int64_t k = 0; k < n; ++k) {
+        float a = fabsf(v[k]);
+        if (a > m) m = a;
+    }
+    if (m == 0.0f) {
+        for (int64_t k = 0; k < n; ++k) q[k] = 0;
+        *delta_out = 0.0f;
+        return;
+    }
+    float delta = m / (float)ORC_QMAX;
+    float inv = (float)ORC_QMAX / m;
+    for (int64_t k = 0; k < n; ++k) q[k] = quantize_one(v[k], inv);
+    *delta_out = delta;
+}
+
+/* Inverse RMS of one bf16 row: 1 / sqrt(mean(x^2) + eps), sum of squares in binary64 taken in
+ * index order, then each later step rounded to binary32. */
+static float row_inv_rms(const uint16_t *x, int64_t K, float eps)
+{
+    double ss = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+        double v = (double)bf16_to_f32(x[k]);
+        ss += v * v;
+    }
+    float ms = (float)(ss / (double)K);
+    float r = sqrtf(ms + eps);
+    return 1.0f / r;
+}
+
+/*
+ * Per-input-channel abs-max over the rows of a row-major bf16 matrix a[rows, cols] (leading
+ * dimension ld elements): amax[j] = max_r |a[r, j]|.
+ *   [MIGRATE] section 3 (max|X_j| from calibration samples); [TAMING] "System Architecture"
+ *   (flowchart: "Calculate max(|X|) per channel", "Calculate max(|W|) per channel").
+ * With norm_gamma non-null each row is first replaced by its RMSNorm output
+ *   y = (x * inv_rms) * gamma_j,
+ * the input the linear layer actually sees ([W8A8] "The trick: move the range into the weights":
+ * X comes out of a normalisation layer).
+ * accumulate != 0 keeps a running maximum with the values already in amax (calibration over
+ * several batches); otherwise amax is overwritten.
+ * For a weight stored [N, K] (output channel n, input channel k) the same call over rows n gives
+ * max|W_k| per input channel.
+ */
+void orc_calibrate_absmax(const uint16_t *a, int64_t rows, int64_t cols, int64_t ld,
+                          const float *norm_gamma, float eps, float *amax, int accumulate)
+{
+    if (!accumulate)
+        for (int64_t j = 0; j < cols; ++j) amax[j] = 0.0f;
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *row = a + r * ld;
+        float ir = norm_gamma ? row_inv_rms(row, cols, eps) : 1.0f;
+        for (int64_t j = 0; j < cols; ++j) {
+            float v = bf16_to_f32(row[j]);
+            if (norm_gamma) v = (v * ir) * norm_gamma[j];
+            float av = fabsf(v);
+            if (av > amax[j]) amax[j] = av;
+        }
+    }
+}
+
+/*
+ * Smoothing factors, [MIGRATE] section 3 and [W8A8] "The trick: move the range into the weights":
+ *   s_j = max|X_j|^alpha / max|W_j|^(1 - alpha),
+ * evaluated in binary64 and rounded once to binary32, then floored at 1e-5 as in the
+ * [TAMING] "Implementation in PyTorch" listing (clamp of s). Both abs-maxima are floored at 1e-5
+ * first so that an all-zero channel gives a finite s.
+ * The fold into the preceding norm, [W8A8] "The trick..." (s folded into the norm weights):
+ *   fold_j = gamma_j / s_j, or 1 / s_j when gamma is null (no norm: the activations are divided
+ *   by s directly, [TAMING] flowchart "Smoothing: X_hat = X / s").
+ * fold may be null.
+ */
+void orc_compute_scales(const float *amax_x, const float *amax_w, int64_t K, float alpha,
+                        const float *gamma, float *s, float *fold)
+{
+    double ea = (double)alpha;
+    double eb = 1.0 - (double)alpha;
+    for (int64_t j = 0; j < K; ++j) {
+        double a = (double)fmaxf(amax_x[j], ORC_FLOOR);
+        double b = (double)fmaxf(amax_w[j], ORC_FLOOR);
+        float sj = (float)(pow(a, ea) / pow(b, eb));
+        sj = fmaxf(sj, ORC_FLOOR);
+        s[j] = sj;
+        if (fold) fold[j] = gamma ? gamma[j] / sj : 1.0f / sj;
+    }
+}
+
+/*
+ * Weight smoothing and per-output-channel INT8 quantisation.
+ *   W_hat = diag(s) * W ([MIGRATE] section 2; [TAMING] flowchart "Update Weights"): the weights
+ *   that read input channel k are multiplied by s_k. Stored [N, K], that is column k.
+ *   Then one symmetric scale per output row n ([MIGRATE] section 7: "one scale per output row").
+ * s null means unsmoothed (s = 1).
+ */
+void orc_smooth_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *s,
+                                int8_t *wq, float *w_scale, float *work /* [K] */)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        const uint16_t *row = w + n * K;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = bf16_to_f32(row[k]);
+            work[k] = s ? v * s[k] : v;
+        }
+        quantize_row(work, K, wq + n * K, &w_scale[n]);
+    }
+}
+
+/*
+ * Online activation path for T tokens of width K.
+ *   apply_norm != 0: y = (x * inv_rms) * fold_k with fold = gamma / s folded into the RMSNorm
+ *   weight ([W8A8] "The trick..."); apply_norm == 0: y = x * fold_k with fold = 1 / s
+ *   ([TAMING] flowchart "Smoothing: X_hat = X / s").
+ *   Then one dynamic symmetric scale per token ([MIGRATE] section 7; [W8A8] "The full model,
+ *   served": each token's maximum is found before the matrix product).
+ */
+void orc_rmsnorm_smooth_quant(const uint16_t *x, int64_t T, int64_t K, const float *fold,
+                              float eps, int apply_norm, int8_t *xq, float *x_scale,
+                              float *work /* [K] */)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        const uint16_t *row = x + t * K;
+        float ir = apply_norm ? row_inv_rms(row, K, eps) : 1.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = bf16_to_f32(row[k]);
+            work[k] = apply_norm ? (v * ir) * fold[k] : v * fold[k];
+        }
+        quantize_row(work, K, xq + t * K, &x_scale[t]);
+    }
+}
+
+/*
+ * INT8 x INT8 -> INT32 product of the quantised activations xq[T, K] and weights wq[N, K]
+ * (both stored with K contiguous): acc[t, n] = sum_k xq[t, k] * wq[n, k].
+ * [MIGRATE] section 7 ("INT8 x INT8 -> INT32 tensor-core operation"); [TAMING] flowchart
+ * "INT8 GEMM". Exact: |acc| <= K * 127^2 < 2^31 for K <= 133,000.
+ * Computed for the listed token rows and output columns only (all of them when the lists are
+ * null); acc is [nrows, ncols].
+ */
+void orc_gemm_s8(const int8_t *xq, int64_t T, const int8_t *wq, int64_t N, int64_t K,
+                 const int64_t *row_idx, int64_t nrows, const int64_t *col_idx, int64_t ncols,
+                 int32_t *acc)
+{
+    if (!row_idx) nrows = T;
+    if (!col_idx) ncols = N;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t t = row_idx ? row_idx[i] : i;
+        const int8_t *xr = xq + t * K;
+        for (int64_t c = 0; c < ncols; ++c) {
+            int64_t n = col_idx ? col_idx[c] : c;
+            const int8_t *wr = wq + n * K;
+            int32_t sum = 0;
+            for (int64_t k = 0; k < K; ++k) sum += (int32_t)xr[k] * (int32_t)wr[k];
+            acc[i * ncols + c] = sum;
+        }
+    }
+}
+
+/*
+ * Dequantisation epilogue, [MIGRATE] section 7 (Y = scale_x * scale_w * Y_int32) and the
+ * [TAMING] flowchart ("Add Bias & Dequantize"):
+ *   y[t, n] = bf16( float(acc) * (x_scale[t] * w_scale[n]) + bias[n] ),
+ * each operation rounded to binary32, the bias (bf16, optional) added last.
+ * acc is [nrows, ncols] for the listed rows / columns (all when the lists are null).
+ */
+void orc_dequant(const int32_t *acc, const float *x_scale, const float *w_scale,
+                 const uint16_t *bias, const int64_t *row_idx, int64_t nrows,
+                 const int64_t *col_idx, int64_t ncols, uint16_t *y)
+{
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t t = row_idx ? row_idx[i] : i;
+        for (int64_t c = 0; c < ncols; ++c) {
+            int64_t n = col_idx ? col_idx[c] : c;
+            float sc = x_scale[t] * w_scale[n];
+            float v = (float)acc[i * ncols + c] * sc;
+            if (bias) v = v + bf16_to_f32(bias[n]);
+            y[i * ncols + c] = f32_to_bf16_rne(v);
+        }
+    }
+}

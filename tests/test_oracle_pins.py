@@ -1,0 +1,341 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+Each test checks the oracle against something the pages or the mathematics fix: worked examples the
+pages print (fixtures under tests/golden, each with its source), closed forms at alpha = 0 and 1,
+invariants of the quantiser, independent library routines (numpy int64 matmul, numpy max, torch's
+bf16 rounding) and a rigorous error bound of the whole quantised chain against the exact fp64 product.
+The tests are chosen so that a plausible slip in the oracle (a transposed operand, a dropped term, the
+wrong exponent or tie rule, a wrong index) fails at least one of them.
+"""
+import numpy as np
+import pytest
+import torch
+
+from conftest import num, read_golden
+from post_quantization_calib_b200 import synth
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def bits_to_f64(h: np.ndarray) -> np.ndarray:
+    return (h.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def rand_bf16(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return bf16_bits((torch.randn(*shape, generator=g) * scale).to(torch.bfloat16))
+
+
+# --------------------------------------------------------------------------------------------
+# bf16 rounding: torch's CPU conversion is an independent implementation of round-to-nearest-even.
+
+def test_bf16_rounding_matches_torch(orc):
+    g = torch.Generator().manual_seed(1)
+    v = torch.randn(4000, generator=g, dtype=torch.float32) * 10.0 ** torch.randint(-6, 6, (4000,), generator=g)
+    # exact ties: low 16 bits == 0x8000, with even and odd kept parts
+    ties = np.array([0x3F808000, 0x3F818000, 0xBF808000, 0xBF818000, 0x7F7F8000], np.uint32).view(np.float32)
+    allv = np.concatenate([v.numpy(), ties, np.array([0.0, -0.0, 1e-40, np.inf, -np.inf], np.float32)])
+    ours = orc.f32_to_bf16(allv)
+    ref = bf16_bits(torch.from_numpy(allv).to(torch.bfloat16))
+    assert np.array_equal(ours, ref)
+
+
+# --------------------------------------------------------------------------------------------
+# Abs-max reductions ("06 -- SmoothQuant...", section 3; "Taming the Outliers...", System Architecture)
+
+def test_absmax_matches_numpy_bruteforce(orc):
+    a = rand_bf16((37, 48), 2, scale=3.0)
+    ref = np.abs(bits_to_f64(a)).max(axis=0).astype(np.float32)
+    assert np.array_equal(orc.calibrate_absmax(a), ref)
+
+
+def test_absmax_strided_rows_and_running_max(orc):
+    a = rand_bf16((20, 64), 3)
+    sub = np.ascontiguousarray(a)  # full buffer, reduce only the first 40 columns with ld = 64
+    rows, ld, cols = 20, 64, 40
+    amax = np.zeros(cols, np.float32)
+    orc.lib().orc_calibrate_absmax(sub.ctypes.data, rows, cols, ld, None, 1e-6, amax.ctypes.data, 0)
+    ref = np.abs(bits_to_f64(a[:, :cols])).max(axis=0)
+    assert np.array_equal(amax.astype(np.float64), ref)
+    # running max over two batches equals the max over their concatenation
+    b1, b2 = rand_bf16((9, 32), 4), rand_bf16((11, 32), 5, scale=2.0)
+    m = orc.calibrate_absmax(b1)
+    m = orc.calibrate_absmax(b2, amax=m, accumulate=True)
+    assert np.array_equal(m, orc.calibrate_absmax(np.concatenate([b1, b2])))
+
+
+def test_absmax_with_rmsnorm_against_fp64(orc):
+    # rows of small magnitude so that eps = 1e-6 changes the result by tens of percent:
+    # a dropped eps, a missing gamma or the mean over the wrong axis fails this.
+    x = rand_bf16((16, 256), 6, scale=1e-3)
+    gamma = (1.0 + 0.1 * np.random.default_rng(6).standard_normal(256)).astype(np.float32)
+    eps = 1e-6
+    got = orc.calibrate_absmax(x, norm_gamma=gamma, eps=eps).astype(np.float64)
+    xf = bits_to_f64(x)
+    y = xf / np.sqrt((xf ** 2).mean(axis=1, keepdims=True) + eps) * gamma.astype(np.float64)
+    ref = np.abs(y).max(axis=0)
+    assert np.allclose(got, ref, rtol=4e-7, atol=0)
+
+
+# --------------------------------------------------------------------------------------------
+# Smoothing factors: closed forms at the ends of the alpha range and the worked example.
+
+def test_alpha_one_closed_form(orc):
+    fx = read_golden("alpha_special_cases.txt")
+    assert num(fx["alpha_one_smoothed_channel_max"]) == 1.0
+    x = rand_bf16((64, 96), 7, scale=4.0)
+    ax = orc.calibrate_absmax(x)
+    aw = orc.calibrate_absmax(rand_bf16((80, 96), 8, scale=0.02))
+    s, fold = orc.compute_scales(ax, aw, 1.0)
+    assert np.array_equal(s, np.maximum(ax, np.float32(1e-5)))  # s_j = max|X_j|
+    # every smoothed activation channel then peaks at exactly 1 (x / s in binary32)
+    xs = bits_to_f64(x).astype(np.float32) / s[None, :]
+    assert np.array_equal(np.abs(xs).max(axis=0), np.ones(96, np.float32))
+    # and the folded reciprocal gives 1 to within one binary32 ulp
+    assert np.all(np.abs(np.abs(bits_to_f64(x).astype(np.float32) * fold).max(axis=0) - 1.0) <= 2.0 ** -23)
+
+
+def test_alpha_zero_closed_form(orc):
+    fx = read_golden("alpha_special_cases.txt")
+    assert num(fx["alpha_zero_smoothed_weight_max"]) == 1.0
+    ax = orc.calibrate_absmax(rand_bf16((64, 96), 9, scale=4.0))
+    w = rand_bf16((80, 96), 10, scale=0.02)
+    aw = orc.calibrate_absmax(w)
+    s, _ = orc.compute_scales(ax, aw, 0.0)
+    # s_j = 1 / max|W_j|: correctly rounded reciprocal of the weight maximum
+    ref = (1.0 / aw.astype(np.float64))
+    assert np.all(np.abs(s.astype(np.float64) / ref - 1.0) <= 2.0 ** -24)
+    # smoothed weight columns (diag(s) W) then peak at 1 within a binary32 ulp
+    wmax = np.abs(bits_to_f64(w).astype(np.float32) * s[None, :]).max(axis=0)
+    assert np.all(np.abs(wmax - 1.0) <= 2.0 ** -23)
+
+
+def test_worked_example_s25(orc):
+    fx = read_golden("outlier_channel_worked_example.txt")
+    ax = np.array([num(fx["channel_absmax"])], np.float32)
+    aw = np.array([num(fx["weight_absmax_derived"])], np.float32)
+    s, fold = orc.compute_scales(ax, aw, num(fx["alpha"]))
+    assert s[0] == np.float32(num(fx["s"]))
+    # the outlier channel's range [-50, 50] becomes [-2, 2] ...
+    chan = np.array([[-50.0], [50.0], [12.5]], np.float32)
+    sm = np.abs(chan / s[None, :]).max()
+    assert sm == num(fx["smoothed_absmax"])
+    # ... and a per-tensor INT8 scale drops from 50/127 to 2/127
+    assert np.isclose(50.0 / 127, num(fx["scale_before"])) and np.isclose(sm / 127, num(fx["scale_after"]))
+
+
+def test_scales_floor_and_fold(orc):
+    ax = np.array([0.0, 3.0, 7.5, 1e-9], np.float32)
+    aw = np.array([0.5, 0.0, 0.1, 0.2], np.float32)
+    gamma = np.array([1.1, 0.9, 1.0, 1.3], np.float32)
+    s, fold = orc.compute_scales(ax, aw, 0.5, gamma)
+    assert np.all(np.isfinite(s)) and np.all(s >= np.float32(1e-5))
+    # fold times s gives back gamma to within one rounding
+    assert np.allclose(fold.astype(np.float64) * s, gamma, rtol=2 ** -23, atol=0)
+    s2, fold2 = orc.compute_scales(ax, aw, 0.5, None)
+    assert np.array_equal(s, s2) and np.allclose(fold2.astype(np.float64) * s2, 1.0, rtol=2 ** -23)
+
+
+def test_scale_exponent_is_one_minus_alpha(orc):
+    # the variant with exponent alpha on the weight term would give s = (ax/aw)^alpha; at
+    # alpha = 0.25, ax = 16, aw = 1/16: 16^0.25 / (1/16)^0.75 = 2 * 8 = 16, whereas the variant
+    # gives (256)^0.25 = 4.
+    s, _ = orc.compute_scales(np.array([16.0], np.float32), np.array([1.0 / 16], np.float32), 0.25)
+    assert s[0] == 16.0
+
+
+# --------------------------------------------------------------------------------------------
+# Quantiser ("Taming the Outliers...", Why Outliers Break Quantization; tie rule: half away from 0)
+
+def test_quantiser_tie_rule_and_range(orc):
+    # one weight row with max 127 gives delta = 1 and 1/delta = 1 exactly, so the codes are the
+    # rounded values themselves: ties go away from zero (half-to-even would give 2, -2, 0, 0).
+    row = np.array([[2.5, -2.5, 0.5, -0.5, 1.5, 127.0, -126.5, 3.25]], np.float32)
+    wq, ws = orc.smooth_quantize_weight(bf16_bits(torch.from_numpy(row).to(torch.bfloat16)))
+    assert ws[0] == 1.0
+    assert wq[0].tolist() == [3, -3, 1, -1, 2, 127, -127, 3]
+    z, zs = orc.smooth_quantize_weight(np.zeros((2, 16), np.uint16))
+    assert np.all(z == 0) and np.all(zs == 0)
+
+
+def test_step_size_worked_example(orc):
+    fx = read_golden("step_size_example.txt")
+    for mkey, dkey, ckey in (("max_a", "delta_a", "code_a"), ("max_b", "delta_b", "code_b_arithmetic")):
+        row = torch.tensor([[num(fx[mkey]), num(fx["value"])]], dtype=torch.float32).to(torch.bfloat16)
+        wq, ws = orc.smooth_quantize_weight(bf16_bits(row))
+        # the page prints the step to three significant digits
+        assert abs(ws[0] - num(fx[dkey])) <= 1e-3 * num(fx[dkey])
+        assert wq[0, 0] == 127 and wq[0, 1] == int(num(fx[ckey]))
+
+
+def test_level_width_example(orc):
+    fx = read_golden("level_width_example.txt")
+    top = num(fx["tensor_max"])
+    vals = np.concatenate([[top], np.linspace(-num(fx["median_channel_max"]), num(fx["median_channel_max"]), 501)])
+    x = bf16_bits(torch.tensor(vals[None, :], dtype=torch.float32).to(torch.bfloat16))
+    xq, xs = orc.rmsnorm_smooth_quant(x, np.ones(x.shape[1], np.float32), apply_norm=False)
+    assert abs(2 * xs[0] * 127 / 255 - num(fx["level_width"])) < 0.005  # 255 levels over [-17.5, 17.5]
+    levels = np.unique(xq[0, 1:])
+    assert abs(len(levels) - num(fx["levels_about"])) <= 1
+
+
+def test_six_channel_example(orc):
+    fx = read_golden("six_channel_example.txt")
+    v = np.array([float(t) for t in fx["vector"].split()], np.float32)
+    j = int(num(fx["outlier_index_1based"])) - 1
+    s = np.ones_like(v)
+    s[j] = num(fx["s_outlier"])
+    x = bf16_bits(torch.from_numpy(v[None, :]).to(torch.bfloat16))
+    xq, xs = orc.rmsnorm_smooth_quant(x, (1.0 / s).astype(np.float32), apply_norm=False)
+    # after smoothing the outlier channel is the row maximum, about 1.2 (8.7 is 8.6875 in bf16)
+    assert xq[0, j] == 127
+    assert abs(xs[0] * 127 - num(fx["smoothed_outlier"])) < 0.01
+
+
+def test_quantiser_invariants_random(orc):
+    x = rand_bf16((33, 200), 11, scale=2.0)
+    fold = (0.5 + np.random.default_rng(11).random(200)).astype(np.float32)
+    xq, xs = orc.rmsnorm_smooth_quant(x, fold, apply_norm=False)
+    assert np.all(np.abs(xq).max(axis=1) == 127)            # the row maximum maps to +-127
+    y = bits_to_f64(x) * fold.astype(np.float64)
+    err = np.abs(xq * xs[:, None].astype(np.float64) - y)
+    assert np.all(err <= xs[:, None] * (0.5 + 2e-5) + 4 * 2.0 ** -24 * np.abs(y))
+    assert np.allclose(xs, np.abs(y).max(axis=1) / 127, rtol=3e-7, atol=0)
+
+
+def test_rmsnorm_constant_rows_and_scale_invariance(orc):
+    K = 128
+    x = np.zeros((3, K), np.float32)
+    x[0] = 0.75
+    x[1] = -3.0
+    x[2, ::2] = 2.0
+    x[2, 1::2] = -2.0
+    xb = bf16_bits(torch.from_numpy(x).to(torch.bfloat16))
+    xq, xs = orc.rmsnorm_smooth_quant(xb, np.ones(K, np.float32), eps=0.0, apply_norm=True)
+    assert np.all(xq[0] == 127) and np.all(xq[1] == -127)
+    assert np.all(xq[2, ::2] == 127) and np.all(xq[2, 1::2] == -127)
+    assert np.allclose(xs, 1.0 / 127, rtol=2e-7)
+    # doubling a row leaves its codes unchanged (RMSNorm is scale free; power-of-two scaling is exact)
+    r = rand_bf16((4, K), 12)
+    r2 = bf16_bits(torch.from_numpy(bits_to_f64(r).astype(np.float32) * 2).to(torch.bfloat16))
+    f = (1 + 0.1 * np.random.default_rng(12).standard_normal(K)).astype(np.float32)
+    assert np.array_equal(orc.rmsnorm_smooth_quant(r, f, eps=0.0)[0], orc.rmsnorm_smooth_quant(r2, f, eps=0.0)[0])
+
+
+# --------------------------------------------------------------------------------------------
+# INT8 GEMM ("06 -- SmoothQuant...", section 7): numpy int64 matmul is the independent check.
+
+def test_gemm_matches_numpy_int64(orc):
+    rng = np.random.default_rng(13)
+    xq = rng.integers(-127, 128, (29, 160), dtype=np.int8)
+    wq = rng.integers(-127, 128, (41, 160), dtype=np.int8)
+    ref = xq.astype(np.int64) @ wq.astype(np.int64).T
+    assert np.array_equal(orc.gemm_s8(xq, wq), ref)
+    rows, cols = np.array([28, 0, 5]), np.array([40, 3])
+    assert np.array_equal(orc.gemm_s8(xq, wq, rows, cols), ref[np.ix_(rows, cols)])
+
+
+def test_gemm_extreme_codes(orc):
+    K = 8192
+    xq = np.full((2, K), 127, np.int8)
+    xq[1] = -127
+    wq = np.full((3, K), -127, np.int8)
+    wq[1] = 127
+    wq[2, ::2] = 127
+    acc = orc.gemm_s8(xq, wq)
+    assert acc.tolist() == [[-K * 16129, K * 16129, 0], [K * 16129, -K * 16129, 0]]
+
+
+# --------------------------------------------------------------------------------------------
+# Dequant epilogue: against the exact fp64 value within one bf16 rounding.
+
+def test_dequant_against_fp64(orc):
+    rng = np.random.default_rng(14)
+    acc = rng.integers(-2 ** 27, 2 ** 27, (17, 23)).astype(np.int32)
+    xs = (rng.random(17) * 0.1).astype(np.float32)
+    ws = (rng.random(23) * 0.001).astype(np.float32)
+    bias = bf16_bits(torch.from_numpy(rng.standard_normal(23).astype(np.float32) * 0.02).to(torch.bfloat16))
+    y = bits_to_f64(orc.dequant(acc, xs, ws, bias))
+    ref = acc.astype(np.float64) * xs[:, None].astype(np.float64) * ws[None, :] + bits_to_f64(bias)[None, :]
+    assert np.all(np.abs(y - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6 * (np.abs(acc) * xs[:, None] * ws[None, :]) + 1e-30)
+    # zero accumulators give the bias exactly; no bias gives exact zeros
+    z = orc.dequant(np.zeros((2, 23), np.int32), xs[:2], ws, bias)
+    assert np.array_equal(z, np.broadcast_to(bias, (2, 23)))
+    assert np.all(bits_to_f64(orc.dequant(np.zeros((2, 23), np.int32), xs[:2], ws)) == 0)
+
+
+# --------------------------------------------------------------------------------------------
+# The whole chain: quantised smoothed linear vs the exact fp64 product, within the rigorous bound
+# implied by the two quantisers (half a step each, plus binary32 roundings). Also checks the
+# invariance Y = (X diag(s)^-1)(diag(s) W) that lets the smoothed product stand for X W.
+
+def _chain_bound_check(orc, x, w, gamma, bias, alpha, eps, apply_norm):
+    T, K = x.shape
+    ax = orc.calibrate_absmax(x, norm_gamma=gamma if apply_norm else None, eps=eps)
+    aw = orc.calibrate_absmax(w)
+    s, fold = orc.compute_scales(ax, aw, alpha, gamma if apply_norm else None)
+    wq, ws = orc.smooth_quantize_weight(w, s)
+    xq, xs = orc.rmsnorm_smooth_quant(x, fold, eps=eps, apply_norm=apply_norm)
+    y, acc = orc.w8a8_linear(xq, xs, wq, ws, bias)
+
+    xf, wf = bits_to_f64(x), bits_to_f64(w)
+    if apply_norm:
+        xin = xf / np.sqrt((xf ** 2).mean(axis=1, keepdims=True) + eps) * gamma.astype(np.float64)
+    else:
+        xin = xf
+    b = bits_to_f64(bias) if bias is not None else np.zeros(w.shape[0])
+    exact = xin @ wf.T + b
+    sd = s.astype(np.float64)
+    xhat, what = xin / sd, wf * sd            # smoothed operands in exact arithmetic
+    assert np.allclose(xhat @ what.T + b, exact, rtol=1e-12, atol=1e-12)   # invariance, fp64
+
+    ea = xs[:, None] * (0.5 + 2e-5) + 6 * 2.0 ** -24 * np.abs(xhat)     # [T, K]
+    eb = ws[:, None] * (0.5 + 2e-5) + 2 * 2.0 ** -24 * np.abs(what)     # [N, K]
+    bound = ea @ np.abs(what).T + np.abs(xhat) @ eb.T + ea @ eb.T
+    yq = acc.astype(np.float64) * xs[:, None] * ws[None, :] + b
+    assert np.all(np.abs(yq - exact) <= bound * (1 + 1e-9) + 1e-12)
+    yo = bits_to_f64(y)
+    assert np.all(np.abs(yo - yq) <= 2.0 ** -8 * np.abs(yq) + 1e-6 * np.abs(yq) + 1e-30)
+    return exact, yo
+
+
+def test_chain_error_bound_no_norm(orc):
+    w_ = synth.WORKLOADS[0]
+    K, N, T = 256, 96, 40
+    ch = synth.outlier_channels(K, synth.OutlierSpec(6, 50.0, 50.0), 21)
+    x = bf16_bits(synth.outlier_tokens(T, K, ch, 22))
+    w = bf16_bits(synth.normal_weight(N, K, 23))
+    bias = bf16_bits(synth.bias_vector(N, 24))
+    _chain_bound_check(orc, x, w, None, bias, w_.alpha, 1e-6, False)
+
+
+def test_chain_error_bound_with_norm(orc):
+    K, N, T = 256, 80, 33
+    ch = synth.outlier_channels(K, synth.OutlierSpec(5, 10.0, 100.0), 31)
+    x = bf16_bits(synth.outlier_tokens(T, K, ch, 32))
+    w = bf16_bits(synth.normal_weight(N, K, 33))
+    gamma = synth.norm_gamma(K, 34).numpy()
+    _chain_bound_check(orc, x, w, gamma, None, 0.5, 1e-6, True)
+
+
+def test_smoothing_reduces_error_on_outlier_data(orc):
+    # qualitative claim of the pages ("SmoothQuant and W8A8...", One layer, measured; the MSE
+    # comparison of "Taming the Outliers..."): on outlier-shaped data the smoothed W8A8 output is
+    # closer to the exact product than the unsmoothed one.
+    K, N, T = 512, 128, 64
+    ch = synth.outlier_channels(K, synth.OutlierSpec(16, 10.0, 25.0, pinned=25.0), 41)
+    x = bf16_bits(synth.outlier_tokens(T, K, ch, 42))
+    w = bf16_bits(synth.normal_weight(N, K, 43))
+    exact = bits_to_f64(x) @ bits_to_f64(w).T
+
+    def err(s):
+        fold = (1.0 / s).astype(np.float32) if s is not None else np.ones(K, np.float32)
+        wq, ws = orc.smooth_quantize_weight(w, s)
+        xq, xs = orc.rmsnorm_smooth_quant(x, fold, apply_norm=False)
+        y, _ = orc.w8a8_linear(xq, xs, wq, ws)
+        return np.linalg.norm(bits_to_f64(y) - exact) / np.linalg.norm(exact)
+
+    s, _ = orc.compute_scales(orc.calibrate_absmax(x), orc.calibrate_absmax(w), 0.5)
+    assert err(s) < 0.7 * err(None)
