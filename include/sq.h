@@ -1,0 +1,173 @@
+/*
+ * sq.h -- C ABI of libsq, the SmoothQuant smoothed W8A8 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer, as the pages describe it:
+ *   offline  per-input-channel abs-maxima of calibration activations and of the weight,
+ *            smoothing factors s_j = max|X_j|^alpha / max|W_j|^(1-alpha), the smoothed weight
+ *            diag(s) * W quantised to INT8 with one scale per output channel;
+ *   online   1/s folded into the preceding RMSNorm weight, per-token dynamic symmetric INT8
+ *            quantisation of the normalised activations, INT8 x INT8 -> INT32 GEMM, and a
+ *            dequantisation epilogue (per-token scale x per-channel scale, plus bias) to bf16.
+ *
+ * Pages cited (title, then section / equation / figure):
+ *   [MIGRATE] "06 -- SmoothQuant: Migrating Difficulty from Activations to Weights"
+ *   [TAMING]  "Taming the Outliers: A Deep Dive into SmoothQuant for LLM Quantization"
+ *   [W8A8]    "SmoothQuant and W8A8: Quantizing Activations Too"
+ *   [WOVS]    "SmoothQuant: Weight-Only vs W8A8"
+ *
+ * Conventions for every entry point
+ *   - Tensor pointers are caller-owned DEVICE memory on the current CUDA device. The library
+ *     allocates nothing and keeps no pointer after a call returns.
+ *   - Matrices are row-major. bf16 data is passed as `const void *` (IEEE bfloat16 bit patterns).
+ *     Sizes are element counts (int64_t).
+ *   - `stream` is a cudaStream_t passed as `void *` (NULL = the legacy default stream). Each call
+ *     enqueues its kernels on that stream and returns without synchronising; only
+ *     sq_device_status() synchronises.
+ *   - Outputs must not alias inputs.
+ *   - Arguments are validated before anything is launched; a failed check returns its code and
+ *     launches nothing. sq_last_error() then gives a one-line reason (per host thread).
+ *   - Arithmetic: binary32 with every operation separately rounded (no contraction into fused
+ *     multiply-adds), except the RMSNorm sum of squares (binary64) and the smoothing-factor power
+ *     (binary64, rounded once to binary32). INT8 codes use round-half-away-from-zero and are
+ *     clamped to [-127, 127].
+ */
+#ifndef SQ_H
+#define SQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SQ_OK = 0,
+    SQ_ERR_INVALID_ARG = 1,   /* null pointer, negative or inconsistent size, alpha outside [0,1] */
+    SQ_ERR_UNSUPPORTED = 2,   /* a size this build does not handle (limits stated per call) */
+    SQ_ERR_MISALIGNED = 3,    /* pointer or leading dimension not aligned as required */
+    SQ_ERR_ARCH = 4,          /* current device is not compute capability 10.0 (B200 class) */
+    SQ_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
+    SQ_ERR_TIMEOUT = 6        /* a bounded device-side wait ran out (reported by sq_device_status) */
+} sq_status;
+
+/* Name of a status code ("SQ_OK", ...). Never NULL. */
+const char *sq_status_string(int status);
+
+/* One-line reason for the last non-SQ_OK status returned on this host thread ("" if none). */
+const char *sq_last_error(void);
+
+/* Library version string. */
+const char *sq_version(void);
+
+/*
+ * Per-input-channel abs-max: amax[j] = max over rows r of |a[r, j]|.
+ *   [MIGRATE] section 3 "How to choose s" (max|X_j| from calibration samples);
+ *   [TAMING] "System Architecture" (flowchart nodes "Calculate max(|X|) per channel" and
+ *   "Calculate max(|W|) per channel").
+ * a          bf16 [rows, cols], row stride `ld` elements. For activations: calibration tokens x
+ *            channels. For a weight stored [N, K] (nn.Linear orientation), rows = N, cols = K gives
+ *            max|W_k| per input channel k.
+ * norm_gamma nullable fp32 [cols]. When given, each row is replaced by its RMSNorm output
+ *            (x / sqrt(mean(x^2) + eps)) * gamma before the reduction -- the input the linear
+ *            layer actually sees when it is fed by a norm ([W8A8] "The trick: move the range into
+ *            the weights").
+ * amax       fp32 [cols], in/out. accumulate = 0 overwrites it; accumulate = 1 keeps a running
+ *            maximum with its current contents (calibration streamed in batches).
+ * Requirements: rows >= 0, cols >= 8, cols % 8 == 0, ld % 8 == 0, ld >= cols, `a` 16-byte aligned,
+ * amax 4-byte aligned; with norm_gamma, cols <= 16384 (else SQ_ERR_UNSUPPORTED).
+ * rows == 0 with accumulate = 0 sets amax to 0.
+ */
+sq_status sq_calibrate_absmax(const void *a, int64_t rows, int64_t cols, int64_t ld,
+                              const float *norm_gamma, float eps, float *amax, int accumulate,
+                              void *stream);
+
+/*
+ * Smoothing factors and the folded norm weight.
+ *   [MIGRATE] section 3; [W8A8] "The trick: move the range into the weights" (formula and the
+ *   fold into the norm's weights); clamp of s from [TAMING] "Implementation in PyTorch".
+ *   s[j]    = max(fl32(pow(a_j, alpha) / pow(b_j, 1 - alpha)), 1e-5) with a_j = max(amax_x[j], 1e-5),
+ *             b_j = max(amax_w[j], 1e-5), the powers and the quotient in binary64.
+ *   fold[j] = gamma[j] / s[j]  (gamma non-null: the RMSNorm weight with 1/s folded in), or
+ *             1 / s[j]         (gamma null: a layer fed directly, x is multiplied by 1/s).
+ * amax_x, amax_w fp32 [K]; gamma nullable fp32 [K]; s fp32 [K] out; fold nullable fp32 [K] out.
+ * 0 <= alpha <= 1 (alpha = 1: s = max|X_j|; alpha = 0: s = 1/max|W_j|). K >= 1.
+ */
+sq_status sq_compute_scales(const float *amax_x, const float *amax_w, int64_t K, float alpha,
+                            const float *gamma, float *s, float *fold, void *stream);
+
+/*
+ * Smoothed weight, quantised to INT8 with one symmetric scale per output channel.
+ *   W_hat = diag(s) * W: [MIGRATE] section 2 and section 7 (one scale per output row);
+ *   [TAMING] "System Architecture" (nodes "Update Weights: W_hat = diag(s) * W", "Quantize W_hat").
+ *   w'[n,k] = w[n,k] * s[k]; m_n = max_k |w'[n,k]|; w_scale[n] = m_n / 127;
+ *   wq[n,k] = clamp(round_half_away(w'[n,k] * (127 / m_n)), -127, 127); a zero row gives scale 0.
+ * w bf16 [N, K]; s nullable fp32 [K] (null = unsmoothed); wq int8 [N, K] out; w_scale fp32 [N] out.
+ * Requirements: N >= 0, K >= 8, K % 8 == 0, K <= 16384, w 16-byte aligned, wq 8-byte aligned.
+ */
+sq_status sq_smooth_quantize_weight(const void *w, int64_t N, int64_t K, const float *s,
+                                    int8_t *wq, float *w_scale, void *stream);
+
+/*
+ * Online activation quantisation, fused with the RMSNorm that carries the folded 1/s.
+ *   [W8A8] "The trick: move the range into the weights" (1/s folded into the norm weight);
+ *   [MIGRATE] section 7 (X' INT8 with one scale per token); [W8A8] "The full model, served"
+ *   (a dynamic scale means finding each token's maximum before every matrix product).
+ *   apply_norm = 1: y[t,k] = (x[t,k] * inv_rms_t) * fold[k], inv_rms_t = 1 / sqrt(mean_k x^2 + eps)
+ *   apply_norm = 0: y[t,k] = x[t,k] * fold[k]            (fold = 1/s; eps ignored)
+ *   m_t = max_k |y[t,k]|; x_scale[t] = m_t / 127; xq[t,k] = clamp(round_half_away(y * (127/m_t)), +-127).
+ * x bf16 [T, K]; fold fp32 [K]; xq int8 [T, K] out; x_scale fp32 [T] out.
+ * Requirements: T >= 0, K >= 8, K % 8 == 0, K <= 16384, x 16-byte aligned, xq 8-byte aligned.
+ */
+sq_status sq_rmsnorm_smooth_quant(const void *x, int64_t T, int64_t K, const float *fold, float eps,
+                                  int apply_norm, int8_t *xq, float *x_scale, void *stream);
+
+/*
+ * W8A8 linear: INT8 x INT8 -> INT32 GEMM with the dequantisation fused into its epilogue.
+ *   [MIGRATE] section 7 ("a straight INT8 x INT8 -> INT32 tensor-core operation, followed by a
+ *   dequant Y = scale_x * scale_w * Y_int32"); [TAMING] "System Architecture" (nodes "INT8 GEMM",
+ *   "Add Bias & Dequantize").
+ *   acc[t,n] = sum_k xq[t,k] * wq[n,k]   (exact in int32)
+ *   y[t,n]   = bf16_rn( float(acc) * (x_scale[t] * w_scale[n]) + bias[n] )
+ * xq int8 [T, K]; x_scale fp32 [T]; wq int8 [N, K]; w_scale fp32 [N]; bias nullable bf16 [N];
+ * y bf16 [T, N] out; acc_out nullable int32 [T, N] out (raw accumulators, for verification).
+ * workspace / workspace_bytes: reserved; pass NULL / 0 (sq_w8a8_linear_workspace_size returns 0).
+ * Requirements: T >= 0, N >= 8, N % 8 == 0, K >= 16, K % 16 == 0, K <= 131072; xq, wq, y 16-byte
+ * aligned; acc_out 16-byte aligned. The GEMM runs on the tensor cores (tcgen05, TMEM accumulators,
+ * TMA-fed shared-memory pipeline); its device-side waits are bounded and report SQ_ERR_TIMEOUT
+ * through sq_device_status() instead of hanging.
+ */
+sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, const int8_t *wq,
+                         const float *w_scale, int64_t N, int64_t K, const void *bias, void *y,
+                         int32_t *acc_out, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace sq_w8a8_linear needs for these sizes (0 in this build). */
+size_t sq_w8a8_linear_workspace_size(int64_t T, int64_t N, int64_t K);
+
+/*
+ * Synchronises `stream`, then reports the device-side status word of the current device:
+ * SQ_OK, SQ_ERR_TIMEOUT (a bounded wait in a kernel ran out; the kernel stopped its work and
+ * returned, the context stays usable) or SQ_ERR_CUDA (an asynchronous CUDA error). Reading the
+ * word clears it. The word is shared by every stream on the device.
+ */
+sq_status sq_device_status(void *stream);
+
+/*
+ * Sets the limit, in nanoseconds, of every bounded device-side wait launched afterwards on the
+ * current device (default 2e9 = 2 s). Values below 1000 are raised to 1000.
+ */
+sq_status sq_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * Self-test of the timeout path: launches one small kernel whose thread waits, with the bounded
+ * wait the GEMM uses, on a shared-memory barrier that nothing ever completes. The wait runs out
+ * after the configured limit, the kernel records SQ_ERR_TIMEOUT in the status word and returns.
+ * Used by the test suite to show that an expired wait ends in a status, not a hang.
+ */
+sq_status sq_selftest_wait_timeout(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_H */

@@ -1,0 +1,539 @@
+// sq_gemm.cu -- W8A8 linear on the sm_100a tensor cores: INT8 x INT8 -> INT32 with the
+// dequantisation (per-token scale x per-output-channel scale, plus bias) fused into the epilogue.
+//
+// Pages cited (title, then section / equation / figure):
+//   [MIGRATE] "06 -- SmoothQuant: Migrating Difficulty from Activations to Weights", section 7
+//             ("Bit-level and kernel-level realities": INT8 x INT8 -> INT32 followed by
+//             Y = scale_x * scale_w * Y_int32)
+//   [TAMING]  "Taming the Outliers: A Deep Dive into SmoothQuant for LLM Quantization",
+//             "System Architecture" (flowchart nodes "INT8 GEMM" and "Add Bias & Dequantize")
+//
+// The pages name the operation, not a kernel design (their INT8 kernels target earlier tensor-core
+// generations). This kernel is written for B200:
+//   * persistent: one CTA per SM (the shared-memory footprint admits exactly one), tiles
+//     128 tokens x 256 output channels handed out round-robin in bands of M tiles for L2 reuse;
+//   * warp 0 (one lane) streams 128-byte K slices of both operands into a 4-stage shared-memory
+//     ring with TMA (128-byte swizzle), completion tracked by mbarrier transaction counts;
+//   * warp 1 (one lane) issues tcgen05.mma.kind::i8 (M=128, N=256, K=32, signed x signed -> s32)
+//     into a tensor-memory accumulator; two accumulators of 256 columns alternate so the epilogue
+//     of one tile overlaps the main loop of the next;
+//   * warps 2..5 read the accumulator with tcgen05.ld (each warp its own 32-lane quarter), apply
+//     y = bf16(float(acc) * (x_scale * w_scale) + bias) in binary32 with explicit rounding, stage
+//     64-column boxes in swizzled shared memory and write them with TMA stores (the TMA clips rows
+//     beyond T and columns beyond N).
+// Every mbarrier wait is bounded by a wall-clock limit (%globaltimer). When one runs out, the
+// kernel records SQ_ERR_TIMEOUT in a device status word, every role leaves its loop, in-flight
+// copies and MMAs are waited for (again with a limit), tensor memory is released and the kernel
+// returns. No wait can hang the GPU.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sq_internal.h"
+
+namespace {
+
+// Device-side status word: 0 or the first sq_status a kernel recorded.
+__device__ unsigned int g_sq_status;
+
+constexpr int BM = 128;            // tokens per tile (MMA M)
+constexpr int BN = 256;            // output channels per tile (MMA N)
+constexpr int BK = 128;            // K bytes per pipeline stage (one 128-byte swizzle row)
+constexpr int UMMA_K = 32;         // K per tcgen05.mma.kind::i8
+constexpr int STAGES = 4;
+constexpr int A_STAGE = BM * BK;   // 16 KB
+constexpr int B_STAGE = BN * BK;   // 32 KB
+constexpr int EPI_WARPS = 4;
+constexpr int OUT_COLS = 64;       // bf16 columns per TMA store box (128 bytes)
+constexpr int OUT_ROWS = 32;       // rows per box: one warp's TMEM lane quarter
+constexpr int OUT_BOX = OUT_COLS * 2 * OUT_ROWS;
+constexpr int THREADS = 64 + 32 * EPI_WARPS;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int BAND = 16;           // M tiles per raster band
+
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
+constexpr int OFF_OUT = OFF_B + STAGES * B_STAGE;
+constexpr int OFF_BAR = OFF_OUT + EPI_WARPS * 2 * OUT_BOX;
+constexpr int NBARS = 2 * STAGES + 5;   // full[S], empty[S], tfull[2], tempty[2], done
+constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+constexpr int SMEM_USED = OFF_MISC + 16;
+constexpr int SMEM_TOTAL = SMEM_USED + 1024;    // slack to align the base to 1024 bytes
+static_assert(SMEM_TOTAL <= 232448, "shared memory budget of one sm_100 CTA");
+
+// Instruction descriptor of tcgen05.mma.kind::i8: D = s32, A and B signed 8-bit, both K-major,
+// N >> 3 at bits 17..22, M >> 4 at bits 24..28.
+constexpr uint32_t make_idesc(int M, int N) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+constexpr uint32_t IDESC = make_idesc(BM, BN);
+
+// ------------------------------------------------------------------------------------------------
+// PTX wrappers.
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void record_status(unsigned int code) { atomicCAS(&g_sq_status, 0u, code); }
+
+// Waits until the phase of `bar` with parity `parity` has completed. Returns false when
+// `limit_ns` elapsed first or (when `abort_flag` is given) another role of the CTA gave up.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                       const volatile int *abort_flag) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try(bar, parity)) return true;
+        if ((i & 127u) == 0u) {
+            if (abort_flag && *abort_flag) return false;
+            if (global_ns() - t0 > limit_ns) return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void give_up(volatile int *abort_flag) {
+    record_status(SQ_ERR_TIMEOUT);
+    *abort_flag = 1;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void prefetch_map(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory descriptor of a K-major operand tile written by TMA with the 128-byte swizzle:
+// rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), leading byte offset 1
+// (unused for swizzled K-major layouts), descriptor version 1, layout type 2 (128-byte swizzle).
+__device__ __forceinline__ uint64_t kmajor_sw128_desc(uint32_t saddr) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1u) << 16) |
+           (static_cast<uint64_t>(1024u >> 4) << 32) | (static_cast<uint64_t>(1u) << 46) |
+           (static_cast<uint64_t>(2u) << 61);
+}
+
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int &m, int &n) {
+    const int per_band = BAND * n_tiles;
+    const int band = t / per_band;
+    const int within = t - band * per_band;
+    const int bs = min(BAND, m_tiles - band * BAND);
+    n = within / bs;
+    m = band * BAND + (within - n * bs);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// ------------------------------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(THREADS, 1)
+k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmY, const float *__restrict__ x_scale,
+              const float *__restrict__ w_scale, const __nv_bfloat16 *__restrict__ bias,
+              int32_t *__restrict__ acc_out, int T, int N, int K, int m_tiles, int n_tiles,
+              uint64_t limit_ns)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem + OFF_A;
+    uint8_t *sB = smem + OFF_B;
+    uint8_t *sOut = smem + OFF_OUT;
+    const uint32_t bar0 = smem_u32(smem + OFF_BAR);
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+    auto tfull = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
+    auto tempty = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
+    const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) { mbar_init(full(s), 1); mbar_init(empty(s), 1); }
+        for (int b = 0; b < 2; ++b) { mbar_init(tfull(b), 1); mbar_init(tempty(b), 32 * EPI_WARPS); }
+        mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_async_smem();
+    }
+    if (warp == 0 && lane == 0) { prefetch_map(&tmA); prefetch_map(&tmB); prefetch_map(&tmY); }
+    if (warp == 1) { tmem_alloc(smem_u32(tmem_slot), TMEM_COLS); tmem_relinquish(); }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int k_blocks = (K + BK - 1) / BK;
+    const int num_tiles = m_tiles * n_tiles;
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long fills = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+                int m, n;
+                tile_coords(t, m_tiles, n_tiles, m, n);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait(empty(stage), phase ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
+                    mbar_expect_tx(full(stage), A_STAGE + B_STAGE);
+                    tma_load_2d(smem_u32(sA + stage * A_STAGE), &tmA, full(stage), kb * BK, m * BM);
+                    tma_load_2d(smem_u32(sB + stage * B_STAGE), &tmB, full(stage), kb * BK, n * BN);
+                    ++fills;
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok) give_up(abort_flag);
+            // Wait for the last fill of every stage to land, so no copy is in flight at exit.
+            for (int s = 0; s < STAGES; ++s) {
+                if (fills <= s) break;
+                const long long last = s + ((fills - 1 - s) / STAGES) * STAGES;
+                if (!mbar_wait(full(s), static_cast<uint32_t>((last / STAGES) & 1), limit_ns, nullptr))
+                    record_status(SQ_ERR_TIMEOUT);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            bool issued = false;
+            int lt = 0;
+            for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++lt) {
+                const int buf = lt & 1;
+                const uint32_t use = static_cast<uint32_t>(lt >> 1);
+                if (!mbar_wait(tempty(buf), (use & 1u) ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait(full(stage), phase, limit_ns, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * A_STAGE);
+                    const uint32_t b0 = smem_u32(sB + stage * B_STAGE);
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                        mma_i8(d_tmem, kmajor_sw128_desc(a0 + kk * UMMA_K), kmajor_sw128_desc(b0 + kk * UMMA_K), IDESC,
+                               (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    issued = true;
+                    tc_commit(empty(stage));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit(tfull(buf));
+            }
+            if (!ok) give_up(abort_flag);
+            // Every MMA issued above has completed once this commit's barrier flips.
+            if (issued) {
+                tc_commit(done_bar);
+                if (!mbar_wait(done_bar, 0, limit_ns, nullptr)) record_status(SQ_ERR_TIMEOUT);
+            }
+        }
+    } else {
+        // ---------------- epilogue ----------------
+        const int quad = warp & 3;                  // TMEM lanes this warp may read: 32*quad .. +31
+        uint8_t *stage_buf = sOut + (warp - 2) * 2 * OUT_BOX;
+        int nstores = 0;
+        int lt = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++lt) {
+            const int buf = lt & 1;
+            const uint32_t use = static_cast<uint32_t>(lt >> 1);
+            if (!mbar_wait(tfull(buf), use & 1u, limit_ns, abort_flag)) { give_up(abort_flag); break; }
+            tc_fence_after();
+            int m, n;
+            tile_coords(t, m_tiles, n_tiles, m, n);
+            const int row0 = m * BM + quad * 32;     // first token row of this warp's quarter
+            const int row = row0 + lane;
+            if (row0 < T) {
+                const float xs = row < T ? __ldg(x_scale + row) : 0.0f;
+                for (int c = 0; c < BN / OUT_COLS; ++c) {
+                    const int col0 = n * BN + c * OUT_COLS;
+                    if (col0 >= N) break;
+                    uint32_t r[2][32];
+                    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                                           static_cast<uint32_t>(buf * BN + c * OUT_COLS);
+                    tmem_ld32(taddr, r[0]);
+                    tmem_ld32(taddr + 32, r[1]);
+                    tmem_ld_wait();
+                    if (acc_out != nullptr && row < T) {
+                        int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + col0);
+#pragma unroll
+                        for (int g = 0; g < OUT_COLS / 4; ++g) {
+                            if (col0 + 4 * g < N)
+                                dst[g] = make_int4(static_cast<int>(r[g >> 3][(4 * g) & 31]), static_cast<int>(r[g >> 3][(4 * g + 1) & 31]),
+                                                   static_cast<int>(r[g >> 3][(4 * g + 2) & 31]), static_cast<int>(r[g >> 3][(4 * g + 3) & 31]));
+                        }
+                    }
+                    // y = bf16(float(acc) * (x_scale * w_scale) + bias), eight columns per 16-byte chunk
+                    uint32_t packed[OUT_COLS / 2];
+#pragma unroll
+                    for (int g = 0; g < OUT_COLS / 4; ++g) {
+                        const int col = col0 + 4 * g;
+                        float4 ws = make_float4(0.f, 0.f, 0.f, 0.f);
+                        float b4[4] = {0.f, 0.f, 0.f, 0.f};
+                        if (col < N) {
+                            ws = __ldg(reinterpret_cast<const float4 *>(w_scale + col));
+                            if (bias != nullptr) {
+                                const uint2 bb = __ldg(reinterpret_cast<const uint2 *>(bias + col));
+                                b4[0] = __uint_as_float(bb.x << 16);
+                                b4[1] = __uint_as_float(bb.x & 0xFFFF0000u);
+                                b4[2] = __uint_as_float(bb.y << 16);
+                                b4[3] = __uint_as_float(bb.y & 0xFFFF0000u);
+                            }
+                        }
+                        const float wsv[4] = {ws.x, ws.y, ws.z, ws.w};
+                        float v[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = 4 * g + e;
+                            const float acc = __int2float_rn(static_cast<int>(r[j >> 5][j & 31]));
+                            v[e] = __fmul_rn(acc, __fmul_rn(xs, wsv[e]));
+                            if (bias != nullptr) v[e] = __fadd_rn(v[e], b4[e]);
+                        }
+                        packed[2 * g] = pack_bf16x2(v[0], v[1]);
+                        packed[2 * g + 1] = pack_bf16x2(v[2], v[3]);
+                    }
+                    // stage the 32 x 64 box in 128-byte-swizzled layout, then one TMA store
+                    uint8_t *sb = stage_buf + (nstores & 1) * OUT_BOX;
+                    if (lane == 0) bulk_wait_read_1();
+                    __syncwarp();
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int pos = q ^ (lane & 7);
+                        *reinterpret_cast<uint4 *>(sb + lane * 128 + pos * 16) =
+                            make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                    }
+                    fence_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmY, smem_u32(sb), col0, row0);
+                        bulk_commit();
+                    }
+                    ++nstores;
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(tempty(buf));
+        }
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// One thread waits, with the same bounded wait as the GEMM, on a barrier nothing completes.
+__global__ void k_selftest_wait(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        abort_flag = 0;
+        mbar_init(smem_u32(&bar), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        if (!mbar_wait(smem_u32(&bar), 0, limit_ns, &abort_flag)) record_status(SQ_ERR_TIMEOUT);
+    }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Host side.
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+sq_status get_encoder(EncodeTiledFn *out) {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+        if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
+            return sq::fail(SQ_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    *out = fn;
+    return SQ_OK;
+}
+
+sq_status encode_2d(EncodeTiledFn enc, CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
+                    uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, const char *what) {
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return sq::fail(SQ_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with CUresult %d", what, (int)r);
+    return SQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, const int8_t *wq,
+                         const float *w_scale, int64_t N, int64_t K, const void *bias, void *y,
+                         int32_t *acc_out, void *workspace, size_t workspace_bytes, void *stream)
+{
+    using sq::fail;
+    (void)workspace;
+    (void)workspace_bytes;
+    if (T < 0 || N < 8 || K < 16) return fail(SQ_ERR_INVALID_ARG, "sq_w8a8_linear: need T >= 0, N >= 8, K >= 16");
+    if (!wq || !w_scale) return fail(SQ_ERR_INVALID_ARG, "sq_w8a8_linear: wq and w_scale are required");
+    if (T > 0 && (!xq || !x_scale || !y)) return fail(SQ_ERR_INVALID_ARG, "sq_w8a8_linear: xq, x_scale and y are required");
+    if (N % 8 != 0 || K % 16 != 0) return fail(SQ_ERR_MISALIGNED, "sq_w8a8_linear: N must be a multiple of 8 and K of 16");
+    if (K > 131072 || N > 0x7FFFFFFF || T > 0x7FFFFFFF)
+        return fail(SQ_ERR_UNSUPPORTED, "sq_w8a8_linear: K must be <= 131072 and T, N < 2^31");
+    if ((xq && !sq::aligned(xq, 16)) || !sq::aligned(wq, 16) || (y && !sq::aligned(y, 16)) ||
+        (acc_out && !sq::aligned(acc_out, 16)) || !sq::aligned(w_scale, 16) || (x_scale && !sq::aligned(x_scale, 4)) ||
+        (bias && !sq::aligned(bias, 8)))
+        return fail(SQ_ERR_MISALIGNED, "sq_w8a8_linear: xq, wq, y, acc_out, w_scale need 16-byte, bias 8-byte, x_scale 4-byte alignment");
+    int dev = 0;
+    SQ_TRY_ARCH(dev);
+    if (T == 0) return SQ_OK;
+
+    EncodeTiledFn enc = nullptr;
+    sq_status st = get_encoder(&enc);
+    if (st != SQ_OK) return st;
+    CUtensorMap mA, mB, mY;
+    st = encode_2d(enc, &mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, T, K, BK, BM, "xq");
+    if (st == SQ_OK) st = encode_2d(enc, &mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, K, N, K, BK, BN, "wq");
+    if (st == SQ_OK) st = encode_2d(enc, &mY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, T, N * 2, OUT_COLS, OUT_ROWS, "y");
+    if (st != SQ_OK) return st;
+
+    static int configured[64];
+    if (!configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k_w8a8_linear, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TOTAL);
+        if (e != cudaSuccess) return sq::cuda_status(e, "cudaFuncSetAttribute(w8a8_linear)");
+        configured[dev] = 1;
+    }
+    const int m_tiles = static_cast<int>((T + BM - 1) / BM);
+    const int n_tiles = static_cast<int>((N + BN - 1) / BN);
+    const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
+    if (tiles > 0x7FFFFFFF) return fail(SQ_ERR_UNSUPPORTED, "sq_w8a8_linear: too many tiles");
+    const int grid = static_cast<int>(tiles < sq::sm_count(dev) ? tiles : sq::sm_count(dev));
+    k_w8a8_linear<<<grid, THREADS, SMEM_TOTAL, sq::as_stream(stream)>>>(
+        mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out, static_cast<int>(T),
+        static_cast<int>(N), static_cast<int>(K), m_tiles, n_tiles, sq::wait_timeout_ns(dev));
+    return sq::cuda_status(cudaGetLastError(), "launch(w8a8_linear)");
+}
+
+size_t sq_w8a8_linear_workspace_size(int64_t T, int64_t N, int64_t K) {
+    (void)T;
+    (void)N;
+    (void)K;
+    return 0;
+}
+
+sq_status sq_device_status(void *stream) {
+    int dev = 0;
+    SQ_TRY_ARCH(dev);
+    cudaError_t e = cudaStreamSynchronize(sq::as_stream(stream));
+    if (e != cudaSuccess) return sq::cuda_status(e, "cudaStreamSynchronize");
+    unsigned int word = 0;
+    e = cudaMemcpyFromSymbol(&word, g_sq_status, sizeof word);
+    if (e != cudaSuccess) return sq::cuda_status(e, "cudaMemcpyFromSymbol(status)");
+    if (word != 0) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_sq_status, &zero, sizeof zero);
+        if (e != cudaSuccess) return sq::cuda_status(e, "cudaMemcpyToSymbol(status)");
+        return sq::fail(static_cast<sq_status>(word), "device status word reported %s", sq_status_string(static_cast<int>(word)));
+    }
+    return SQ_OK;
+}
+
+sq_status sq_selftest_wait_timeout(void *stream) {
+    int dev = 0;
+    SQ_TRY_ARCH(dev);
+    k_selftest_wait<<<1, 32, 0, sq::as_stream(stream)>>>(sq::wait_timeout_ns(dev));
+    return sq::cuda_status(cudaGetLastError(), "launch(selftest_wait)");
+}
+
+}  // extern "C"

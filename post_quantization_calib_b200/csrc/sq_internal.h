@@ -1,0 +1,36 @@
+// sq_internal.h -- host-side helpers shared by the libsq translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sq.h"
+
+namespace sq {
+
+// Records a one-line reason for `st` (thread-local) and returns st.
+sq_status fail(sq_status st, const char *fmt, ...);
+
+// Checks that the current device is compute capability 10.0; caches per device.
+sq_status check_arch(int *device_out = nullptr);
+
+// SM count of the current device (cached).
+int sm_count(int device);
+
+// cudaError_t -> SQ_OK / SQ_ERR_CUDA with the CUDA error text recorded.
+sq_status cuda_status(cudaError_t e, const char *what);
+
+// Per-device limit of bounded device-side waits, in ns.
+uint64_t wait_timeout_ns(int device);
+void set_wait_timeout_ns(int device, uint64_t ns);
+
+inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+}  // namespace sq
+
+#define SQ_TRY_ARCH(dev)                        \
+    do {                                        \
+        sq_status _st = sq::check_arch(&(dev)); \
+        if (_st != SQ_OK) return _st;           \
+    } while (0)

@@ -44,7 +44,7 @@ class Workload:
     index: int
     T: int                      # online tokens
     K: int                      # input channels (hidden size)
-    Ns: Tuple[int, ...]         # output widths of the projections sharing one smoothing factor
+    Ns: Tuple[int, ...]         # output width of each smoothing group's fused GEMM
     calib_rows: int             # calibration tokens in total
     calib_chunk: int            # calibration tokens per streamed chunk
     alpha: float
@@ -57,11 +57,16 @@ class Workload:
 
     @property
     def N(self) -> int:
+        """Output channels over all smoothing groups."""
         return int(sum(self.Ns))
 
-    def linear_ops(self) -> int:
-        """Integer multiply-adds x 2 of the group's GEMMs at T tokens."""
-        return 2 * self.T * self.N * self.K
+    def group_N(self, g: int) -> int:
+        """Output channels of smoothing group g (one fused GEMM per group)."""
+        return int(self.Ns[g])
+
+    def linear_ops(self, T: Optional[int] = None) -> int:
+        """2 x multiply-adds of all the workload's GEMMs at T tokens (default: the workload's T)."""
+        return 2 * (self.T if T is None else T) * self.N * self.K
 
 
 def _w(name, index, **kw) -> Workload:
@@ -174,3 +179,21 @@ def split_rows(total: int, parts: int) -> Sequence[Tuple[int, int]]:
         out.append((start, start + n))
         start += n
     return out
+
+
+def group_inputs(w: Workload, g: int = 0, device="cpu", T: Optional[int] = None, rank: int = 0) -> dict:
+    """All seeded tensors of smoothing group ``g`` of workload ``w``.
+
+    Returns a dict with ``channels`` (outlier indices, factors), ``gamma`` (fp32 [K] or None),
+    ``weight`` (bf16 [N_g, K]), ``bias`` (bf16 [N_g] or None) and ``x`` (bf16 [T, K] online tokens;
+    each rank draws its own tokens). Calibration tokens come from ``calibration_chunks``.
+    """
+    K, N = w.K, w.group_N(g)
+    ch = outlier_channels(K, w.outliers, seed_for(w.index, "outliers", g))
+    return {
+        "channels": ch,
+        "gamma": norm_gamma(K, seed_for(w.index, "gamma", g), device) if w.norm else None,
+        "weight": normal_weight(N, K, seed_for(w.index, "w", g), device),
+        "bias": bias_vector(N, seed_for(w.index, "bias", g), device) if w.bias else None,
+        "x": outlier_tokens(w.T if T is None else T, K, ch, seed_for(w.index, "x", g, rank), device),
+    }
