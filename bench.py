@@ -316,7 +316,7 @@ def main_gpu(args, rank, local_rank, world):
     W_h = W.cpu().pin_memory()
     X_h = X.cpu().pin_memory()
     y_h = torch.empty(T, N, dtype=torch.bfloat16).pin_memory()
-    e2e_steps = max(2, min(args.steps, 20))
+    e2e_steps = 0 if args.no_e2e else max(2, min(args.steps, 20))
 
     def e2e_step():
         calib.copy_(calib_h, non_blocking=True)
@@ -325,7 +325,8 @@ def main_gpu(args, rank, local_rank, world):
         step()
         y_h.copy_(y, non_blocking=True)
 
-    e2e_step()
+    if e2e_steps:
+        e2e_step()
     barrier()
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
@@ -335,7 +336,7 @@ def main_gpu(args, rank, local_rank, world):
         e2e_step()
     b.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(b) / e2e_steps
+    e2e_ms = a.elapsed_time(b) / e2e_steps if e2e_steps else float("nan")
     te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
@@ -419,6 +420,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the timed CPU oracle sample")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     args = ap.parse_args()
     rank, local_rank, world = sqdist.env_rank()
     if world != args.gpus and world == 1 and args.gpus > 1:
