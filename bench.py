@@ -57,13 +57,14 @@ def src_sha(name: str) -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str, source: str):
-    """DRAM bytes per launch from a committed ncu summary, if taken on the current kernel source."""
+def recorded_traffic(stage: str, source: str):
+    """DRAM bytes per launch of a stage's kernel from a committed ncu summary, if the counters were
+    taken on the current kernel source (else None)."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        d = json.load(f).get(kernel)
+        d = json.load(f).get(stage)
     if not d or d.get("source_sha") != src_sha(source):
         return None
     return d.get("bytes_per_launch")
@@ -129,9 +130,9 @@ def stage_work(w, T, N, K, calib_rows):
     }
 
 
-KERNEL_OF = {"calib_absmax": ("k_absmax", "sq_rowwise.cu"), "weight_absmax": ("k_absmax", "sq_rowwise.cu"),
-             "scales": ("k_scales", "sq_rowwise.cu"), "weight_quant": ("k_rowquant", "sq_rowwise.cu"),
-             "act_quant": ("k_rowquant", "sq_rowwise.cu"), "gemm": ("k_w8a8_linear", "sq_gemm.cu")}
+KERNEL_OF = {"calib_absmax": ("k_rows<ABSMAX,NORM>", "sq_rowwise.cu"), "weight_absmax": ("k_rows<ABSMAX>", "sq_rowwise.cu"),
+             "scales": ("k_scales", "sq_rowwise.cu"), "weight_quant": ("k_rows<QUANT>", "sq_rowwise.cu"),
+             "act_quant": ("k_rows<QUANT,NORM>", "sq_rowwise.cu"), "gemm": ("k_w8a8_linear", "sq_gemm.cu")}
 LAUNCHES = {"calib_absmax": 2, "weight_absmax": 2, "scales": 1, "weight_quant": 1, "act_quant": 1, "gemm": 1}
 
 
@@ -312,11 +313,10 @@ def main_gpu(args, rank, local_rank, world):
     value = world * w.linear_ops() * args.steps / (elapsed_ms * 1e-3) / 1e12
 
     # ---- end to end through the C ABI with host buffers: pinned H2D of this step's inputs, D2H of y
-    calib_h = calib.cpu().pin_memory()
-    W_h = W.cpu().pin_memory()
-    X_h = X.cpu().pin_memory()
-    y_h = torch.empty(T, N, dtype=torch.bfloat16).pin_memory()
     e2e_steps = 0 if args.no_e2e else max(2, min(args.steps, 20))
+    pin = (lambda t: t.cpu().pin_memory()) if e2e_steps else (lambda t: t.cpu()[:0])
+    calib_h, W_h, X_h = pin(calib), pin(W), pin(X)
+    y_h = torch.empty(T, N, dtype=torch.bfloat16).pin_memory() if e2e_steps else torch.empty(0)
 
     def e2e_step():
         calib.copy_(calib_h, non_blocking=True)
@@ -341,8 +341,8 @@ def main_gpu(args, rank, local_rank, world):
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
     e2e_ms = float(te.item())
-    h2d = calib_h.numel() * 2 + W_h.numel() * 2 + X_h.numel() * 2
-    d2h = y_h.numel() * 2
+    h2d = (calib.numel() + W.numel() + X.numel()) * 2 if e2e_steps else 0
+    d2h = y.numel() * 2 if e2e_steps else 0
 
     if world > 1:
         dist.barrier()
@@ -375,7 +375,7 @@ def main_gpu(args, rank, local_rank, world):
         roof = {"bound": "hbm", "achieved": stages[dom]["gbs"], "peak": hbm, "unit": "GB/s",
                 "frac": stages[dom]["gbs"] / hbm}
         peak_note = f"HBM peak = {src} copy bandwidth"
-    roof["traffic"] = recorded_traffic(kern, srcfile)
+    roof["traffic"] = recorded_traffic(dom, srcfile)
     roof["kernel"] = kern
     roof["stage"] = dom
     roof["peak_source"] = peak_note

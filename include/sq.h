@@ -63,8 +63,7 @@ const char *sq_version(void);
 /*
  * Per-input-channel abs-max: amax[j] = max over rows r of |a[r, j]|.
  *   [MIGRATE] section 3 "How to choose s" (max|X_j| from calibration samples);
- *   [TAMING] "System Architecture" (flowchart nodes "Calculate max(|X|) per channel" and
- *   "Calculate max(|W|) per channel").
+ *   [TAMING] "System Architecture" (the flowchart's per-channel maximum of |X| and of |W|).
  * a          bf16 [rows, cols], row stride `ld` elements. For activations: calibration tokens x
  *            channels. For a weight stored [N, K] (nn.Linear orientation), rows = N, cols = K gives
  *            max|W_k| per input channel k.
@@ -74,9 +73,10 @@ const char *sq_version(void);
  *            the weights").
  * amax       fp32 [cols], in/out. accumulate = 0 overwrites it; accumulate = 1 keeps a running
  *            maximum with its current contents (calibration streamed in batches).
- * Requirements: rows >= 0, cols >= 8, cols % 8 == 0, ld % 8 == 0, ld >= cols, `a` 16-byte aligned,
- * amax 4-byte aligned; with norm_gamma, cols <= 16384 (else SQ_ERR_UNSUPPORTED).
- * rows == 0 with accumulate = 0 sets amax to 0.
+ * Requirements: rows >= 0, 8 <= cols <= 16384 (else SQ_ERR_UNSUPPORTED), cols % 8 == 0, ld % 8 == 0,
+ * ld >= cols, `a` and norm_gamma 16-byte aligned, amax 4-byte aligned.
+ * rows == 0 with accumulate = 0 sets amax to 0. With norm_gamma, rows whose values all lie below
+ * 2^-100 in magnitude (or contain subnormal bf16) may see the inexact squares of those values.
  */
 sq_status sq_calibrate_absmax(const void *a, int64_t rows, int64_t cols, int64_t ld,
                               const float *norm_gamma, float eps, float *amax, int accumulate,
@@ -99,7 +99,7 @@ sq_status sq_compute_scales(const float *amax_x, const float *amax_w, int64_t K,
 /*
  * Smoothed weight, quantised to INT8 with one symmetric scale per output channel.
  *   W_hat = diag(s) * W: [MIGRATE] section 2 and section 7 (one scale per output row);
- *   [TAMING] "System Architecture" (nodes "Update Weights: W_hat = diag(s) * W", "Quantize W_hat").
+ *   [TAMING] "System Architecture" (the flowchart's weight-update and weight-quantisation nodes).
  *   w'[n,k] = w[n,k] * s[k]; m_n = max_k |w'[n,k]|; w_scale[n] = m_n / 127;
  *   wq[n,k] = clamp(round_half_away(w'[n,k] * (127 / m_n)), -127, 127); a zero row gives scale 0.
  * w bf16 [N, K]; s nullable fp32 [K] (null = unsmoothed); wq int8 [N, K] out; w_scale fp32 [N] out.
@@ -124,9 +124,9 @@ sq_status sq_rmsnorm_smooth_quant(const void *x, int64_t T, int64_t K, const flo
 
 /*
  * W8A8 linear: INT8 x INT8 -> INT32 GEMM with the dequantisation fused into its epilogue.
- *   [MIGRATE] section 7 ("a straight INT8 x INT8 -> INT32 tensor-core operation, followed by a
- *   dequant Y = scale_x * scale_w * Y_int32"); [TAMING] "System Architecture" (nodes "INT8 GEMM",
- *   "Add Bias & Dequantize").
+ *   [MIGRATE] section 7 (the integer product accumulated in 32 bits on the tensor cores, then
+ *   scaled by the activation and weight scales); [TAMING] "System Architecture" (the flowchart's
+ *   GEMM node and its bias-and-dequantise node).
  *   acc[t,n] = sum_k xq[t,k] * wq[n,k]   (exact in int32)
  *   y[t,n]   = bf16_rn( float(acc) * (x_scale[t] * w_scale[n]) + bias[n] )
  * xq int8 [T, K]; x_scale fp32 [T]; wq int8 [N, K]; w_scale fp32 [N]; bias nullable bf16 [N];

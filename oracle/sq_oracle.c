@@ -16,7 +16,7 @@
  *   - Quantiser: symmetric, delta = max|v| / 127, code = round-half-away-from-zero(v * (127/max|v|)),
  *     clamped to [-127, 127]. The pages leave the tie rule open ([TAMING], "Why Outliers Break
  *     Quantization") or use half-to-even in a listing; half-away is the fixed reading. The
- *     reciprocal-multiply form (v * fl32(127/m)) is the fixed reading of "v / delta".
+ *     reciprocal-multiply form (v * fl32(127/m)) is the fixed reading of dividing v by delta.
  *   - All per-element arithmetic is binary32 with each operation rounded (compile with
  *     -ffp-contract=off, no fast-math); the RMSNorm sum of squares is accumulated in binary64.
  *   - RMSNorm is the standard x / sqrt(mean(x^2) + eps) * gamma (the pages name RMSNorm but do not
@@ -110,11 +110,11 @@ static float row_inv_rms(const uint16_t *x, int64_t K, float eps)
  * Per-input-channel abs-max over the rows of a row-major bf16 matrix a[rows, cols] (leading
  * dimension ld elements): amax[j] = max_r |a[r, j]|.
  *   [MIGRATE] section 3 (max|X_j| from calibration samples); [TAMING] "System Architecture"
- *   (flowchart: "Calculate max(|X|) per channel", "Calculate max(|W|) per channel").
+ *   (the flowchart's per-channel maximum of |X| and of |W|).
  * With norm_gamma non-null each row is first replaced by its RMSNorm output
  *   y = (x * inv_rms) * gamma_j,
- * the input the linear layer actually sees ([W8A8] "The trick: move the range into the weights":
- * X comes out of a normalisation layer).
+ * the input the linear layer actually sees (per [W8A8] "The trick: move the range into the weights",
+ * the smoothed layers read the output of a norm).
  * accumulate != 0 keeps a running maximum with the values already in amax (calibration over
  * several batches); otherwise amax is overwritten.
  * For a weight stored [N, K] (output channel n, input channel k) the same call over rows n gives
@@ -145,7 +145,7 @@ void orc_calibrate_absmax(const uint16_t *a, int64_t rows, int64_t cols, int64_t
  * first so that an all-zero channel gives a finite s.
  * The fold into the preceding norm, [W8A8] "The trick..." (s folded into the norm weights):
  *   fold_j = gamma_j / s_j, or 1 / s_j when gamma is null (no norm: the activations are divided
- *   by s directly, [TAMING] flowchart "Smoothing: X_hat = X / s").
+ *   by s directly, the smoothing node of the [TAMING] flowchart).
  * fold may be null.
  */
 void orc_compute_scales(const float *amax_x, const float *amax_w, int64_t K, float alpha,
@@ -165,9 +165,9 @@ void orc_compute_scales(const float *amax_x, const float *amax_w, int64_t K, flo
 
 /*
  * Weight smoothing and per-output-channel INT8 quantisation.
- *   W_hat = diag(s) * W ([MIGRATE] section 2; [TAMING] flowchart "Update Weights"): the weights
+ *   W_hat = diag(s) * W ([MIGRATE] section 2; the weight-update node of the [TAMING] flowchart): the weights
  *   that read input channel k are multiplied by s_k. Stored [N, K], that is column k.
- *   Then one symmetric scale per output row n ([MIGRATE] section 7: "one scale per output row").
+ *   Then one symmetric scale per output row n ([MIGRATE] section 7).
  * s null means unsmoothed (s = 1).
  */
 void orc_smooth_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const float *s,
@@ -187,7 +187,7 @@ void orc_smooth_quantize_weight(const uint16_t *w, int64_t N, int64_t K, const f
  * Online activation path for T tokens of width K.
  *   apply_norm != 0: y = (x * inv_rms) * fold_k with fold = gamma / s folded into the RMSNorm
  *   weight ([W8A8] "The trick..."); apply_norm == 0: y = x * fold_k with fold = 1 / s
- *   ([TAMING] flowchart "Smoothing: X_hat = X / s").
+ *   (the smoothing node of the [TAMING] flowchart).
  *   Then one dynamic symmetric scale per token ([MIGRATE] section 7; [W8A8] "The full model,
  *   served": each token's maximum is found before the matrix product).
  */
@@ -209,8 +209,8 @@ void orc_rmsnorm_smooth_quant(const uint16_t *x, int64_t T, int64_t K, const flo
 /*
  * INT8 x INT8 -> INT32 product of the quantised activations xq[T, K] and weights wq[N, K]
  * (both stored with K contiguous): acc[t, n] = sum_k xq[t, k] * wq[n, k].
- * [MIGRATE] section 7 ("INT8 x INT8 -> INT32 tensor-core operation"); [TAMING] flowchart
- * "INT8 GEMM". Exact: |acc| <= K * 127^2 < 2^31 for K <= 133,000.
+ * [MIGRATE] section 7 (an integer product accumulated in 32 bits on the tensor cores); the GEMM
+ * node of the [TAMING] flowchart. Exact: |acc| <= K * 127^2 < 2^31 for K <= 133,000.
  * Computed for the listed token rows and output columns only (all of them when the lists are
  * null); acc is [nrows, ncols].
  */
@@ -236,7 +236,7 @@ void orc_gemm_s8(const int8_t *xq, int64_t T, const int8_t *wq, int64_t N, int64
 
 /*
  * Dequantisation epilogue, [MIGRATE] section 7 (Y = scale_x * scale_w * Y_int32) and the
- * [TAMING] flowchart ("Add Bias & Dequantize"):
+ * bias-and-dequantise node of the [TAMING] flowchart:
  *   y[t, n] = bf16( float(acc) * (x_scale[t] * w_scale[n]) + bias[n] ),
  * each operation rounded to binary32, the bias (bf16, optional) added last.
  * acc is [nrows, ncols] for the listed rows / columns (all when the lists are null).

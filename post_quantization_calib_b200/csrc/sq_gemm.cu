@@ -6,7 +6,7 @@
 //             ("Bit-level and kernel-level realities": INT8 x INT8 -> INT32 followed by
 //             Y = scale_x * scale_w * Y_int32)
 //   [TAMING]  "Taming the Outliers: A Deep Dive into SmoothQuant for LLM Quantization",
-//             "System Architecture" (flowchart nodes "INT8 GEMM" and "Add Bias & Dequantize")
+//             "System Architecture" (the flowchart's GEMM node and its bias-and-dequantise node)
 //
 // The pages name the operation, not a kernel design (their INT8 kernels target earlier tensor-core
 // generations). This kernel is written for B200:
@@ -30,7 +30,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "sq_device.cuh"
 #include "sq_internal.h"
+
+using namespace sqdev;
 
 namespace {
 
@@ -73,52 +76,7 @@ constexpr uint32_t IDESC = make_idesc(BM, BN);
 // ------------------------------------------------------------------------------------------------
 // PTX wrappers.
 
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ uint64_t global_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
 __device__ __forceinline__ void record_status(unsigned int code) { atomicCAS(&g_sq_status, 0u, code); }
-
-// Waits until the phase of `bar` with parity `parity` has completed. Returns false when
-// `limit_ns` elapsed first or (when `abort_flag` is given) another role of the CTA gave up.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns,
-                                       const volatile int *abort_flag) {
-    if (mbar_try(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
-    for (uint32_t i = 1;; ++i) {
-        if (mbar_try(bar, parity)) return true;
-        if ((i & 127u) == 0u) {
-            if (abort_flag && *abort_flag) return false;
-            if (global_ns() - t0 > limit_ns) return false;
-        }
-    }
-}
 
 __device__ __forceinline__ void give_up(volatile int *abort_flag) {
     record_status(SQ_ERR_TIMEOUT);
@@ -234,7 +192,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         for (int b = 0; b < 2; ++b) { mbar_init(tfull(b), 1); mbar_init(tempty(b), 32 * EPI_WARPS); }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_init_fence();
         fence_async_smem();
     }
     if (warp == 0 && lane == 0) { prefetch_map(&tmA); prefetch_map(&tmB); prefetch_map(&tmY); }
@@ -416,7 +374,7 @@ __global__ void k_selftest_wait(uint64_t limit_ns) {
     if (threadIdx.x == 0) {
         abort_flag = 0;
         mbar_init(smem_u32(&bar), 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        mbar_init_fence();
         if (!mbar_wait(smem_u32(&bar), 0, limit_ns, &abort_flag)) record_status(SQ_ERR_TIMEOUT);
     }
 }
@@ -455,6 +413,21 @@ sq_status encode_2d(EncodeTiledFn enc, CUtensorMap *map, CUtensorMapDataType dt,
 }
 
 }  // namespace
+
+namespace sq {
+
+unsigned int *device_status_word(int device) {
+    static unsigned int *addr[64];
+    if (device < 0 || device >= 64) return nullptr;
+    if (!addr[device]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_sq_status) != cudaSuccess) return nullptr;
+        addr[device] = static_cast<unsigned int *>(p);
+    }
+    return addr[device];
+}
+
+}  // namespace sq
 
 extern "C" {
 

@@ -20,6 +20,10 @@ int sm_count(int device);
 // cudaError_t -> SQ_OK / SQ_ERR_CUDA with the CUDA error text recorded.
 sq_status cuda_status(cudaError_t e, const char *what);
 
+// Device address of the status word (SQ_OK or the first error a kernel recorded) on `device`,
+// which must be the current device. NULL if it cannot be resolved.
+unsigned int *device_status_word(int device);
+
 // Per-device limit of bounded device-side waits, in ns.
 uint64_t wait_timeout_ns(int device);
 void set_wait_timeout_ns(int device, uint64_t ns);

@@ -5,9 +5,8 @@ path and the CPU oracle consume what it returns, so it is the one module they sh
 
 Shape of the data (the pages' description of LLM activations):
   * activations: N(0, 1) tokens in which a fixed, seeded set of input channels is scaled up by
-    10-100x -- "a few hidden dimensions carry values far larger than the others, consistently,
-    token after token" ("SmoothQuant and W8A8: Quantizing Activations Too", "Why activations are
-    the hard part"); the generator pattern (randn, a randperm-chosen fraction of channels multiplied
+    10-100x -- the same few channels are large in every token ("SmoothQuant and W8A8: Quantizing
+    Activations Too", section "Why activations are the hard part"); the generator pattern (randn, a randperm-chosen fraction of channels multiplied
     by a large factor) is the one in the "Implementation in PyTorch" section of "Taming the
     Outliers: A Deep Dive into SmoothQuant for LLM Quantization".
   * weights: N(0, 0.02), roughly normal with no dominant channel ("06 -- SmoothQuant: Migrating

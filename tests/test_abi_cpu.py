@@ -71,6 +71,7 @@ def test_absmax_argument_checks(sqmod):
     assert L.sq_calibrate_absmax(FAKE, 4, 60, 64, None, 1e-6, FAKE, 0, None) == SQ_ERR_MISALIGNED
     assert L.sq_calibrate_absmax(FAKE + 8, 4, 64, 64, None, 1e-6, FAKE, 0, None) == SQ_ERR_MISALIGNED
     assert L.sq_calibrate_absmax(FAKE, 4, 32768, 32768, FAKE, 1e-6, FAKE, 0, None) == SQ_ERR_UNSUPPORTED
+    assert L.sq_calibrate_absmax(FAKE, 4, 16392, 16392, None, 1e-6, FAKE, 0, None) == SQ_ERR_UNSUPPORTED
     assert "cols" in sqmod.sq_last_error()
 
 
