@@ -56,6 +56,12 @@ static __device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uin
     }
 }
 
+// mbar_wait with the common case (phase already complete) inlined.
+static __device__ __forceinline__ bool mbar_ready(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                                  const volatile int *abort_flag) {
+    return mbar_try(bar, parity) || mbar_wait(bar, parity, limit_ns, abort_flag);
+}
+
 // ---------------------------------------------------------------------------------- TMA bulk copy
 // Global -> shared copy of `bytes` (multiple of 16; both addresses 16-byte aligned), completion
 // counted on the mbarrier's transaction count. Destination is this CTA's own shared memory.

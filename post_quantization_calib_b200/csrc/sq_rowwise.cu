@@ -54,10 +54,10 @@ namespace {
 
 constexpr float kFloor = 1e-5f;   // floor of abs-maxima and of s ([TAMING] listing clamps s at 1e-5)
 constexpr float kQmax = 127.0f;   // symmetric INT8 range [-127, 127]
-constexpr int kCluster = 8;       // CTAs per cluster in the column abs-max
+constexpr int kMaxCluster = 8;    // largest cluster tried for the column abs-max
 constexpr int kMaxK = 16384;      // widest row held on chip by the row kernels
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr int kWarps = 8;                   // consumer warps per CTA
+constexpr int kThreads = 32 * (kWarps + 1); // plus one producer warp
 constexpr int kMaxStages = 6;
 constexpr uint32_t kSqBias = 485u << 20;   // binary64 exponent bias mapping bf16 x to x * 2^-411
 
@@ -129,33 +129,54 @@ __device__ __forceinline__ uint32_t codes2(uint64_t y, uint64_t inv2) {
     return __byte_perm(fl, fh, 0x0040);
 }
 
-template <int WPR, int VPL, int MODE, bool NORM>
+// 3-input maximum (one instruction on sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// One CTA = 8 consumer warps in row groups of WPR warps + 1 producer warp. A group processes units of
+// R consecutive rows; lane l of warp w of the group holds 8-element vectors v = i * 32 * WPR +
+// 32 * w + l (i < VPL) of every row of the unit.
+template <int WPR, int VPL, int R, int MODE, bool NORM, bool FULL>
 __global__ void __launch_bounds__(kThreads, 2) k_rows(const RowArgs p)
 {
     constexpr int G = kWarps / WPR;   // row groups per CTA
-    constexpr int GT = 32 * WPR;      // threads per row group
+    constexpr int GT = 32 * WPR;      // consumer threads per row group
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[G * kMaxStages];
-    __shared__ double s_ss[2][kWarps];
-    __shared__ float s_mx[2][kWarps];
+    __shared__ __align__(8) uint64_t s_empty[G * kMaxStages];
+    __shared__ double s_ss[2][kWarps][R];
+    __shared__ float s_mx[2][kWarps][R];
+    __shared__ int s_abort[G];
+    __shared__ long long s_consumed[G];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int group = warp / WPR, wig = warp % WPR, gtid = wig * 32 + lane;
-    const bool leader = gtid == 0;
+    const bool producer = warp == kWarps;                 // the last warp refills the rings
+    const int group = producer ? lane : warp / WPR;        // producer lane g serves group g
+    const int wig = warp % WPR, gtid = wig * 32 + lane;
+    const bool leader = !producer && gtid == 0;
     const int K = p.K, nvec = K >> 3;
     const uint32_t rowbytes = static_cast<uint32_t>(K) * 2u;
+    const uint32_t slotbytes = rowbytes * R;
     const int stages = p.stages;
     uint8_t *ring = smem;
-    const size_t ring_bytes = static_cast<size_t>(G) * stages * rowbytes;
+    const size_t ring_bytes = static_cast<size_t>(G) * stages * slotbytes;
     float4 *c_lo = reinterpret_cast<float4 *>(smem + ring_bytes);   // c[8v .. 8v+3]
     float4 *c_hi = c_lo + nvec;                                     // c[8v+4 .. 8v+7]
 
+    const int64_t units = (p.rows + R - 1) / R;
     const int64_t g0 = static_cast<int64_t>(blockIdx.x) * G + group;
     const int64_t gstride = static_cast<int64_t>(gridDim.x) * G;
-    const int64_t nrows = g0 < p.rows ? (p.rows - 1 - g0) / gstride + 1 : 0;
+    const int64_t nunits = (group < G && g0 < units) ? (units - 1 - g0) / gstride + 1 : 0;
 
     if (tid == 0) {
-        for (int i = 0; i < G * stages; ++i) mbar_init(smem_u32(&s_full[i]), 1);
+        for (int i = 0; i < G * stages; ++i) {
+            mbar_init(smem_u32(&s_full[i]), 1);
+            mbar_init(smem_u32(&s_empty[i]), WPR);
+        }
+        for (int g = 0; g < G; ++g) { s_abort[g] = 0; s_consumed[g] = 0; }
         mbar_init_fence();
     }
     if (MODE == MODE_QUANT && p.vec != nullptr) {
@@ -164,15 +185,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_rows(const RowArgs p)
     }
     __syncthreads();
 
-    auto slot = [&](int s) { return ring + (static_cast<size_t>(group) * stages + s) * rowbytes; };
+    auto slot = [&](int s) { return ring + (static_cast<size_t>(group) * stages + s) * slotbytes; };
     auto full_bar = [&](int s) { return smem_u32(&s_full[group * stages + s]); };
-    auto issue = [&](int64_t j) {
-        const int s = static_cast<int>(j % stages);
-        mbar_expect_tx(full_bar(s), rowbytes);
-        bulk_g2s(smem_u32(slot(s)), p.src + (g0 + j * gstride) * p.ld_bytes, rowbytes, full_bar(s));
-    };
-    if (leader)
-        for (int64_t j = 0; j < nrows && j < stages; ++j) issue(j);
+    auto empty_bar = [&](int s) { return smem_u32(&s_empty[group * stages + s]); };
+    volatile int *abort_flag = &s_abort[group < G ? group : 0];
 
     float mx[VPL][8];          // ABSMAX with norm: running max of fl(|x| * inv_rms) per column
     uint32_t mh[VPL][4];       // ABSMAX without norm: running max of |x| as bf16 pairs
@@ -184,140 +200,227 @@ __global__ void __launch_bounds__(kThreads, 2) k_rows(const RowArgs p)
         for (int k = 0; k < 4; ++k) mh[i][k] = 0u;
     }
 
-    // Row j of this group sits in slot j % stages. Every lane reads the slot twice (sum of squares,
-    // then the values themselves) instead of keeping it in registers across the group barrier; the
-    // slot of row j-1 is refilled at row j's barrier, after every lane has finished with it.
-    int64_t consumed = 0, issued = nrows < stages ? nrows : stages;
+    int64_t issued = 0;
     bool failed = false;
-    for (int64_t j = 0; j < nrows; ++j) {
-        const int s = static_cast<int>(j % stages);
-        const bool ok = mbar_wait(full_bar(s), static_cast<uint32_t>((j / stages) & 1), p.limit_ns, nullptr);
-        const uint4 *rp = reinterpret_cast<const uint4 *>(slot(s));
-        double ss = 0.0;
-        if (NORM) {
-            double ss1 = 0.0;
-#pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int v = i * GT + gtid;
-                const uint4 r = (ok && v < nvec) ? rp[v] : make_uint4(0u, 0u, 0u, 0u);
-                ss = add_squares(r.x, ss);
-                ss1 = add_squares(r.y, ss1);
-                ss = add_squares(r.z, ss);
-                ss1 = add_squares(r.w, ss1);
+    if (producer) {
+        // Lane g keeps group g's ring full: a slot is refilled as soon as the group's warps have
+        // released it, independently of the group's progress on later units.
+        if (lane < G) {
+            int s = 0;
+            uint32_t phase = 0;
+            for (int64_t j = 0; j < nunits; ++j) {
+                if (!mbar_ready(empty_bar(s), phase ^ 1u, p.limit_ns, abort_flag)) {
+                    if (!*abort_flag) failed = true;
+                    *abort_flag = 1;
+                    break;
+                }
+                const int64_t r0 = (g0 + j * gstride) * R;
+                const int nr = static_cast<int>(p.rows - r0 < R ? p.rows - r0 : R);
+                mbar_expect_tx(full_bar(s), rowbytes * static_cast<uint32_t>(nr));
+                for (int r = 0; r < nr; ++r)
+                    bulk_g2s(smem_u32(slot(s) + r * rowbytes), p.src + (r0 + r) * p.ld_bytes, rowbytes, full_bar(s));
+                issued = j + 1;
+                if (++s == stages) { s = 0; phase ^= 1u; }
             }
-            ss = warp_sum(ss + ss1);
         }
-        // One group-wide step: partial sums become visible, every lane is done with row j-1, and a
-        // failed wait anywhere in the group stops the whole group at the same row.
-        bool any_fail;
-        if (WPR == 1) {
-            any_fail = __any_sync(0xFFFFFFFFu, !ok);
-            __syncwarp();
-        } else {
-            if (NORM && lane == 0) s_ss[j & 1][warp] = ss;
-            any_fail = named_sync_or(1 + group, GT, !ok);
+    } else {
+        int64_t consumed = 0;
+        int s = 0;
+        uint32_t phase = 0;
+        for (int64_t j = 0; j < nunits; ++j) {
+            const bool ok = mbar_ready(full_bar(s), phase, p.limit_ns, abort_flag);
+            const int64_t r0 = (g0 + j * gstride) * R;
+            const int nr = static_cast<int>(p.rows - r0 < R ? p.rows - r0 : R);   // uniform in the group
+            const uint4 *rp = reinterpret_cast<const uint4 *>(slot(s));
+            const int rv = static_cast<int>(rowbytes / 16);                           // vectors per row
+            double ss[R];
+#pragma unroll
+            for (int r = 0; r < R; ++r) ss[r] = 0.0;
             if (NORM) {
-                ss = 0.0;
 #pragma unroll
-                for (int w = 0; w < WPR; ++w) ss += s_ss[j & 1][group * WPR + w];
-            }
-        }
-        if (any_fail) { failed = true; break; }
-        consumed = j + 1;
-        if (leader && j >= 1 && issued < nrows) issue(issued++);
-        const int64_t row = g0 + j * gstride;
-        const float ir = NORM ? inv_rms(__dmul_rn(ss, 0x1p822), K, p.inv_k, p.eps) : 1.0f;
-        const uint64_t ir2 = pack2(ir, ir);
-
-        if (MODE == MODE_ABSMAX) {
+                for (int r = 0; r < R; ++r) {
+                    if (r < nr) {
+                        double a = 0.0, b = 0.0;
 #pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int v = i * GT + gtid;
-                const uint4 r = v < nvec ? rp[v] : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint32_t w = word_of(r, k);
-                    if (NORM) {
-                        const uint64_t ay = mul2_rn(pack2u((w & 0x7FFFu) << 16, w & 0x7FFF0000u), ir2);
-                        uint32_t al, ah;
-                        unpack2(ay, al, ah);
-                        mx[i][2 * k] = fmaxf(mx[i][2 * k], __uint_as_float(al));
-                        mx[i][2 * k + 1] = fmaxf(mx[i][2 * k + 1], __uint_as_float(ah));
-                    } else {
-                        __nv_bfloat162 cur = *reinterpret_cast<__nv_bfloat162 *>(&mh[i][k]);
-                        const uint32_t a = w & 0x7FFF7FFFu;
-                        cur = __hmax2(cur, *reinterpret_cast<const __nv_bfloat162 *>(&a));
-                        mh[i][k] = *reinterpret_cast<uint32_t *>(&cur);
+                        for (int i = 0; i < VPL; ++i) {
+                            const int v = i * GT + gtid;
+                            const uint4 q = (ok && (FULL || v < nvec)) ? rp[r * rv + v] : make_uint4(0u, 0u, 0u, 0u);
+                            a = add_squares(q.x, a);
+                            b = add_squares(q.y, b);
+                            a = add_squares(q.z, a);
+                            b = add_squares(q.w, b);
+                        }
+                        ss[r] = warp_sum(a + b);
                     }
                 }
             }
-        } else {
-            // y = (x * inv_rms) * c  (or x * c, or x), kept in registers as element pairs
-            uint64_t y[VPL][4];
-            float m = 0.0f;
+            // Group-wide step: partial sums become visible, and a failed wait anywhere in the group
+            // stops the whole group at the same unit.
+            bool any_fail;
+            if (WPR == 1) {
+                any_fail = __any_sync(0xFFFFFFFFu, !ok);
+            } else {
+                if (NORM && lane == 0) {
 #pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int v = i * GT + gtid;
-                const uint4 r = v < nvec ? rp[v] : make_uint4(0u, 0u, 0u, 0u);
-                float4 cl = make_float4(1.f, 1.f, 1.f, 1.f), ch = cl;
-                if (p.vec != nullptr && v < nvec) { cl = c_lo[v]; ch = c_hi[v]; }
-                const uint64_t c2[4] = {pack2(cl.x, cl.y), pack2(cl.z, cl.w), pack2(ch.x, ch.y), pack2(ch.z, ch.w)};
+                    for (int r = 0; r < R; ++r) s_ss[j & 1][warp][r] = ss[r];
+                }
+                any_fail = named_sync_or(1 + group, GT, !ok);
+                if (NORM) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint32_t w = word_of(r, k);
-                    const uint64_t x2 = pack2u(w << 16, w & 0xFFFF0000u);
-                    const uint64_t yy = NORM ? mul2_rn(mul2_rn(x2, ir2), c2[k]) : (p.vec != nullptr ? mul2_rn(x2, c2[k]) : x2);
-                    y[i][k] = yy;
-                    uint32_t yl, yh;
-                    unpack2(yy, yl, yh);
-                    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(yl)), fabsf(__uint_as_float(yh))));
+                    for (int r = 0; r < R; ++r) {
+                        double t = 0.0;
+#pragma unroll
+                        for (int w = 0; w < WPR; ++w) t += s_ss[j & 1][group * WPR + w][r];
+                        ss[r] = t;
+                    }
                 }
             }
-            m = warp_max(m);
-            if (WPR > 1) {
-                if (lane == 0) s_mx[j & 1][warp] = m;
-                named_sync(1 + group, GT);
-                m = 0.0f;
-#pragma unroll
-                for (int w = 0; w < WPR; ++w) m = fmaxf(m, s_mx[j & 1][group * WPR + w]);
+            if (any_fail) {
+                if (leader) { if (!*abort_flag) failed = true; *abort_flag = 1; }
+                break;
             }
-            const float delta = m > 0.0f ? __fdiv_rn(m, kQmax) : 0.0f;
-            const float inv = m > 0.0f ? __fdiv_rn(kQmax, m) : 0.0f;
-            const uint64_t inv2 = pack2(inv, inv);
-            uint2 *qrow = reinterpret_cast<uint2 *>(p.q + row * static_cast<int64_t>(K));
+            uint64_t ir2[R];
 #pragma unroll
-            for (int i = 0; i < VPL; ++i) {
-                const int v = i * GT + gtid;
-                if (v < nvec) {
-                    const uint32_t c01 = codes2(y[i][0], inv2), c23 = codes2(y[i][1], inv2);
-                    const uint32_t c45 = codes2(y[i][2], inv2), c67 = codes2(y[i][3], inv2);
-                    qrow[v] = make_uint2(__byte_perm(c01, c23, 0x5410), __byte_perm(c45, c67, 0x5410));
+            for (int r = 0; r < R; ++r) {
+                const float ir = NORM ? inv_rms(__dmul_rn(ss[r], 0x1p822), K, p.inv_k, p.eps) : 1.0f;
+                ir2[r] = pack2(ir, ir);
+            }
+
+            if (MODE == MODE_ABSMAX) {
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) {
+                    const int v = i * GT + gtid;
+                    const bool in = FULL || v < nvec;
+                    uint4 q[R];
+#pragma unroll
+                    for (int r = 0; r < R; ++r) q[r] = (in && r < nr) ? rp[r * rv + v] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        if (NORM) {
+                            float yl[R], yh[R];
+#pragma unroll
+                            for (int r = 0; r < R; ++r) {
+                                const uint32_t w = word_of(q[r], k);
+                                uint32_t l, h;
+                                unpack2(mul2_rn(pack2u(w << 16, w & 0xFFFF0000u), ir2[r]), l, h);
+                                yl[r] = fabsf(__uint_as_float(l));
+                                yh[r] = fabsf(__uint_as_float(h));
+                            }
+                            if (R == 2) {
+                                mx[i][2 * k] = max3f(mx[i][2 * k], yl[0], yl[R - 1]);
+                                mx[i][2 * k + 1] = max3f(mx[i][2 * k + 1], yh[0], yh[R - 1]);
+                            } else {
+                                mx[i][2 * k] = fmaxf(mx[i][2 * k], yl[0]);
+                                mx[i][2 * k + 1] = fmaxf(mx[i][2 * k + 1], yh[0]);
+                            }
+                        } else {
+#pragma unroll
+                            for (int r = 0; r < R; ++r) {
+                                __nv_bfloat162 cur = *reinterpret_cast<__nv_bfloat162 *>(&mh[i][k]);
+                                const uint32_t a = word_of(q[r], k) & 0x7FFF7FFFu;
+                                cur = __hmax2(cur, *reinterpret_cast<const __nv_bfloat162 *>(&a));
+                                mh[i][k] = *reinterpret_cast<uint32_t *>(&cur);
+                            }
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_bar(s));      // this warp is done with the slot
+            } else {
+                // y = (x * inv_rms) * c  (or x * c, or x), kept in registers as element pairs
+                uint64_t y[R][VPL][4];
+                float m[R];
+#pragma unroll
+                for (int r = 0; r < R; ++r) m[r] = 0.0f;
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) {
+                    const int v = i * GT + gtid;
+                    const bool in = FULL || v < nvec;
+                    float4 cl = make_float4(1.f, 1.f, 1.f, 1.f), ch = cl;
+                    if (p.vec != nullptr && in) { cl = c_lo[v]; ch = c_hi[v]; }
+                    const uint64_t c2[4] = {pack2(cl.x, cl.y), pack2(cl.z, cl.w), pack2(ch.x, ch.y), pack2(ch.z, ch.w)};
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        const uint4 q = (in && r < nr) ? rp[r * rv + v] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t w = word_of(q, k);
+                            const uint64_t x2 = pack2u(w << 16, w & 0xFFFF0000u);
+                            const uint64_t yy = NORM ? mul2_rn(mul2_rn(x2, ir2[r]), c2[k]) : (p.vec != nullptr ? mul2_rn(x2, c2[k]) : x2);
+                            y[r][i][k] = yy;
+                            uint32_t yl, yh;
+                            unpack2(yy, yl, yh);
+                            m[r] = max3f(m[r], fabsf(__uint_as_float(yl)), fabsf(__uint_as_float(yh)));
+                        }
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty_bar(s));      // the unit is in registers now
+#pragma unroll
+                for (int r = 0; r < R; ++r) m[r] = warp_max(m[r]);
+                if (WPR > 1) {
+                    if (lane == 0) {
+#pragma unroll
+                        for (int r = 0; r < R; ++r) s_mx[j & 1][warp][r] = m[r];
+                    }
+                    named_sync(1 + group, GT);
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        float t = 0.0f;
+#pragma unroll
+                        for (int w = 0; w < WPR; ++w) t = fmaxf(t, s_mx[j & 1][group * WPR + w][r]);
+                        m[r] = t;
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    if (r < nr) {
+                        const float delta = m[r] > 0.0f ? __fdiv_rn(m[r], kQmax) : 0.0f;
+                        const float inv = m[r] > 0.0f ? __fdiv_rn(kQmax, m[r]) : 0.0f;
+                        const uint64_t inv2 = pack2(inv, inv);
+                        uint2 *qrow = reinterpret_cast<uint2 *>(p.q + (r0 + r) * static_cast<int64_t>(K));
+#pragma unroll
+                        for (int i = 0; i < VPL; ++i) {
+                            const int v = i * GT + gtid;
+                            if (FULL || v < nvec) {
+                                const uint32_t c01 = codes2(y[r][i][0], inv2), c23 = codes2(y[r][i][1], inv2);
+                                const uint32_t c45 = codes2(y[r][i][2], inv2), c67 = codes2(y[r][i][3], inv2);
+                                qrow[v] = make_uint2(__byte_perm(c01, c23, 0x5410), __byte_perm(c45, c67, 0x5410));
+                            }
+                        }
+                        if (leader) p.scale[r0 + r] = delta;
+                    }
                 }
             }
-            if (leader) p.scale[row] = delta;
+            consumed = j + 1;
+            if (++s == stages) { s = 0; phase ^= 1u; }
         }
+        if (leader) s_consumed[group] = consumed;
     }
 
-    if (failed && leader) atomicCAS(p.status, 0u, static_cast<unsigned int>(SQ_ERR_TIMEOUT));
+    if (failed) atomicCAS(p.status, 0u, static_cast<unsigned int>(SQ_ERR_TIMEOUT));
+    __syncthreads();
     // Copies issued but never consumed (only after a failed wait) must land before the CTA exits.
-    if (leader) {
-        for (int64_t j = consumed; j < issued; ++j)
+    if (producer && lane < G) {
+        for (int64_t j = s_consumed[group]; j < issued; ++j)
             if (!mbar_wait(full_bar(static_cast<int>(j % stages)), static_cast<uint32_t>((j / stages) & 1), p.limit_ns, nullptr))
                 atomicCAS(p.status, 0u, static_cast<unsigned int>(SQ_ERR_TIMEOUT));
     }
 
     if (MODE == MODE_ABSMAX) {
-        __syncthreads();                                   // the ring is free: reuse it
+        __syncthreads();                                   // the ring is idle: reuse it
         float *red = reinterpret_cast<float *>(smem);      // [G][K]
+        if (!producer) {
 #pragma unroll
-        for (int i = 0; i < VPL; ++i) {
-            const int v = i * GT + gtid;
-            if (v < nvec) {
-                float *dst = red + static_cast<size_t>(group) * K + v * 8;
+            for (int i = 0; i < VPL; ++i) {
+                const int v = i * GT + gtid;
+                if (FULL || v < nvec) {
+                    float *dst = red + static_cast<size_t>(group) * K + v * 8;
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    dst[2 * k] = NORM ? mx[i][2 * k] : __uint_as_float(mh[i][k] << 16);
-                    dst[2 * k + 1] = NORM ? mx[i][2 * k + 1] : __uint_as_float(mh[i][k] & 0xFFFF0000u);
+                    for (int k = 0; k < 4; ++k) {
+                        dst[2 * k] = NORM ? mx[i][2 * k] : __uint_as_float(mh[i][k] << 16);
+                        dst[2 * k + 1] = NORM ? mx[i][2 * k + 1] : __uint_as_float(mh[i][k] & 0xFFFF0000u);
+                    }
                 }
             }
         }
@@ -331,13 +434,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_rows(const RowArgs p)
         }
         cg::cluster_group cluster = cg::this_cluster();
         cluster.sync();
-        const int share = (K + kCluster - 1) / kCluster;
+        const int csize = static_cast<int>(cluster.num_blocks());
+        const int share = (K + csize - 1) / csize;
         const int c0 = static_cast<int>(cluster.block_rank()) * share;
         const int c1 = min(K, c0 + share);
         for (int c = c0 + tid; c < c1; c += kThreads) {
             float m = 0.0f;
-#pragma unroll
-            for (int q = 0; q < kCluster; ++q) m = fmaxf(m, cluster.map_shared_rank(red, q)[c]);
+            for (int q = 0; q < csize; ++q) m = fmaxf(m, cluster.map_shared_rank(red, q)[c]);
             // abs-maxima are non-negative, where IEEE order equals unsigned integer order
             if (m > 0.0f) atomicMax(reinterpret_cast<unsigned int *>(p.amax + c), __float_as_uint(m));
         }
@@ -373,34 +476,57 @@ __global__ void k_scales(const float *__restrict__ ax, const float *__restrict__
 // Launch geometry and dispatch.
 
 struct Geo {
-    int wpr, vpl, groups, stages;
+    int wpr, vpl, rpu, groups, stages;   // warps per row group, vectors per lane, rows per unit
     size_t smem;
 };
 
+// Row groups hold 64 values per lane per unit where possible (4 vectors x 2 rows).
 Geo row_geo(int K, int mode) {
     const int nvec = K / 8;
     Geo g;
-    g.wpr = nvec <= 256 ? 1 : nvec <= 512 ? 2 : nvec <= 1024 ? 4 : 8;
-    const int per = (nvec + 32 * g.wpr - 1) / (32 * g.wpr);
-    g.vpl = g.wpr > 1 ? 8 : per <= 1 ? 1 : per <= 2 ? 2 : per <= 4 ? 4 : 8;
+    if (nvec <= 128) {
+        g.wpr = 1;
+        const int per = (nvec + 31) / 32;
+        g.vpl = per <= 1 ? 1 : per <= 2 ? 2 : 4;
+        g.rpu = 2;
+    } else if (nvec <= 1024) {
+        g.wpr = nvec <= 256 ? 2 : nvec <= 512 ? 4 : 8;
+        g.vpl = 4;
+        g.rpu = 2;
+    } else {
+        g.wpr = 8;
+        g.vpl = 8;
+        g.rpu = 1;
+    }
     g.groups = kWarps / g.wpr;
-    const size_t rowbytes = static_cast<size_t>(K) * 2;
+    const size_t slotbytes = static_cast<size_t>(K) * 2 * g.rpu;
     const size_t extra = mode == MODE_QUANT ? static_cast<size_t>(K) * 4 : 0;
     const long budget = 96L * 1024 - static_cast<long>(extra);
-    long st = budget / static_cast<long>(g.groups * rowbytes);
+    long st = budget / static_cast<long>(g.groups * slotbytes);
     g.stages = static_cast<int>(st < 2 ? 2 : st > kMaxStages ? kMaxStages : st);
-    const size_t ring = static_cast<size_t>(g.groups) * g.stages * rowbytes;
+    const size_t ring = static_cast<size_t>(g.groups) * g.stages * slotbytes;
     const size_t red = mode == MODE_ABSMAX ? static_cast<size_t>(g.groups) * K * 4 : 0;
     g.smem = (ring > red ? ring : red) + extra;
     return g;
 }
 
-template <int WPR, int VPL, int MODE, bool NORM>
+template <int WPR, int VPL, int R, int MODE, bool NORM, bool FULL>
 sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
-    auto kern = k_rows<WPR, VPL, MODE, NORM>;
+    auto kern = k_rows<WPR, VPL, R, MODE, NORM, FULL>;
     constexpr int G = kWarps / WPR;
     static size_t configured_smem[64];
     static int per_sm[64];
+    static int cluster_size[64], cluster_ctas[64];
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = geo.smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     if (configured_smem[dev] < geo.smem) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(geo.smem));
         if (e != cudaSuccess) return sq::cuda_status(e, "cudaFuncSetAttribute(rows)");
@@ -408,6 +534,20 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, geo.smem);
         if (e != cudaSuccess) return sq::cuda_status(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor(rows)");
         per_sm[dev] = nb > 0 ? nb : 1;
+        if (MODE == MODE_ABSMAX) {
+            // Whole clusters must fit on one GPU processing cluster; take the size that keeps the
+            // most CTAs resident at once (ties: the larger cluster, fewer atomics).
+            cluster_size[dev] = 1;
+            cluster_ctas[dev] = 0;
+            for (int c = kMaxCluster; c >= 2; c /= 2) {
+                attr[0].val.clusterDim.x = c;
+                cfg.gridDim = dim3(c, 1, 1);
+                int nc = 0;
+                if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) != cudaSuccess) { (void)cudaGetLastError(); continue; }
+                if (nc * c > cluster_ctas[dev]) { cluster_ctas[dev] = nc * c; cluster_size[dev] = c; }
+            }
+            if (cluster_ctas[dev] == 0) return sq::fail(SQ_ERR_CUDA, "no cluster configuration fits the abs-max kernel");
+        }
         configured_smem[dev] = geo.smem;
     }
     const int64_t full = static_cast<int64_t>(sq::sm_count(dev)) * per_sm[dev];
@@ -416,42 +556,42 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
     a.status = sq::device_status_word(dev);
     a.limit_ns = sq::wait_timeout_ns(dev);
     if (a.status == nullptr) return sq::fail(SQ_ERR_CUDA, "device status word unavailable");
+    const int64_t units = (a.rows + R - 1) / R;
     if (MODE == MODE_QUANT) {
-        int64_t ctas = (a.rows + G - 1) / G;
+        int64_t ctas = (units + G - 1) / G;
         if (ctas > full) ctas = full;
         kern<<<static_cast<unsigned>(ctas), kThreads, geo.smem, st>>>(a);
         return sq::cuda_status(cudaGetLastError(), "launch(rowquant)");
     }
-    int64_t ctas = (a.rows + 8 * G - 1) / (8 * G);     // at least ~8 rows per group
-    if (ctas > full) ctas = full;
-    ctas = ((ctas + kCluster - 1) / kCluster) * kCluster;
-    cudaLaunchConfig_t cfg = {};
+    // one wave of resident clusters at most, at least ~4 units per group
+    const int csz = cluster_size[dev];
+    int64_t ctas = (units + 4 * G - 1) / (4 * G);
+    if (ctas > cluster_ctas[dev]) ctas = cluster_ctas[dev];
+    ctas = ((ctas + csz - 1) / csz) * csz;
+    attr[0].val.clusterDim.x = csz;
     cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = geo.smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kCluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     return sq::cuda_status(cudaLaunchKernelEx(&cfg, kern, a), "launch(absmax)");
 }
 
+template <int MODE, bool NORM, bool FULL>
+sq_status dispatch_rows_f(const RowArgs &a, const Geo &g, int dev, cudaStream_t st) {
+    switch (g.wpr * 100 + g.vpl * 10 + g.rpu) {
+        case 112: return launch_rows_t<1, 1, 2, MODE, NORM, FULL>(a, g, dev, st);
+        case 122: return launch_rows_t<1, 2, 2, MODE, NORM, FULL>(a, g, dev, st);
+        case 142: return launch_rows_t<1, 4, 2, MODE, NORM, FULL>(a, g, dev, st);
+        case 242: return launch_rows_t<2, 4, 2, MODE, NORM, FULL>(a, g, dev, st);
+        case 442: return launch_rows_t<4, 4, 2, MODE, NORM, FULL>(a, g, dev, st);
+        case 842: return launch_rows_t<8, 4, 2, MODE, NORM, FULL>(a, g, dev, st);
+        default: return launch_rows_t<8, 8, 1, MODE, NORM, FULL>(a, g, dev, st);
+    }
+}
+
+// FULL: the row is exactly VPL vectors per lane of the group (no bounds checks per vector).
 template <int MODE, bool NORM>
 sq_status dispatch_rows(const RowArgs &a, int dev, cudaStream_t st) {
     const Geo g = row_geo(a.K, MODE);
-    switch (g.wpr * 16 + g.vpl) {
-        case 1 * 16 + 1: return launch_rows_t<1, 1, MODE, NORM>(a, g, dev, st);
-        case 1 * 16 + 2: return launch_rows_t<1, 2, MODE, NORM>(a, g, dev, st);
-        case 1 * 16 + 4: return launch_rows_t<1, 4, MODE, NORM>(a, g, dev, st);
-        case 1 * 16 + 8: return launch_rows_t<1, 8, MODE, NORM>(a, g, dev, st);
-        case 2 * 16 + 8: return launch_rows_t<2, 8, MODE, NORM>(a, g, dev, st);
-        case 4 * 16 + 8: return launch_rows_t<4, 8, MODE, NORM>(a, g, dev, st);
-        default: return launch_rows_t<8, 8, MODE, NORM>(a, g, dev, st);
-    }
+    const bool full = (a.K / 8) == g.vpl * 32 * g.wpr;
+    return full ? dispatch_rows_f<MODE, NORM, true>(a, g, dev, st) : dispatch_rows_f<MODE, NORM, false>(a, g, dev, st);
 }
 
 }  // namespace
