@@ -141,6 +141,18 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, cons
                          const float *w_scale, int64_t N, int64_t K, const void *bias, void *y,
                          int32_t *acc_out, void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * Tile shape of sq_w8a8_linear for the calls that follow, in this process, on every device.
+ *   enable = 0 (default): one SM per 128-token x 256-channel tile (tcgen05.mma.cta_group::1).
+ *   enable = 1: pairs of SMs (a two-CTA cluster, tcgen05.mma.cta_group::2) per 256 x 256 tile when
+ *               T >= 256; smaller T keeps the single-SM form.
+ * Both forms compute the same bits. The pair form moves half the weight bytes per SM and needs fewer
+ * SM cycles, but on B200 under its power limit it ran at lower clocks and was no faster, hence the
+ * default. Any other value returns SQ_ERR_INVALID_ARG. Not synchronised with calls in flight on
+ * other host threads.
+ */
+sq_status sq_set_gemm_cta_pair(int enable);
+
 /* Bytes of workspace sq_w8a8_linear needs for these sizes (0 in this build). */
 size_t sq_w8a8_linear_workspace_size(int64_t T, int64_t N, int64_t K);
 

@@ -30,6 +30,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "sq_device.cuh"
 #include "sq_internal.h"
 
@@ -40,6 +42,9 @@ namespace {
 // Device-side status word: 0 or the first sq_status a kernel recorded.
 __device__ unsigned int g_sq_status;
 
+// Host-side choice of the GEMM form (sq_set_gemm_cta_pair).
+std::atomic<int> g_cta_pair{0};
+
 constexpr int BM = 128;            // tokens per tile (MMA M)
 constexpr int BN = 256;            // output channels per tile (MMA N)
 constexpr int BK = 128;            // K bytes per pipeline stage (one 128-byte swizzle row)
@@ -48,7 +53,7 @@ constexpr int STAGES = 4;
 constexpr int A_STAGE = BM * BK;   // 16 KB
 constexpr int B_STAGE = BN * BK;   // 32 KB
 constexpr int EPI_WARPS = 4;
-constexpr int OUT_COLS = 64;       // bf16 columns per TMA store box (128 bytes)
+constexpr int OUT_COLS = 32;       // bf16 columns per TMA store box (64 bytes, 64-byte swizzle)
 constexpr int OUT_ROWS = 32;       // rows per box: one warp's TMEM lane quarter
 constexpr int OUT_BOX = OUT_COLS * 2 * OUT_ROWS;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
@@ -58,7 +63,9 @@ constexpr int BAND = 16;           // M tiles per raster band
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
 constexpr int OFF_OUT = OFF_B + STAGES * B_STAGE;
-constexpr int OFF_BAR = OFF_OUT + EPI_WARPS * 2 * OUT_BOX;
+constexpr int COL_TAB = 2 * BN * 4;   // w_scale and bias (binary32) of one tile's columns
+constexpr int OFF_COL = OFF_OUT + EPI_WARPS * 2 * OUT_BOX;
+constexpr int OFF_BAR = OFF_COL + 2 * COL_TAB;   // one table per accumulator buffer
 constexpr int NBARS = 2 * STAGES + 5;   // full[S], empty[S], tfull[2], tempty[2], done
 constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
 constexpr int SMEM_USED = OFF_MISC + 16;
@@ -125,17 +132,6 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
         : "memory");
 }
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory descriptor of a K-major operand tile written by TMA with the 128-byte swizzle:
@@ -156,9 +152,208 @@ __device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int
     m = band * BAND + (within - n * bs);
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t *>(&h);
+// 2-SM (CTA pair) forms.
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t addr, uint32_t rank) {
+    uint32_t d;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(addr), "r"(rank));
+    return d;
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on `bar_cluster`, a barrier of
+// either CTA of the pair (shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, uint32_t bar_cluster, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait with cluster-scope acquire (the barrier is completed from the peer CTA).
+__device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, uint64_t limit_ns,
+                                               const volatile int *abort_flag) {
+    if (mbar_try_cluster(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_cluster(bar, parity)) return true;
+        if ((i & 127u) == 0u) {
+            if (abort_flag && *abort_flag) return false;
+            if (global_ns() - t0 > limit_ns) return false;
+        }
+    }
+}
+__device__ __forceinline__ void tmem_alloc2(uint32_t slot, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_commit2(uint32_t bar_cluster) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster) : "memory");
+}
+__device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+// Column table of one tile: w_scale and bias (widened to binary32) of its 256 output channels, read
+// by every epilogue lane with broadcast shared-memory loads. The 128 epilogue threads each fetch two
+// columns from global memory one tile ahead and write them when the tile starts; there is one table
+// per accumulator buffer.
+constexpr int EPI_THREADS = 32 * EPI_WARPS;
+constexpr uint32_t EPI_BAR = 1;     // named barrier of the epilogue warps
+
+struct ColShare {
+    float2 w;
+    uint32_t b;
+};
+
+__device__ __forceinline__ void cols_fetch(ColShare &p, int n0, int ep, const float *__restrict__ w_scale,
+                                           const __nv_bfloat16 *__restrict__ bias, int N) {
+    const int col = n0 + 2 * ep;
+    p.w = make_float2(0.f, 0.f);
+    p.b = 0u;
+    if (col < N) {      // N is even: both columns are in range or both beyond it
+        p.w = __ldg(reinterpret_cast<const float2 *>(w_scale + col));
+        if (bias != nullptr) p.b = __ldg(reinterpret_cast<const unsigned int *>(bias + col));
+    }
+}
+
+__device__ __forceinline__ void cols_store(const ColShare &p, float *tab, int ep) {
+    *reinterpret_cast<float2 *>(tab + 2 * ep) = p.w;
+    *reinterpret_cast<float2 *>(tab + BN + 2 * ep) = make_float2(__uint_as_float(p.b << 16), __uint_as_float(p.b & 0xFFFF0000u));
+}
+
+// Two packed pairs (four consecutive binary32 values) from shared memory, same address in every lane.
+__device__ __forceinline__ void lds_pairs(const float *p, uint64_t &a, uint64_t &b) {
+    asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(smem_u32(p)));
+}
+
+__device__ __forceinline__ uint32_t bf16x2_rn(uint64_t v) {
+    uint32_t lo, hi, d;
+    unpack2(v, lo, hi);
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(__uint_as_float(hi)), "f"(__uint_as_float(lo)));
+    return d;
+}
+
+// 32 columns of this warp's TMEM lane quarter into r[0..31] (asynchronous until tmem_ld_wait).
+__device__ __forceinline__ void tmem_ld32p(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+// Orders every later use of r[0..31] after the preceding tcgen05.wait::ld.
+__device__ __forceinline__ void regs_after_wait(uint32_t *r) {
+#pragma unroll
+    for (int i = 0; i < 32; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+// Epilogue of one warp for one output tile: reads its 32 TMEM lanes (token rows row0 .. row0+31) for
+// columns n0 .. n0+255 of accumulator buffer `tcol` (TMEM column offset), applies
+// y = bf16(float(acc) * (x_scale * w_scale) + bias) in binary32 (each operation rounded once, two
+// columns per packed instruction), stages 32 x 32 boxes in 64-byte-swizzled shared memory and writes
+// them with TMA stores; optionally writes the raw accumulators. `tab` is the tile's column table,
+// `xs` the x_scale of this lane's row. The TMEM read of the next 32 columns is in flight while the
+// current 32 are converted. `stage_buf` holds two boxes that alternate; `nstores` counts this warp's
+// stores.
+__device__ __forceinline__ void epilogue_rows(uint32_t tmem_base, int quad, int lane, uint32_t tcol, int row0, int n0,
+                                              float xs, const float *tab, bool has_bias, int32_t *__restrict__ acc_out,
+                                              int T, int N, const CUtensorMap *tmY, uint8_t *stage_buf, int &nstores)
+{
+    if (row0 >= T) return;
+    const int row = row0 + lane;
+    const uint64_t xs2 = pack2(xs, xs);
+    const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tcol;
+    uint32_t ra[32], rb[32];
+    tmem_ld32p(tl, ra);
+#pragma unroll
+    for (int c = 0; c < BN / OUT_COLS; ++c) {
+        uint32_t *cur = (c & 1) ? rb : ra;
+        uint32_t *nxt = (c & 1) ? ra : rb;
+        tmem_ld_wait();
+        regs_after_wait(cur);
+        if (c + 1 < BN / OUT_COLS) tmem_ld32p(tl + (c + 1) * OUT_COLS, nxt);
+        const int col0 = n0 + c * OUT_COLS;
+        if (col0 >= N) continue;
+        if (acc_out != nullptr && row < T) {
+            int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + col0);
+#pragma unroll
+            for (int g = 0; g < OUT_COLS / 4; ++g) {
+                if (col0 + 4 * g < N)
+                    dst[g] = make_int4(static_cast<int>(cur[4 * g]), static_cast<int>(cur[4 * g + 1]),
+                                       static_cast<int>(cur[4 * g + 2]), static_cast<int>(cur[4 * g + 3]));
+            }
+        }
+        uint32_t packed[OUT_COLS / 2];
+#pragma unroll
+        for (int g = 0; g < OUT_COLS / 4; ++g) {
+            uint64_t w01, w23;
+            lds_pairs(tab + c * OUT_COLS + 4 * g, w01, w23);
+            const uint64_t a01 = pack2(__int2float_rn(static_cast<int>(cur[4 * g])), __int2float_rn(static_cast<int>(cur[4 * g + 1])));
+            const uint64_t a23 = pack2(__int2float_rn(static_cast<int>(cur[4 * g + 2])), __int2float_rn(static_cast<int>(cur[4 * g + 3])));
+            uint64_t v01 = mul2_rn(a01, mul2_rn(xs2, w01));
+            uint64_t v23 = mul2_rn(a23, mul2_rn(xs2, w23));
+            if (has_bias) {
+                uint64_t b01, b23;
+                lds_pairs(tab + BN + c * OUT_COLS + 4 * g, b01, b23);
+                v01 = add2_rn(v01, b01);
+                v23 = add2_rn(v23, b23);
+            }
+            packed[2 * g] = bf16x2_rn(v01);
+            packed[2 * g + 1] = bf16x2_rn(v23);
+        }
+        // stage the 32 x 32 box (64-byte rows, 64-byte swizzle: the 16-byte chunk index is XORed
+        // with bits 1..2 of the row), then one TMA store
+        uint8_t *sb = stage_buf + (nstores & 1) * OUT_BOX;
+        if (lane == 0) bulk_wait_read_1();
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int pos = q ^ ((lane >> 1) & 3);
+            *reinterpret_cast<uint4 *>(sb + lane * 64 + pos * 16) =
+                make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(tmY, smem_u32(sb), col0, row0);
+            bulk_commit();
+        }
+        ++nstores;
+    }
+    tmem_ld_wait();     // nothing of this tile's accumulator is still being read
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -175,6 +370,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     uint8_t *sA = smem + OFF_A;
     uint8_t *sB = smem + OFF_B;
     uint8_t *sOut = smem + OFF_OUT;
+    float *sCol = reinterpret_cast<float *>(smem + OFF_COL);
     const uint32_t bar0 = smem_u32(smem + OFF_BAR);
     auto full = [&](int s) { return bar0 + 8u * s; };
     auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
@@ -275,85 +471,36 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         // ---------------- epilogue ----------------
         const int quad = warp & 3;                  // TMEM lanes this warp may read: 32*quad .. +31
         uint8_t *stage_buf = sOut + (warp - 2) * 2 * OUT_BOX;
+        const int ep = threadIdx.x - 64;            // 0 .. 127 among the epilogue threads
         int nstores = 0;
         int lt = 0;
+        // this thread's share of the next tile's column table, and its row's x_scale, one tile ahead
+        ColShare cols;
+        float xs = 0.0f;
+        auto prefetch = [&](int t) {
+            if (t >= num_tiles) return;
+            int m, n;
+            tile_coords(t, m_tiles, n_tiles, m, n);
+            cols_fetch(cols, n * BN, ep, w_scale, bias, N);
+            const int row = m * BM + quad * 32 + lane;
+            xs = row < T ? __ldg(x_scale + row) : 0.0f;
+        };
+        prefetch(blockIdx.x);
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++lt) {
             const int buf = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1);
-            if (!mbar_wait(tfull(buf), use & 1u, limit_ns, abort_flag)) { give_up(abort_flag); break; }
+            const bool ok = mbar_wait(tfull(buf), use & 1u, limit_ns, abort_flag);
+            float *tab = sCol + buf * (COL_TAB / 4);
+            if (ok) cols_store(cols, tab, ep);
+            // every epilogue thread arrives (its wait is bounded); the table is complete after it
+            if (named_sync_or(EPI_BAR, EPI_THREADS, !ok)) { give_up(abort_flag); break; }
             tc_fence_after();
             int m, n;
             tile_coords(t, m_tiles, n_tiles, m, n);
-            const int row0 = m * BM + quad * 32;     // first token row of this warp's quarter
-            const int row = row0 + lane;
-            if (row0 < T) {
-                const float xs = row < T ? __ldg(x_scale + row) : 0.0f;
-                for (int c = 0; c < BN / OUT_COLS; ++c) {
-                    const int col0 = n * BN + c * OUT_COLS;
-                    if (col0 >= N) break;
-                    uint32_t r[2][32];
-                    const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                                           static_cast<uint32_t>(buf * BN + c * OUT_COLS);
-                    tmem_ld32(taddr, r[0]);
-                    tmem_ld32(taddr + 32, r[1]);
-                    tmem_ld_wait();
-                    if (acc_out != nullptr && row < T) {
-                        int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + col0);
-#pragma unroll
-                        for (int g = 0; g < OUT_COLS / 4; ++g) {
-                            if (col0 + 4 * g < N)
-                                dst[g] = make_int4(static_cast<int>(r[g >> 3][(4 * g) & 31]), static_cast<int>(r[g >> 3][(4 * g + 1) & 31]),
-                                                   static_cast<int>(r[g >> 3][(4 * g + 2) & 31]), static_cast<int>(r[g >> 3][(4 * g + 3) & 31]));
-                        }
-                    }
-                    // y = bf16(float(acc) * (x_scale * w_scale) + bias), eight columns per 16-byte chunk
-                    uint32_t packed[OUT_COLS / 2];
-#pragma unroll
-                    for (int g = 0; g < OUT_COLS / 4; ++g) {
-                        const int col = col0 + 4 * g;
-                        float4 ws = make_float4(0.f, 0.f, 0.f, 0.f);
-                        float b4[4] = {0.f, 0.f, 0.f, 0.f};
-                        if (col < N) {
-                            ws = __ldg(reinterpret_cast<const float4 *>(w_scale + col));
-                            if (bias != nullptr) {
-                                const uint2 bb = __ldg(reinterpret_cast<const uint2 *>(bias + col));
-                                b4[0] = __uint_as_float(bb.x << 16);
-                                b4[1] = __uint_as_float(bb.x & 0xFFFF0000u);
-                                b4[2] = __uint_as_float(bb.y << 16);
-                                b4[3] = __uint_as_float(bb.y & 0xFFFF0000u);
-                            }
-                        }
-                        const float wsv[4] = {ws.x, ws.y, ws.z, ws.w};
-                        float v[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = 4 * g + e;
-                            const float acc = __int2float_rn(static_cast<int>(r[j >> 5][j & 31]));
-                            v[e] = __fmul_rn(acc, __fmul_rn(xs, wsv[e]));
-                            if (bias != nullptr) v[e] = __fadd_rn(v[e], b4[e]);
-                        }
-                        packed[2 * g] = pack_bf16x2(v[0], v[1]);
-                        packed[2 * g + 1] = pack_bf16x2(v[2], v[3]);
-                    }
-                    // stage the 32 x 64 box in 128-byte-swizzled layout, then one TMA store
-                    uint8_t *sb = stage_buf + (nstores & 1) * OUT_BOX;
-                    if (lane == 0) bulk_wait_read_1();
-                    __syncwarp();
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int pos = q ^ (lane & 7);
-                        *reinterpret_cast<uint4 *>(sb + lane * 128 + pos * 16) =
-                            make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-                    }
-                    fence_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&tmY, smem_u32(sb), col0, row0);
-                        bulk_commit();
-                    }
-                    ++nstores;
-                }
-            }
+            const float xs_t = xs;
+            prefetch(t + gridDim.x);
+            epilogue_rows(tmem_base, quad, lane, static_cast<uint32_t>(buf * BN), m * BM + quad * 32, n * BN, xs_t, tab,
+                          bias != nullptr, acc_out, T, N, &tmY, stage_buf, nstores);
             tc_fence_before();
             mbar_arrive(tempty(buf));
         }
@@ -365,6 +512,200 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+}
+
+// ------------------------------------------------------------------------------------------------
+// 2-SM variant: a cluster of two CTAs computes a 256 x 256 tile with tcgen05.mma.cta_group::2
+// (M = 256, N = 256, K = 32). Each CTA loads its own 128 rows of A and 128 rows of B (the MMA reads
+// the peer's B half through the pair link), so every SM moves half the B bytes of the single-SM
+// kernel per MMA and a 6-stage ring fits in shared memory. Only the even CTA issues MMAs; every TMA
+// load of both CTAs completes on the even CTA's full barrier; each MMA batch is committed to the
+// empty barriers of both CTAs and each finished accumulator to both CTAs' tfull barriers; the odd
+// CTA's epilogue warps arrive remotely on the even CTA's tempty barrier.
+constexpr int P_STAGES = 6;
+constexpr int P_A_STAGE = BM * BK;          // 16 KB: this CTA's 128 token rows
+constexpr int P_B_STAGE = 128 * BK;         // 16 KB: this CTA's 128 of the tile's 256 channels
+constexpr int P_OFF_A = 0;
+constexpr int P_OFF_B = P_OFF_A + P_STAGES * P_A_STAGE;
+constexpr int P_OFF_OUT = P_OFF_B + P_STAGES * P_B_STAGE;
+constexpr int P_OFF_COL = P_OFF_OUT + EPI_WARPS * 2 * OUT_BOX;
+constexpr int P_OFF_BAR = P_OFF_COL + 2 * COL_TAB;
+constexpr int P_NBARS = 2 * P_STAGES + 5;
+constexpr int P_OFF_MISC = P_OFF_BAR + P_NBARS * 8;
+constexpr int P_SMEM_TOTAL = P_OFF_MISC + 16 + 1024;
+static_assert(P_SMEM_TOTAL <= 232448, "shared memory budget of one sm_100 CTA");
+constexpr uint32_t P_IDESC = make_idesc(2 * BM, BN);
+
+__global__ void __launch_bounds__(THREADS, 1)
+k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmY, const float *__restrict__ x_scale,
+                   const float *__restrict__ w_scale, const __nv_bfloat16 *__restrict__ bias,
+                   int32_t *__restrict__ acc_out, int T, int N, int K, int m_tiles, int n_tiles,
+                   uint64_t limit_ns)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem + P_OFF_A;
+    uint8_t *sB = smem + P_OFF_B;
+    uint8_t *sOut = smem + P_OFF_OUT;
+    float *sCol = reinterpret_cast<float *>(smem + P_OFF_COL);
+    const uint32_t bar0 = smem_u32(smem + P_OFF_BAR);
+    auto full = [&](int st) { return bar0 + 8u * st; };
+    auto empty = [&](int st) { return bar0 + 8u * (P_STAGES + st); };
+    auto tfull = [&](int b) { return bar0 + 8u * (2 * P_STAGES + b); };
+    auto tempty = [&](int b) { return bar0 + 8u * (2 * P_STAGES + 2 + b); };
+    const uint32_t done_bar = bar0 + 8u * (2 * P_STAGES + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + P_OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + P_OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();             // 0: issues the MMAs; 1: its peer
+    const int cid = blockIdx.x >> 1;
+    const int ncl = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < P_STAGES; ++st) { mbar_init(full(st), 1); mbar_init(empty(st), 1); }
+        for (int b = 0; b < 2; ++b) { mbar_init(tfull(b), 1); mbar_init(tempty(b), 2 * EPI_WARPS); }
+        mbar_init(done_bar, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+        fence_async_smem();
+    }
+    if (warp == 0 && lane == 0) { prefetch_map(&tmA); prefetch_map(&tmB); prefetch_map(&tmY); }
+    if (warp == 1) { tmem_alloc2(smem_u32(tmem_slot), TMEM_COLS); tmem_relinquish2(); }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();                                 // both CTAs' barriers exist before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int k_blocks = (K + BK - 1) / BK;
+    const int num_tiles = m_tiles * n_tiles;
+
+    if (warp == 0) {
+        // ---------------- TMA producer (both CTAs) ----------------
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            long long fills = 0;
+            bool ok = true;
+            for (int t = cid; t < num_tiles && ok; t += ncl) {
+                int m, n;
+                tile_coords(t, m_tiles, n_tiles, m, n);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait_cluster(empty(stage), phase ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
+                    if (rank == 0) mbar_expect_tx(full(stage), 2u * (P_A_STAGE + P_B_STAGE));
+                    const uint32_t fb = mapa_rank(full(stage), 0);
+                    tma_load_2d_pair(smem_u32(sA + stage * P_A_STAGE), &tmA, fb, kb * BK, m * 2 * BM + static_cast<int>(rank) * BM);
+                    tma_load_2d_pair(smem_u32(sB + stage * P_B_STAGE), &tmB, fb, kb * BK, n * BN + static_cast<int>(rank) * 128);
+                    ++fills;
+                    if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            if (!ok) give_up(abort_flag);
+            // The even CTA's full barriers count the bytes of both CTAs: once the last fill of every
+            // stage has completed there, no copy of either CTA is in flight.
+            if (rank == 0) {
+                for (int st = 0; st < P_STAGES; ++st) {
+                    if (fills <= st) break;
+                    const long long last = st + ((fills - 1 - st) / P_STAGES) * P_STAGES;
+                    if (!mbar_wait(full(st), static_cast<uint32_t>((last / P_STAGES) & 1), limit_ns, nullptr))
+                        record_status(SQ_ERR_TIMEOUT);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (even CTA only) ----------------
+        if (lane == 0 && rank == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            bool issued = false;
+            int lt = 0;
+            for (int t = cid; t < num_tiles && ok; t += ncl, ++lt) {
+                const int buf = lt & 1;
+                const uint32_t use = static_cast<uint32_t>(lt >> 1);
+                if (!mbar_wait_cluster(tempty(buf), (use & 1u) ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                for (int kb = 0; kb < k_blocks; ++kb) {
+                    if (!mbar_wait(full(stage), phase, limit_ns, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sA + stage * P_A_STAGE);
+                    const uint32_t b0 = smem_u32(sB + stage * P_B_STAGE);
+#pragma unroll
+                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                        mma_i8_pair(d_tmem, kmajor_sw128_desc(a0 + kk * UMMA_K), kmajor_sw128_desc(b0 + kk * UMMA_K), P_IDESC,
+                                    (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    issued = true;
+                    tc_commit2(mapa_rank(empty(stage), 0));
+                    tc_commit2(mapa_rank(empty(stage), 1));
+                    if (++stage == P_STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit2(mapa_rank(tfull(buf), 0));
+                tc_commit2(mapa_rank(tfull(buf), 1));
+            }
+            if (!ok) give_up(abort_flag);
+            if (issued) {
+                tc_commit2(mapa_rank(done_bar, 0));
+                if (!mbar_wait(done_bar, 0, limit_ns, nullptr)) record_status(SQ_ERR_TIMEOUT);
+            }
+        }
+    } else {
+        // ---------------- epilogue (both CTAs, each its 128 rows of the tile) ----------------
+        const int quad = warp & 3;
+        uint8_t *stage_buf = sOut + (warp - 2) * 2 * OUT_BOX;
+        const int ep = threadIdx.x - 64;
+        int nstores = 0;
+        int lt = 0;
+        ColShare cols;
+        float xs = 0.0f;
+        auto prefetch = [&](int t) {
+            if (t >= num_tiles) return;
+            int m, n;
+            tile_coords(t, m_tiles, n_tiles, m, n);
+            cols_fetch(cols, n * BN, ep, w_scale, bias, N);
+            const int row = m * 2 * BM + static_cast<int>(rank) * BM + quad * 32 + lane;
+            xs = row < T ? __ldg(x_scale + row) : 0.0f;
+        };
+        prefetch(cid);
+        for (int t = cid; t < num_tiles; t += ncl, ++lt) {
+            const int buf = lt & 1;
+            const uint32_t use = static_cast<uint32_t>(lt >> 1);
+            const bool ok = mbar_wait_cluster(tfull(buf), use & 1u, limit_ns, abort_flag);
+            float *tab = sCol + buf * (COL_TAB / 4);
+            if (ok) cols_store(cols, tab, ep);
+            if (named_sync_or(EPI_BAR, EPI_THREADS, !ok)) { give_up(abort_flag); break; }
+            tc_fence_after();
+            int m, n;
+            tile_coords(t, m_tiles, n_tiles, m, n);
+            const float xs_t = xs;
+            prefetch(t + ncl);
+            epilogue_rows(tmem_base, quad, lane, static_cast<uint32_t>(buf * BN),
+                          m * 2 * BM + static_cast<int>(rank) * BM + quad * 32, n * BN, xs_t, tab, bias != nullptr, acc_out,
+                          T, N, &tmY, stage_buf, nstores);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(mapa_rank(tempty(buf), 0));   // one arrival per warp, on the even CTA
+        }
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) {
+        // After a timeout the peer may still have copies in flight towards this pair's barriers;
+        // give them time to land (they need microseconds) before the pair leaves.
+        const uint64_t t0 = global_ns();
+        while (global_ns() - t0 < 50000ull) {}
+    }
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc2(tmem_base, TMEM_COLS);
 }
 
 // One thread waits, with the same bounded wait as the GEMM, on a barrier nothing completes.
@@ -401,13 +742,14 @@ sq_status get_encoder(EncodeTiledFn *out) {
 }
 
 sq_status encode_2d(EncodeTiledFn enc, CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner,
-                    uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, const char *what) {
+                    uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz,
+                    const char *what) {
     const cuuint64_t dims[2] = {inner, outer};
     const cuuint64_t strides[1] = {row_bytes};
     const cuuint32_t box[2] = {box_inner, box_outer};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                     swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return sq::fail(SQ_ERR_CUDA, "cuTensorMapEncodeTiled(%s) failed with CUresult %d", what, (int)r);
     return SQ_OK;
 }
@@ -455,11 +797,48 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, cons
     EncodeTiledFn enc = nullptr;
     sq_status st = get_encoder(&enc);
     if (st != SQ_OK) return st;
+    const bool pair = g_cta_pair.load(std::memory_order_relaxed) != 0 && T >= 2 * BM;   // 256-row tiles on CTA pairs
     CUtensorMap mA, mB, mY;
-    st = encode_2d(enc, &mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, T, K, BK, BM, "xq");
-    if (st == SQ_OK) st = encode_2d(enc, &mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, K, N, K, BK, BN, "wq");
-    if (st == SQ_OK) st = encode_2d(enc, &mY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, T, N * 2, OUT_COLS, OUT_ROWS, "y");
+    st = encode_2d(enc, &mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, T, K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B, "xq");
+    if (st == SQ_OK) st = encode_2d(enc, &mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, K, N, K, BK, pair ? 128 : BN, CU_TENSOR_MAP_SWIZZLE_128B, "wq");
+    if (st == SQ_OK) st = encode_2d(enc, &mY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, T, N * 2, OUT_COLS, OUT_ROWS, CU_TENSOR_MAP_SWIZZLE_64B, "y");
     if (st != SQ_OK) return st;
+    if (pair) {
+        static int pconfigured[64], pclusters[64];
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.blockDim = dim3(THREADS, 1, 1);
+        cfg.dynamicSmemBytes = P_SMEM_TOTAL;
+        cfg.stream = sq::as_stream(stream);
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (!pconfigured[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(k_w8a8_linear_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_TOTAL);
+            if (e != cudaSuccess) return sq::cuda_status(e, "cudaFuncSetAttribute(w8a8_linear_pair)");
+            cfg.gridDim = dim3(2, 1, 1);
+            int nc = 0;
+            e = cudaOccupancyMaxActiveClusters(&nc, k_w8a8_linear_pair, &cfg);
+            if (e != cudaSuccess) return sq::cuda_status(e, "cudaOccupancyMaxActiveClusters(w8a8_linear_pair)");
+            if (nc < 1) return sq::fail(SQ_ERR_CUDA, "no CTA pair of the GEMM fits on this device");
+            pclusters[dev] = nc;
+            pconfigured[dev] = 1;
+        }
+        const int m_tiles = static_cast<int>((T + 2 * BM - 1) / (2 * BM));
+        const int n_tiles = static_cast<int>((N + BN - 1) / BN);
+        const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
+        if (tiles > 0x7FFFFFFF) return fail(SQ_ERR_UNSUPPORTED, "sq_w8a8_linear: too many tiles");
+        const int clusters = static_cast<int>(tiles < pclusters[dev] ? tiles : pclusters[dev]);
+        cfg.gridDim = dim3(2 * clusters, 1, 1);
+        return sq::cuda_status(
+            cudaLaunchKernelEx(&cfg, k_w8a8_linear_pair, mA, mB, mY, x_scale, w_scale,
+                               reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out, static_cast<int>(T), static_cast<int>(N),
+                               static_cast<int>(K), m_tiles, n_tiles, sq::wait_timeout_ns(dev)),
+            "launch(w8a8_linear_pair)");
+    }
 
     static int configured[64];
     if (!configured[dev]) {
@@ -476,6 +855,12 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, cons
         mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out, static_cast<int>(T),
         static_cast<int>(N), static_cast<int>(K), m_tiles, n_tiles, sq::wait_timeout_ns(dev));
     return sq::cuda_status(cudaGetLastError(), "launch(w8a8_linear)");
+}
+
+sq_status sq_set_gemm_cta_pair(int enable) {
+    if (enable != 0 && enable != 1) return sq::fail(SQ_ERR_INVALID_ARG, "sq_set_gemm_cta_pair: enable must be 0 or 1");
+    g_cta_pair.store(enable, std::memory_order_relaxed);
+    return SQ_OK;
 }
 
 size_t sq_w8a8_linear_workspace_size(int64_t T, int64_t N, int64_t K) {

@@ -16,7 +16,7 @@ import torch
 __all__ = [
     "SQError", "lib", "sq_calibrate_absmax", "sq_compute_scales", "sq_smooth_quantize_weight",
     "sq_rmsnorm_smooth_quant", "sq_w8a8_linear", "sq_w8a8_linear_workspace_size", "sq_device_status",
-    "sq_set_wait_timeout_ns", "sq_selftest_wait_timeout", "sq_status_string", "sq_last_error",
+    "sq_set_wait_timeout_ns", "sq_selftest_wait_timeout", "sq_set_gemm_cta_pair", "sq_status_string", "sq_last_error",
     "sq_version", "LIB_PATH", "EXPORTS",
 ]
 
@@ -43,6 +43,7 @@ EXPORTS = {
     "sq_device_status": (_i, [_p]),
     "sq_set_wait_timeout_ns": (_i, [_u64]),
     "sq_selftest_wait_timeout": (_i, [_p]),
+    "sq_set_gemm_cta_pair": (_i, [_i]),
 }
 
 
@@ -215,6 +216,11 @@ def sq_device_status(stream=None) -> int:
 
 def sq_set_wait_timeout_ns(ns: int) -> None:
     _check(_lib.sq_set_wait_timeout_ns(int(ns)), "sq_set_wait_timeout_ns")
+
+
+def sq_set_gemm_cta_pair(enable: bool) -> None:
+    """Selects the GEMM form for later calls: CTA pairs (True) or one SM per tile (False, default)."""
+    _check(_lib.sq_set_gemm_cta_pair(1 if enable else 0), "sq_set_gemm_cta_pair")
 
 
 def sq_selftest_wait_timeout(stream=None) -> None:

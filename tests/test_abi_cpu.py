@@ -59,6 +59,14 @@ def test_workspace_size_is_zero(sqmod):
     assert sqmod.sq_w8a8_linear_workspace_size(8192, 4096, 4096) == 0
 
 
+def test_gemm_form_setter_checks_its_argument(sqmod):
+    L = sqmod._lib
+    assert L.sq_set_gemm_cta_pair(2) == 1            # SQ_ERR_INVALID_ARG
+    assert L.sq_set_gemm_cta_pair(-1) == 1
+    assert L.sq_set_gemm_cta_pair(1) == 0
+    assert L.sq_set_gemm_cta_pair(0) == 0            # back to the default
+
+
 # Argument checks run before any CUDA call, so they behave the same with or without a GPU.
 FAKE = 0x10000   # a 16-byte aligned address that is never dereferenced
 

@@ -235,6 +235,37 @@ def test_absmax_strided_rows_and_empty(sq, orc):
     ok_status(sq)
 
 
+# The CTA-pair GEMM (cta_group::2, 256 x 256 tiles) against the single-SM form and the oracle:
+# ragged T and N, K not a multiple of the 128-byte stage, bias on and off, and T below 256 (which
+# keeps the single-SM form even when pairs are enabled).
+PAIR_SHAPES = [(256, 256, 128, False), (300, 520, 272, True), (777, 1288, 2064, True), (1024, 4096, 4096, False),
+               (200, 264, 512, True)]
+
+
+@pytest.mark.parametrize("T,N,K,bias", PAIR_SHAPES)
+def test_cta_pair_gemm_matches(sq, orc, T, N, K, bias):
+    dev = "cuda"
+    g = torch.Generator(device="cpu").manual_seed(T + 3 * N + 7 * K)
+    xq = torch.randint(-127, 128, (T, K), dtype=torch.int8, generator=g).to(dev)
+    wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, generator=g).to(dev)
+    xs = (torch.rand(T, generator=g) * 1e-2).to(dev)
+    ws = (torch.rand(N, generator=g) * 1e-2).to(dev)
+    b = (torch.randn(N, generator=g)).to(torch.bfloat16).to(dev) if bias else None
+    outs = []
+    try:
+        for pair in (False, True):
+            sq.sq_set_gemm_cta_pair(pair)
+            acc = torch.empty(T, N, dtype=torch.int32, device=dev)
+            y = sq.sq_w8a8_linear(xq, xs, wq, ws, bias=b, acc_out=acc)
+            ok_status(sq)
+            outs.append((y, acc))
+    finally:
+        sq.sq_set_gemm_cta_pair(False)
+    assert torch.equal(outs[0][1], outs[1][1]) and torch.equal(outs[0][0], outs[1][0])
+    rows = sample_indices(T, 24, T)
+    check_linear(sq, orc, xq, xs, wq, ws, b, outs[1][0], outs[1][1], rows=rows)
+
+
 def test_deterministic_bytes(sq):
     w = synth.WORKLOADS[1]
     d = synth.group_inputs(w, 0, "cuda", T=1000)
