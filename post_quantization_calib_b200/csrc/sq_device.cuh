@@ -71,6 +71,12 @@ static __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, u
                  : "memory");
 }
 
+// Orders this thread's earlier shared-memory accesses (generic proxy) before its later TMA
+// (async proxy) accesses to shared memory.
+static __device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------------- barriers
 static __device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -9,33 +9,38 @@
 //   [W8A8]    "SmoothQuant and W8A8: Quantizing Activations Too"
 //
 // Design (B200). One kernel template serves the abs-max (MODE_ABSMAX) and the quantisers
-// (MODE_QUANT). A CTA of 8 warps is split into row groups of 1, 2, 4 or 8 warps (enough lanes to hold
-// one row of up to 16384 bf16 in registers, 64 per lane). Each group streams its own rows through a
-// 2-6 slot shared-memory ring filled by TMA bulk copies (one 1-D copy per row, completion on an
-// mbarrier), so several rows per group are in flight while the group computes on the current one.
-// Per row, the group's lanes hold the row in registers; reductions are warp shuffles plus, for
-// groups of several warps, one named barrier that also releases the ring slot.
+// (MODE_QUANT). A CTA (one per SM) has 16 warps, 4 per scheduler. Rows of up to 2048 elements are
+// handled by a single warp each, wider rows by row groups of 2, 4 or 8 warps; narrower rows are
+// batched R at a time, so that a unit always gives a lane 8 vectors of 8 elements (64 element-rows)
+// against a fixed per-unit cost. Each row group streams its units through its own shared-memory ring
+// of 2-4 slots, filled with TMA bulk copies (one 1-D copy per row, completion on an mbarrier): as
+// soon as the group has read a slot for the last time, its leader lane issues the copies of the unit
+// that goes there next, so two or more units per group are in flight while the group computes on the
+// current one. There is no separate producer warp, so all 16 warps compute.
+//
+// Per unit, sums and maxima of the R rows are reduced across the warp with one butterfly that
+// halves the number of values at each exchange, so a lane ends up with the total of one row; the
+// per-row scalar steps (1/rms, the quantisation step and its reciprocal) then run once, in parallel
+// across lanes, and are broadcast with shuffles.
 //
 // Instruction budget. These kernels must retire about 8-12 bf16 elements per SM cycle to keep up
-// with HBM, so each element gets only a dozen instructions and none on the quarter-rate conversion
-// pipe:
+// with HBM, so each element gets only a few instructions:
 //   * the RMSNorm sum of squares is binary64, but each operand is built with integer operations:
 //     the bf16 exponent and mantissa are placed in the binary64 fields with exponent bias +485, which
 //     is exactly x * 2^-411 for every normal |x| >= 2^-100 (and a zero becomes 2^-538, whose square
 //     2^-1076 rounds away inside the fused multiply-add); the binary64 accumulator is rescaled by
 //     2^822 at the end. Squares of |x| < 2^-100 (and of subnormal bf16) are not exact; they are
 //     below 2^-200 and cannot move a binary32 result unless the whole row is that small.
-//   * INT8 codes use round-toward-zero adds instead of conversions: r = rz(|t| + 0.5) and
-//     w = rz(r + 2^23) give 2^23 + round_half_away(|t|) exactly; the sign is applied with one exact
-//     fused multiply-add that leaves the two's-complement code in the low byte of the result.
-//     |t| <= fl(m * fl(127/m)) <= 127.00001, so the code never leaves [-127, 127].
+//   * INT8 codes: v = rz(t + copysign(1/2, t)) (round toward zero cannot carry the sum across an
+//     integer), then a truncating conversion gives round_half_away(t); |t| <= fl(m * fl(127/m))
+//     <= 127.00001, so the code never leaves [-127, 127].
 //   * pairs of binary32 values use the packed f32x2 instructions of sm_100.
 // Arithmetic otherwise follows the RMSNorm / quantiser definitions step by step with explicit
 // round-to-nearest operations (nothing is contracted into fused multiply-adds), so results are
 // bit-identical to the definitions.
 //
-// The column abs-max keeps per-column running maxima in registers, combines the groups of a CTA in
-// shared memory and the 8 CTAs of a thread-block cluster through distributed shared memory, then
+// The column abs-max keeps per-column running maxima in registers, combines the warps of a CTA in
+// shared memory and the CTAs of a thread-block cluster through distributed shared memory, then
 // issues one atomic max per column per cluster. For a norm-fed input the maximum of
 // fl(fl(|x| * inv_rms) * |gamma|) over rows equals fl(max(fl(|x| * inv_rms)) * |gamma|) because
 // rounding is monotone, so gamma is applied once per column at the end.
@@ -56,10 +61,11 @@ constexpr float kFloor = 1e-5f;   // floor of abs-maxima and of s ([TAMING] list
 constexpr float kQmax = 127.0f;   // symmetric INT8 range [-127, 127]
 constexpr int kMaxCluster = 8;    // largest cluster tried for the column abs-max
 constexpr int kMaxK = 16384;      // widest row held on chip by the row kernels
-constexpr int kWarps = 8;                   // consumer warps per CTA
-constexpr int kThreads = 32 * (kWarps + 1); // plus one producer warp
-constexpr int kMaxStages = 6;
+constexpr int kWarps = 16;                  // warps per CTA
+constexpr int kThreads = 32 * kWarps;
+constexpr int kMaxStages = 4;
 constexpr uint32_t kSqBias = 485u << 20;   // binary64 exponent bias mapping bf16 x to x * 2^-411
+constexpr unsigned kAll = 0xFFFFFFFFu;
 
 enum { MODE_ABSMAX = 0, MODE_QUANT = 1 };
 
@@ -88,45 +94,77 @@ __device__ __forceinline__ float inv_rms(double ss, int K, double inv_k, float e
     return __frcp_rn(r);
 }
 
-__device__ __forceinline__ double warp_sum(double v) {
+// Butterfly reduction of R per-lane values (one per row of a unit) across the warp. Each exchange
+// halves the number of values a lane holds; when one is left the remaining exchanges are plain.
+// Afterwards every lane holds the total of row (lane / (32 / R)).
+template <int R>
+__device__ __forceinline__ double rows_sum(double (&v)[R], int lane) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    return v;
+    for (int step = 0; step < 5; ++step) {
+        const int o = 16 >> step;
+        const int n = R >> step;
+        if (n >= 2) {
+            const bool up = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < n / 2; ++i) {
+                const double send = up ? v[i] : v[i + n / 2];
+                const double keep = up ? v[i + n / 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(kAll, send, o);
+            }
+        } else {
+            v[0] += __shfl_xor_sync(kAll, v[0], o);
+        }
+    }
+    return v[0];
 }
 
-__device__ __forceinline__ float warp_max(float v) {
+template <int R>
+__device__ __forceinline__ float rows_max(float (&v)[R], int lane) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-    return v;
+    for (int step = 0; step < 5; ++step) {
+        const int o = 16 >> step;
+        const int n = R >> step;
+        if (n >= 2) {
+            const bool up = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < n / 2; ++i) {
+                const float send = up ? v[i] : v[i + n / 2];
+                const float keep = up ? v[i + n / 2] : v[i];
+                v[i] = fmaxf(keep, __shfl_xor_sync(kAll, send, o));
+            }
+        } else {
+            v[0] = fmaxf(v[0], __shfl_xor_sync(kAll, v[0], o));
+        }
+    }
+    return v[0];
 }
 
-// Adds the squares of the two bf16 values of `w` to the scaled binary64 accumulator.
-__device__ __forceinline__ double add_squares(uint32_t w, double ss) {
-    const double a_hi = __hiloint2double(static_cast<int>(mad_hi(w & 0x7FFF0000u, 1u << 29, kSqBias)), 0);
-    const double a_lo = __hiloint2double(static_cast<int>((w & 0x7FFFu) * 8192u + kSqBias), 0);
-    ss = __fma_rn(a_hi, a_hi, ss);
-    return __fma_rn(a_lo, a_lo, ss);
+// Adds the squares of the two bf16 values of `w` to the scaled binary64 accumulators a and b.
+__device__ __forceinline__ void add_squares(uint32_t w, double &a, double &b) {
+    const double d_hi = __hiloint2double(static_cast<int>(mad_hi(w & 0x7FFF0000u, 1u << 29, kSqBias)), 0);
+    const double d_lo = __hiloint2double(static_cast<int>((w & 0x7FFFu) * 8192u + kSqBias), 0);
+    a = __fma_rn(d_hi, d_hi, a);
+    b = __fma_rn(d_lo, d_lo, b);
 }
 
 __device__ __forceinline__ uint32_t word_of(const uint4 &v, int k) {
     return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
 }
 
-// Signed INT8 codes of the two values of `y` (scaled by inv): the code of the low element in the
-// low byte, of the high element in the next byte.
-__device__ __forceinline__ uint32_t codes2(uint64_t y, uint64_t inv2) {
-    const uint64_t t = mul2_rn(y, inv2);
+// bf16 pair -> packed binary32 pair (exact)
+__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) { return pack2u(w << 16, w & 0xFFFF0000u); }
+
+// Signed INT8 codes of the two values of t: round half away from zero. v = rz(t + copysign(1/2, t))
+// has the integer part of the exactly rounded value, and the conversion truncates it.
+__device__ __forceinline__ uint32_t codes2(uint64_t t) {
     uint32_t tl, th;
     unpack2(t, tl, th);
-    const uint64_t sgn = pack2u((tl & 0x80000000u) | 0x3F800000u, (th & 0x80000000u) | 0x3F800000u);   // +-1
-    const uint64_t at = mul2_rn(t, sgn);                                                  // |t|
-    const uint64_t r = add2_rz(at, pack2(0.5f, 0.5f));                                    // rz(|t| + 1/2)
-    const uint64_t w = add2_rz(r, pack2(8388608.0f, 8388608.0f));                         // 2^23 + q
-    const uint64_t qm = add2_rn(w, pack2(-8388736.0f, -8388736.0f));                      // q - 128
-    const uint64_t f = fma2_rn(sgn, qm, pack2(8388736.0f, 8388736.0f));                   // 2^23 + 128 +- (q - 128)
-    uint32_t fl, fh;
-    unpack2(f, fl, fh);
-    return __byte_perm(fl, fh, 0x0040);
+    const uint64_t half = pack2u((tl & 0x80000000u) | 0x3F000000u, (th & 0x80000000u) | 0x3F000000u);
+    uint32_t vl, vh;
+    unpack2(add2_rz(t, half), vl, vh);
+    const int ql = __float2int_rz(__uint_as_float(vl));
+    const int qh = __float2int_rz(__uint_as_float(vh));
+    return __byte_perm(static_cast<uint32_t>(ql), static_cast<uint32_t>(qh), 0x0040);   // bytes: ql, qh in 0, 1
 }
 
 // 3-input maximum (one instruction on sm_100)
@@ -136,59 +174,64 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return d;
 }
 
-// One CTA = 8 consumer warps in row groups of WPR warps + 1 producer warp. A group processes units of
-// R consecutive rows; lane l of warp w of the group holds 8-element vectors v = i * 32 * WPR +
-// 32 * w + l (i < VPL) of every row of the unit.
+// One CTA = 16 warps in row groups of WPR warps. A group processes units of R consecutive rows; lane l
+// of warp w of the group covers the 8-element vectors v = i * 32 * WPR + 32 * w + l (i < VPL) of
+// every row of the unit. R > 1 only with WPR == 1.
 template <int WPR, int VPL, int R, int MODE, bool NORM, bool FULL>
-__global__ void __launch_bounds__(kThreads, 2) k_rows(const RowArgs p)
+__global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
 {
     constexpr int G = kWarps / WPR;   // row groups per CTA
     constexpr int GT = 32 * WPR;      // consumer threads per row group
+    constexpr int SUB = 32 / R;       // lanes that hold one row's total after a butterfly
+    static_assert(R == 1 || WPR == 1, "several rows per unit only with one warp per row");
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[G * kMaxStages];
-    __shared__ __align__(8) uint64_t s_empty[G * kMaxStages];
-    __shared__ double s_ss[2][kWarps][R];
-    __shared__ float s_mx[2][kWarps][R];
+    __shared__ double s_ss[2][kWarps];
+    __shared__ float s_mx[2][kWarps];
     __shared__ int s_abort[G];
-    __shared__ long long s_consumed[G];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const bool producer = warp == kWarps;                 // the last warp refills the rings
-    const int group = producer ? lane : warp / WPR;        // producer lane g serves group g
+    const int group = warp / WPR;
     const int wig = warp % WPR, gtid = wig * 32 + lane;
-    const bool leader = !producer && gtid == 0;
+    const bool leader = gtid == 0;
     const int K = p.K, nvec = K >> 3;
     const uint32_t rowbytes = static_cast<uint32_t>(K) * 2u;
     const uint32_t slotbytes = rowbytes * R;
     const int stages = p.stages;
     uint8_t *ring = smem;
     const size_t ring_bytes = static_cast<size_t>(G) * stages * slotbytes;
-    float4 *c_lo = reinterpret_cast<float4 *>(smem + ring_bytes);   // c[8v .. 8v+3]
-    float4 *c_hi = c_lo + nvec;                                     // c[8v+4 .. 8v+7]
+    const size_t red_bytes = MODE == MODE_ABSMAX ? static_cast<size_t>(G) * K * 4 : 0;
+    float4 *c_lo = reinterpret_cast<float4 *>(smem + (ring_bytes > red_bytes ? ring_bytes : red_bytes));   // c[8v .. 8v+3]
+    float4 *c_hi = c_lo + nvec;                                                                              // c[8v+4 .. 8v+7]
+    const bool has_vec = p.vec != nullptr;
 
     const int64_t units = (p.rows + R - 1) / R;
     const int64_t g0 = static_cast<int64_t>(blockIdx.x) * G + group;
     const int64_t gstride = static_cast<int64_t>(gridDim.x) * G;
-    const int64_t nunits = (group < G && g0 < units) ? (units - 1 - g0) / gstride + 1 : 0;
+    const int64_t nunits = g0 < units ? (units - 1 - g0) / gstride + 1 : 0;
 
     if (tid == 0) {
-        for (int i = 0; i < G * stages; ++i) {
-            mbar_init(smem_u32(&s_full[i]), 1);
-            mbar_init(smem_u32(&s_empty[i]), WPR);
-        }
-        for (int g = 0; g < G; ++g) { s_abort[g] = 0; s_consumed[g] = 0; }
+        for (int i = 0; i < G * stages; ++i) mbar_init(smem_u32(&s_full[i]), 1);
+        for (int g = 0; g < G; ++g) s_abort[g] = 0;
         mbar_init_fence();
     }
-    if (MODE == MODE_QUANT && p.vec != nullptr) {
+    if (MODE == MODE_QUANT && has_vec) {
         const float4 *cv = reinterpret_cast<const float4 *>(p.vec);
         for (int v = tid; v < nvec; v += kThreads) { c_lo[v] = __ldg(cv + 2 * v); c_hi[v] = __ldg(cv + 2 * v + 1); }
     }
     __syncthreads();
 
-    auto slot = [&](int s) { return ring + (static_cast<size_t>(group) * stages + s) * slotbytes; };
-    auto full_bar = [&](int s) { return smem_u32(&s_full[group * stages + s]); };
-    auto empty_bar = [&](int s) { return smem_u32(&s_empty[group * stages + s]); };
-    volatile int *abort_flag = &s_abort[group < G ? group : 0];
+    auto slot = [&](int st) { return ring + (static_cast<size_t>(group) * stages + st) * slotbytes; };
+    auto full_bar = [&](int st) { return smem_u32(&s_full[group * stages + st]); };
+    volatile int *abort_flag = &s_abort[group];
+    // Leader only: the copies of unit j (nr rows) into slot st, counted on its full barrier.
+    auto issue = [&](int64_t j, int st) {
+        const int64_t r0 = (g0 + j * gstride) * R;
+        const int nr = static_cast<int>(p.rows - r0 < R ? p.rows - r0 : R);
+        mbar_expect_tx(full_bar(st), rowbytes * static_cast<uint32_t>(nr));
+        for (int r = 0; r < nr; ++r)
+            bulk_g2s(smem_u32(slot(st) + r * rowbytes), p.src + (r0 + r) * p.ld_bytes, rowbytes, full_bar(st));
+    };
 
     float mx[VPL][8];          // ABSMAX with norm: running max of fl(|x| * inv_rms) per column
     uint32_t mh[VPL][4];       // ABSMAX without norm: running max of |x| as bf16 pairs
@@ -200,134 +243,120 @@ __global__ void __launch_bounds__(kThreads, 2) k_rows(const RowArgs p)
         for (int k = 0; k < 4; ++k) mh[i][k] = 0u;
     }
 
-    int64_t issued = 0;
+    int64_t issued = 0, consumed = 0;
     bool failed = false;
-    if (producer) {
-        // Lane g keeps group g's ring full: a slot is refilled as soon as the group's warps have
-        // released it, independently of the group's progress on later units.
-        if (lane < G) {
-            int s = 0;
-            uint32_t phase = 0;
-            for (int64_t j = 0; j < nunits; ++j) {
-                if (!mbar_ready(empty_bar(s), phase ^ 1u, p.limit_ns, abort_flag)) {
-                    if (!*abort_flag) failed = true;
-                    *abort_flag = 1;
-                    break;
-                }
-                const int64_t r0 = (g0 + j * gstride) * R;
-                const int nr = static_cast<int>(p.rows - r0 < R ? p.rows - r0 : R);
-                mbar_expect_tx(full_bar(s), rowbytes * static_cast<uint32_t>(nr));
-                for (int r = 0; r < nr; ++r)
-                    bulk_g2s(smem_u32(slot(s) + r * rowbytes), p.src + (r0 + r) * p.ld_bytes, rowbytes, full_bar(s));
-                issued = j + 1;
-                if (++s == stages) { s = 0; phase ^= 1u; }
-            }
+    if (leader) {
+        issued = nunits < stages ? nunits : stages;
+        for (int64_t j = 0; j < issued; ++j) issue(j, static_cast<int>(j));
+    }
+    // Leader only, after the group's last read of slot st (unit j): refill it with unit j + stages.
+    auto refill = [&](int64_t j, int st) {
+        if (j + stages < nunits && !*abort_flag) {
+            fence_proxy_async_smem();
+            issue(j + stages, st);
+            issued = j + stages + 1;
         }
-    } else {
-        int64_t consumed = 0;
-        int s = 0;
+    };
+    {
+        int st = 0;
         uint32_t phase = 0;
+        const int rv = static_cast<int>(rowbytes / 16);   // vectors per row in a slot
         for (int64_t j = 0; j < nunits; ++j) {
-            const bool ok = mbar_ready(full_bar(s), phase, p.limit_ns, abort_flag);
+            const bool ok = mbar_ready(full_bar(st), phase, p.limit_ns, abort_flag);
             const int64_t r0 = (g0 + j * gstride) * R;
             const int nr = static_cast<int>(p.rows - r0 < R ? p.rows - r0 : R);   // uniform in the group
-            const uint4 *rp = reinterpret_cast<const uint4 *>(slot(s));
-            const int rv = static_cast<int>(rowbytes / 16);                           // vectors per row
-            double ss[R];
-#pragma unroll
-            for (int r = 0; r < R; ++r) ss[r] = 0.0;
-            if (NORM) {
-#pragma unroll
-                for (int r = 0; r < R; ++r) {
-                    if (r < nr) {
-                        double a = 0.0, b = 0.0;
-#pragma unroll
-                        for (int i = 0; i < VPL; ++i) {
-                            const int v = i * GT + gtid;
-                            const uint4 q = (ok && (FULL || v < nvec)) ? rp[r * rv + v] : make_uint4(0u, 0u, 0u, 0u);
-                            a = add_squares(q.x, a);
-                            b = add_squares(q.y, b);
-                            a = add_squares(q.z, a);
-                            b = add_squares(q.w, b);
-                        }
-                        ss[r] = warp_sum(a + b);
-                    }
-                }
-            }
-            // Group-wide step: partial sums become visible, and a failed wait anywhere in the group
-            // stops the whole group at the same unit.
+            const uint4 *rp = reinterpret_cast<const uint4 *>(slot(st));
+            // a failed wait anywhere in the group stops the whole group at the same unit
             bool any_fail;
-            if (WPR == 1) {
-                any_fail = __any_sync(0xFFFFFFFFu, !ok);
-            } else {
-                if (NORM && lane == 0) {
-#pragma unroll
-                    for (int r = 0; r < R; ++r) s_ss[j & 1][warp][r] = ss[r];
-                }
-                any_fail = named_sync_or(1 + group, GT, !ok);
-                if (NORM) {
-#pragma unroll
-                    for (int r = 0; r < R; ++r) {
-                        double t = 0.0;
-#pragma unroll
-                        for (int w = 0; w < WPR; ++w) t += s_ss[j & 1][group * WPR + w][r];
-                        ss[r] = t;
-                    }
-                }
-            }
+            if (WPR == 1) any_fail = __any_sync(kAll, !ok);
+            else any_fail = named_sync_or(1 + group, GT, !ok);
             if (any_fail) {
                 if (leader) { if (!*abort_flag) failed = true; *abort_flag = 1; }
                 break;
             }
-            uint64_t ir2[R];
+
+            // ---- pass A: the unit's rows into registers (QUANT) and the sums of squares (NORM)
+            uint4 xr[R][VPL];
+            double ssr[R];
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                const float ir = NORM ? inv_rms(__dmul_rn(ss[r], 0x1p822), K, p.inv_k, p.eps) : 1.0f;
-                ir2[r] = pack2(ir, ir);
-            }
-
-            if (MODE == MODE_ABSMAX) {
+                double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
 #pragma unroll
                 for (int i = 0; i < VPL; ++i) {
                     const int v = i * GT + gtid;
-                    const bool in = FULL || v < nvec;
-                    uint4 q[R];
+                    const bool in = (FULL || v < nvec) && r < nr;
+                    if (MODE == MODE_ABSMAX && !NORM) continue;
+                    const uint4 q = in ? rp[r * rv + v] : make_uint4(0u, 0u, 0u, 0u);
+                    if (MODE == MODE_QUANT) xr[r][i] = q;
+                    if (NORM) {
+                        if (i & 1) { add_squares(q.x, a2, a3); add_squares(q.y, a2, a3); add_squares(q.z, a2, a3); add_squares(q.w, a2, a3); }
+                        else { add_squares(q.x, a0, a1); add_squares(q.y, a0, a1); add_squares(q.z, a0, a1); add_squares(q.w, a0, a1); }
+                    }
+                }
+                ssr[r] = (a0 + a1) + (a2 + a3);
+            }
+            if (MODE == MODE_QUANT) {
+                // the unit is in registers now: the slot can be refilled
+                if (WPR == 1) { __syncwarp(); if (leader) refill(j, st); }
+                else if (!NORM) { named_sync(1 + group, GT); if (leader) refill(j, st); }
+            }
+
+            // ---- 1 / rms of every row of the unit, broadcast to all lanes
+            float ir[R];
+            if (NORM) {
+                double ss = rows_sum<R>(ssr, lane);             // total of row lane / SUB
+                if (WPR > 1) {
+                    if (lane == 0) s_ss[j & 1][warp] = ss;
+                    named_sync(1 + group, GT);
+                    if (MODE == MODE_QUANT && leader) refill(j, st);   // every warp has read the slot
+                    ss = 0.0;
 #pragma unroll
-                    for (int r = 0; r < R; ++r) q[r] = (in && r < nr) ? rp[r * rv + v] : make_uint4(0u, 0u, 0u, 0u);
+                    for (int w = 0; w < WPR; ++w) ss += s_ss[j & 1][group * WPR + w];
+                }
+                const float mine = inv_rms(__dmul_rn(ss, 0x1p822), K, p.inv_k, p.eps);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
+                for (int r = 0; r < R; ++r) ir[r] = __shfl_sync(kAll, mine, r * SUB);
+            } else {
+#pragma unroll
+                for (int r = 0; r < R; ++r) ir[r] = 1.0f;
+            }
+
+            if (MODE == MODE_ABSMAX) {
+                // ---- pass B: running column maxima
+#pragma unroll
+                for (int i = 0; i < VPL; ++i) {
+                    const int v = i * GT + gtid;
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        if (!((FULL || v < nvec) && r < nr)) continue;
                         if (NORM) {
-                            float yl[R], yh[R];
+                            const uint64_t ir2 = pack2(ir[r], ir[r]);
+                            const uint4 q = rp[r * rv + v];
 #pragma unroll
-                            for (int r = 0; r < R; ++r) {
-                                const uint32_t w = word_of(q[r], k);
+                            for (int k = 0; k < 4; ++k) {
                                 uint32_t l, h;
-                                unpack2(mul2_rn(pack2u(w << 16, w & 0xFFFF0000u), ir2[r]), l, h);
-                                yl[r] = fabsf(__uint_as_float(l));
-                                yh[r] = fabsf(__uint_as_float(h));
-                            }
-                            if (R == 2) {
-                                mx[i][2 * k] = max3f(mx[i][2 * k], yl[0], yl[R - 1]);
-                                mx[i][2 * k + 1] = max3f(mx[i][2 * k + 1], yh[0], yh[R - 1]);
-                            } else {
-                                mx[i][2 * k] = fmaxf(mx[i][2 * k], yl[0]);
-                                mx[i][2 * k + 1] = fmaxf(mx[i][2 * k + 1], yh[0]);
+                                unpack2(mul2_rn(bf2_to_f2(word_of(q, k)), ir2), l, h);
+                                mx[i][2 * k] = fmaxf(mx[i][2 * k], fabsf(__uint_as_float(l)));
+                                mx[i][2 * k + 1] = fmaxf(mx[i][2 * k + 1], fabsf(__uint_as_float(h)));
                             }
                         } else {
+                            const uint4 q = rp[r * rv + v];
 #pragma unroll
-                            for (int r = 0; r < R; ++r) {
+                            for (int k = 0; k < 4; ++k) {
                                 __nv_bfloat162 cur = *reinterpret_cast<__nv_bfloat162 *>(&mh[i][k]);
-                                const uint32_t a = word_of(q[r], k) & 0x7FFF7FFFu;
+                                const uint32_t a = word_of(q, k) & 0x7FFF7FFFu;
                                 cur = __hmax2(cur, *reinterpret_cast<const __nv_bfloat162 *>(&a));
                                 mh[i][k] = *reinterpret_cast<uint32_t *>(&cur);
                             }
                         }
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));      // this warp is done with the slot
+                // this group is done with the slot
+                if (WPR == 1) __syncwarp();
+                else named_sync(1 + group, GT);
+                if (leader) refill(j, st);
             } else {
-                // y = (x * inv_rms) * c  (or x * c, or x), kept in registers as element pairs
+                // ---- pass B: y = (x * inv_rms) * c  (or x * c, or x) as element pairs, row maxima
                 uint64_t y[R][VPL][4];
                 float m[R];
 #pragma unroll
@@ -337,16 +366,15 @@ __global__ void __launch_bounds__(kThreads, 2) k_rows(const RowArgs p)
                     const int v = i * GT + gtid;
                     const bool in = FULL || v < nvec;
                     float4 cl = make_float4(1.f, 1.f, 1.f, 1.f), ch = cl;
-                    if (p.vec != nullptr && in) { cl = c_lo[v]; ch = c_hi[v]; }
+                    if (has_vec && in) { cl = c_lo[v]; ch = c_hi[v]; }
                     const uint64_t c2[4] = {pack2(cl.x, cl.y), pack2(cl.z, cl.w), pack2(ch.x, ch.y), pack2(ch.z, ch.w)};
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
-                        const uint4 q = (in && r < nr) ? rp[r * rv + v] : make_uint4(0u, 0u, 0u, 0u);
+                        const uint64_t ir2 = pack2(ir[r], ir[r]);
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            const uint32_t w = word_of(q, k);
-                            const uint64_t x2 = pack2u(w << 16, w & 0xFFFF0000u);
-                            const uint64_t yy = NORM ? mul2_rn(mul2_rn(x2, ir2[r]), c2[k]) : (p.vec != nullptr ? mul2_rn(x2, c2[k]) : x2);
+                            const uint64_t x2 = bf2_to_f2(word_of(xr[r][i], k));
+                            const uint64_t yy = NORM ? mul2_rn(mul2_rn(x2, ir2), c2[k]) : (has_vec ? mul2_rn(x2, c2[k]) : x2);
                             y[r][i][k] = yy;
                             uint32_t yl, yh;
                             unpack2(yy, yl, yh);
@@ -354,63 +382,55 @@ __global__ void __launch_bounds__(kThreads, 2) k_rows(const RowArgs p)
                         }
                     }
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty_bar(s));      // the unit is in registers now
-#pragma unroll
-                for (int r = 0; r < R; ++r) m[r] = warp_max(m[r]);
+                float mrow = rows_max<R>(m, lane);               // maximum of row lane / SUB
                 if (WPR > 1) {
-                    if (lane == 0) {
-#pragma unroll
-                        for (int r = 0; r < R; ++r) s_mx[j & 1][warp][r] = m[r];
-                    }
+                    if (lane == 0) s_mx[j & 1][warp] = mrow;
                     named_sync(1 + group, GT);
+                    mrow = 0.0f;
 #pragma unroll
-                    for (int r = 0; r < R; ++r) {
-                        float t = 0.0f;
-#pragma unroll
-                        for (int w = 0; w < WPR; ++w) t = fmaxf(t, s_mx[j & 1][group * WPR + w][r]);
-                        m[r] = t;
-                    }
+                    for (int w = 0; w < WPR; ++w) mrow = fmaxf(mrow, s_mx[j & 1][group * WPR + w]);
                 }
+                // step and reciprocal of the row this lane holds; one lane per row stores the step
+                const float delta = mrow > 0.0f ? __fdiv_rn(mrow, kQmax) : 0.0f;
+                const float inv_m = mrow > 0.0f ? __fdiv_rn(kQmax, mrow) : 0.0f;
+                if (wig == 0 && (lane % SUB) == 0 && lane / SUB < nr) p.scale[r0 + lane / SUB] = delta;
+                // ---- pass C: codes
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
+                    const float iv = __shfl_sync(kAll, inv_m, r * SUB);
                     if (r < nr) {
-                        const float delta = m[r] > 0.0f ? __fdiv_rn(m[r], kQmax) : 0.0f;
-                        const float inv = m[r] > 0.0f ? __fdiv_rn(kQmax, m[r]) : 0.0f;
-                        const uint64_t inv2 = pack2(inv, inv);
+                        const uint64_t inv2 = pack2(iv, iv);
                         uint2 *qrow = reinterpret_cast<uint2 *>(p.q + (r0 + r) * static_cast<int64_t>(K));
 #pragma unroll
                         for (int i = 0; i < VPL; ++i) {
                             const int v = i * GT + gtid;
                             if (FULL || v < nvec) {
-                                const uint32_t c01 = codes2(y[r][i][0], inv2), c23 = codes2(y[r][i][1], inv2);
-                                const uint32_t c45 = codes2(y[r][i][2], inv2), c67 = codes2(y[r][i][3], inv2);
+                                const uint32_t c01 = codes2(mul2_rn(y[r][i][0], inv2)), c23 = codes2(mul2_rn(y[r][i][1], inv2));
+                                const uint32_t c45 = codes2(mul2_rn(y[r][i][2], inv2)), c67 = codes2(mul2_rn(y[r][i][3], inv2));
                                 qrow[v] = make_uint2(__byte_perm(c01, c23, 0x5410), __byte_perm(c45, c67, 0x5410));
                             }
                         }
-                        if (leader) p.scale[r0 + r] = delta;
                     }
                 }
             }
             consumed = j + 1;
-            if (++s == stages) { s = 0; phase ^= 1u; }
+            if (++st == stages) { st = 0; phase ^= 1u; }
         }
-        if (leader) s_consumed[group] = consumed;
     }
 
     if (failed) atomicCAS(p.status, 0u, static_cast<unsigned int>(SQ_ERR_TIMEOUT));
-    __syncthreads();
     // Copies issued but never consumed (only after a failed wait) must land before the CTA exits.
-    if (producer && lane < G) {
-        for (int64_t j = s_consumed[group]; j < issued; ++j)
+    if (leader) {
+        for (int64_t j = consumed; j < issued; ++j)
             if (!mbar_wait(full_bar(static_cast<int>(j % stages)), static_cast<uint32_t>((j / stages) & 1), p.limit_ns, nullptr))
                 atomicCAS(p.status, 0u, static_cast<unsigned int>(SQ_ERR_TIMEOUT));
     }
+    __syncthreads();
 
     if (MODE == MODE_ABSMAX) {
         __syncthreads();                                   // the ring is idle: reuse it
         float *red = reinterpret_cast<float *>(smem);      // [G][K]
-        if (!producer) {
+        {
 #pragma unroll
             for (int i = 0; i < VPL; ++i) {
                 const int v = i * GT + gtid;
@@ -480,33 +500,29 @@ struct Geo {
     size_t smem;
 };
 
-// Row groups hold 64 values per lane per unit where possible (4 vectors x 2 rows).
+// A lane covers 8 vectors (64 elements) of a row, or of R rows of a narrow input.
+constexpr size_t kSmemBudget = 225u * 1024u;   // ring + column table (the static part stays below 2 KB)
+
 Geo row_geo(int K, int mode) {
     const int nvec = K / 8;
     Geo g;
-    if (nvec <= 128) {
-        g.wpr = 1;
+    g.wpr = nvec <= 256 ? 1 : nvec <= 512 ? 2 : nvec <= 1024 ? 4 : 8;
+    if (g.wpr == 1) {
         const int per = (nvec + 31) / 32;
-        g.vpl = per <= 1 ? 1 : per <= 2 ? 2 : 4;
-        g.rpu = 2;
-    } else if (nvec <= 1024) {
-        g.wpr = nvec <= 256 ? 2 : nvec <= 512 ? 4 : 8;
-        g.vpl = 4;
-        g.rpu = 2;
+        g.vpl = per <= 1 ? 1 : per <= 2 ? 2 : per <= 4 ? 4 : 8;
+        g.rpu = 8 / g.vpl;
     } else {
-        g.wpr = 8;
         g.vpl = 8;
         g.rpu = 1;
     }
     g.groups = kWarps / g.wpr;
     const size_t slotbytes = static_cast<size_t>(K) * 2 * g.rpu;
-    const size_t extra = mode == MODE_QUANT ? static_cast<size_t>(K) * 4 : 0;
-    const long budget = 96L * 1024 - static_cast<long>(extra);
-    long st = budget / static_cast<long>(g.groups * slotbytes);
+    const size_t ctab = mode == MODE_QUANT ? static_cast<size_t>(K) * 4 : 0;
+    long st = static_cast<long>((kSmemBudget - ctab) / (g.groups * slotbytes));
     g.stages = static_cast<int>(st < 2 ? 2 : st > kMaxStages ? kMaxStages : st);
     const size_t ring = static_cast<size_t>(g.groups) * g.stages * slotbytes;
     const size_t red = mode == MODE_ABSMAX ? static_cast<size_t>(g.groups) * K * 4 : 0;
-    g.smem = (ring > red ? ring : red) + extra;
+    g.smem = (ring > red ? ring : red) + ctab;
     return g;
 }
 
@@ -575,14 +591,14 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
 
 template <int MODE, bool NORM, bool FULL>
 sq_status dispatch_rows_f(const RowArgs &a, const Geo &g, int dev, cudaStream_t st) {
-    switch (g.wpr * 100 + g.vpl * 10 + g.rpu) {
-        case 112: return launch_rows_t<1, 1, 2, MODE, NORM, FULL>(a, g, dev, st);
-        case 122: return launch_rows_t<1, 2, 2, MODE, NORM, FULL>(a, g, dev, st);
-        case 142: return launch_rows_t<1, 4, 2, MODE, NORM, FULL>(a, g, dev, st);
-        case 242: return launch_rows_t<2, 4, 2, MODE, NORM, FULL>(a, g, dev, st);
-        case 442: return launch_rows_t<4, 4, 2, MODE, NORM, FULL>(a, g, dev, st);
-        case 842: return launch_rows_t<8, 4, 2, MODE, NORM, FULL>(a, g, dev, st);
-        default: return launch_rows_t<8, 8, 1, MODE, NORM, FULL>(a, g, dev, st);
+    if (g.wpr == 2) return launch_rows_t<2, 8, 1, MODE, NORM, FULL>(a, g, dev, st);
+    if (g.wpr == 4) return launch_rows_t<4, 8, 1, MODE, NORM, FULL>(a, g, dev, st);
+    if (g.wpr == 8) return launch_rows_t<8, 8, 1, MODE, NORM, FULL>(a, g, dev, st);
+    switch (g.vpl) {
+        case 1: return launch_rows_t<1, 1, 8, MODE, NORM, FULL>(a, g, dev, st);
+        case 2: return launch_rows_t<1, 2, 4, MODE, NORM, FULL>(a, g, dev, st);
+        case 4: return launch_rows_t<1, 4, 2, MODE, NORM, FULL>(a, g, dev, st);
+        default: return launch_rows_t<1, 8, 1, MODE, NORM, FULL>(a, g, dev, st);
     }
 }
 
