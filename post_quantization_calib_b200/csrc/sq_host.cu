@@ -16,6 +16,7 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int g_arch_ok[kMaxDevices];    // 0 unknown, 1 ok, -1 wrong arch
 int g_sms[kMaxDevices];
+int g_l2[kMaxDevices];
 uint64_t g_timeout_ns[kMaxDevices];
 }  // namespace
 
@@ -42,10 +43,11 @@ sq_status check_arch(int *device_out) {
         std::lock_guard<std::mutex> lk(g_mu);
         if (g_arch_ok[dev] == 1) return SQ_OK;
     }
-    int major = 0, minor = 0, sms = 0;
+    int major = 0, minor = 0, sms = 0, l2 = 0;
     e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev);
     if (e != cudaSuccess) return cuda_status(e, "cudaDeviceGetAttribute");
     std::lock_guard<std::mutex> lk(g_mu);
     if (major != 10 || minor != 0) {
@@ -55,6 +57,7 @@ sq_status check_arch(int *device_out) {
     }
     g_arch_ok[dev] = 1;
     g_sms[dev] = sms;
+    g_l2[dev] = l2;
     if (g_timeout_ns[dev] == 0) g_timeout_ns[dev] = 2000000000ull;
     return SQ_OK;
 }
@@ -62,6 +65,11 @@ sq_status check_arch(int *device_out) {
 int sm_count(int device) {
     std::lock_guard<std::mutex> lk(g_mu);
     return g_sms[device] > 0 ? g_sms[device] : 148;
+}
+
+double l2_bytes(int device) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    return g_l2[device] > 0 ? static_cast<double>(g_l2[device]) : 126.0 * 1024 * 1024;
 }
 
 uint64_t wait_timeout_ns(int device) {

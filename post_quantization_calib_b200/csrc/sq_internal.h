@@ -17,6 +17,9 @@ sq_status check_arch(int *device_out = nullptr);
 // SM count of the current device (cached).
 int sm_count(int device);
 
+// L2 cache size in bytes of the current device (cached).
+double l2_bytes(int device);
+
 // cudaError_t -> SQ_OK / SQ_ERR_CUDA with the CUDA error text recorded.
 sq_status cuda_status(cudaError_t e, const char *what);
 

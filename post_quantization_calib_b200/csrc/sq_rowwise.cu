@@ -83,6 +83,7 @@ struct RowArgs {
     float *scale;           // QUANT output [rows]
     unsigned int *status;   // device status word
     uint64_t limit_ns;      // bound of every wait
+    int stream_once;        // input larger than half the L2: its lines are evicted first
 };
 
 // 1 / sqrt(ss / K + eps) with each step rounded as the RMSNorm definition orders it. When K is a
@@ -139,10 +140,28 @@ __device__ __forceinline__ float rows_max(float (&v)[R], int lane) {
     return v[0];
 }
 
+// |x| * 2^-411 in binary64 for the bf16 x held (sign cleared) in bits 30..16 of `a`: one 64-bit
+// multiply-add a * 2^29 + (485 << 52) writes both halves of the register pair (low half zero).
+__device__ __forceinline__ double sq_operand(uint32_t a) {
+    double d;
+    asm("{\n\t.reg .u64 t;\n\tmad.wide.u32 t, %1, 536870912, %2;\n\tmov.b64 %0, t;\n\t}"
+        : "=d"(d) : "r"(a), "l"(static_cast<uint64_t>(kSqBias) << 32));
+    return d;
+}
+
 // Adds the squares of the two bf16 values of `w` to the scaled binary64 accumulators a and b.
+// WIDE: operands built with one 64-bit multiply-add each (fewer instructions, more registers; the
+// quantiser, which keeps its unit in registers, uses the 32-bit form).
+template <bool WIDE>
 __device__ __forceinline__ void add_squares(uint32_t w, double &a, double &b) {
-    const double d_hi = __hiloint2double(static_cast<int>(mad_hi(w & 0x7FFF0000u, 1u << 29, kSqBias)), 0);
-    const double d_lo = __hiloint2double(static_cast<int>((w & 0x7FFFu) * 8192u + kSqBias), 0);
+    double d_hi, d_lo;
+    if (WIDE) {
+        d_hi = sq_operand(w & 0x7FFF0000u);
+        d_lo = sq_operand((w << 16) & 0x7FFF0000u);
+    } else {
+        d_hi = __hiloint2double(static_cast<int>(mad_hi(w & 0x7FFF0000u, 1u << 29, kSqBias)), 0);
+        d_lo = __hiloint2double(static_cast<int>((w & 0x7FFFu) * 8192u + kSqBias), 0);
+    }
     a = __fma_rn(d_hi, d_hi, a);
     b = __fma_rn(d_lo, d_lo, b);
 }
@@ -183,11 +202,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
     constexpr int G = kWarps / WPR;   // row groups per CTA
     constexpr int GT = 32 * WPR;      // consumer threads per row group
     constexpr int SUB = 32 / R;       // lanes that hold one row's total after a butterfly
-    static_assert(R == 1 || WPR == 1, "several rows per unit only with one warp per row");
+    static_assert(R >= 1 && R <= 8 && VPL * R <= 8, "a unit gives a lane at most 64 element-rows");
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[G * kMaxStages];
-    __shared__ double s_ss[2][kWarps];
-    __shared__ float s_mx[2][kWarps];
+    __shared__ double s_ss[2][kWarps][R];
+    __shared__ float s_mx[2][kWarps][R];
     __shared__ int s_abort[G];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -225,12 +244,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
     auto full_bar = [&](int st) { return smem_u32(&s_full[group * stages + st]); };
     volatile int *abort_flag = &s_abort[group];
     // Leader only: the copies of unit j (nr rows) into slot st, counted on its full barrier.
+    const uint64_t policy = l2_evict_first_policy();
     auto issue = [&](int64_t j, int st) {
         const int64_t r0 = (g0 + j * gstride) * R;
         const int nr = static_cast<int>(p.rows - r0 < R ? p.rows - r0 : R);
         mbar_expect_tx(full_bar(st), rowbytes * static_cast<uint32_t>(nr));
-        for (int r = 0; r < nr; ++r)
-            bulk_g2s(smem_u32(slot(st) + r * rowbytes), p.src + (r0 + r) * p.ld_bytes, rowbytes, full_bar(st));
+        // one copy for the whole unit when its rows are contiguous, else one per row
+        const bool packed = p.ld_bytes == static_cast<int64_t>(rowbytes);
+        const int ncopies = packed ? 1 : nr;
+        const uint32_t bytes = packed ? rowbytes * static_cast<uint32_t>(nr) : rowbytes;
+        for (int r = 0; r < ncopies; ++r) {
+            const uint32_t dst = smem_u32(slot(st) + r * rowbytes);
+            const uint8_t *src = p.src + (r0 + r) * p.ld_bytes;
+            if (p.stream_once) bulk_g2s_hint(dst, src, bytes, full_bar(st), policy);
+            else bulk_g2s(dst, src, bytes, full_bar(st));
+        }
     };
 
     float mx[VPL][8];          // ABSMAX with norm: running max of fl(|x| * inv_rms) per column
@@ -266,11 +294,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
             const int64_t r0 = (g0 + j * gstride) * R;
             const int nr = static_cast<int>(p.rows - r0 < R ? p.rows - r0 : R);   // uniform in the group
             const uint4 *rp = reinterpret_cast<const uint4 *>(slot(st));
-            // a failed wait anywhere in the group stops the whole group at the same unit
-            bool any_fail;
-            if (WPR == 1) any_fail = __any_sync(kAll, !ok);
-            else any_fail = named_sync_or(1 + group, GT, !ok);
-            if (any_fail) {
+            // A failed wait anywhere in the group stops the whole group at the same unit (a warp
+            // of a wider group learns it at the group step below, after reading a stale slot).
+            if (WPR == 1 && __any_sync(kAll, !ok)) {
                 if (leader) { if (!*abort_flag) failed = true; *abort_flag = 1; }
                 break;
             }
@@ -289,29 +315,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                     const uint4 q = in ? rp[r * rv + v] : make_uint4(0u, 0u, 0u, 0u);
                     if (MODE == MODE_QUANT) xr[r][i] = q;
                     if (NORM) {
-                        if (i & 1) { add_squares(q.x, a2, a3); add_squares(q.y, a2, a3); add_squares(q.z, a2, a3); add_squares(q.w, a2, a3); }
-                        else { add_squares(q.x, a0, a1); add_squares(q.y, a0, a1); add_squares(q.z, a0, a1); add_squares(q.w, a0, a1); }
+                        if (i & 1) { add_squares<MODE == MODE_ABSMAX>(q.x, a2, a3); add_squares<MODE == MODE_ABSMAX>(q.y, a2, a3); add_squares<MODE == MODE_ABSMAX>(q.z, a2, a3); add_squares<MODE == MODE_ABSMAX>(q.w, a2, a3); }
+                        else { add_squares<MODE == MODE_ABSMAX>(q.x, a0, a1); add_squares<MODE == MODE_ABSMAX>(q.y, a0, a1); add_squares<MODE == MODE_ABSMAX>(q.z, a0, a1); add_squares<MODE == MODE_ABSMAX>(q.w, a0, a1); }
                     }
                 }
                 ssr[r] = (a0 + a1) + (a2 + a3);
             }
-            if (MODE == MODE_QUANT) {
-                // the unit is in registers now: the slot can be refilled
-                if (WPR == 1) { __syncwarp(); if (leader) refill(j, st); }
-                else if (!NORM) { named_sync(1 + group, GT); if (leader) refill(j, st); }
+            if (WPR > 1) {
+                // Group step, the one barrier of the unit for abs-max: partial sums become visible,
+                // failures propagate, and every warp of the group is past its reads of this slot
+                // (quantiser: the unit is in registers) and of the previous unit's slot (abs-max).
+                if (NORM) {
+                    const double part = rows_sum<R>(ssr, lane);   // row lane / SUB, this warp's columns
+                    if (lane % SUB == 0) s_ss[j & 1][warp][lane / SUB] = part;
+                }
+                if (named_sync_or(1 + group, GT, !ok)) {
+                    if (leader) { if (!*abort_flag) failed = true; *abort_flag = 1; }
+                    break;
+                }
+                if (leader) {
+                    if (MODE == MODE_QUANT) refill(j, st);
+                    else if (j > 0) refill(j - 1, st == 0 ? stages - 1 : st - 1);
+                }
+            } else if (MODE == MODE_QUANT) {
+                __syncwarp();                                   // the unit is in registers now
+                if (leader) refill(j, st);
             }
 
             // ---- 1 / rms of every row of the unit, broadcast to all lanes
             float ir[R];
             if (NORM) {
-                double ss = rows_sum<R>(ssr, lane);             // total of row lane / SUB
+                double ss;
                 if (WPR > 1) {
-                    if (lane == 0) s_ss[j & 1][warp] = ss;
-                    named_sync(1 + group, GT);
-                    if (MODE == MODE_QUANT && leader) refill(j, st);   // every warp has read the slot
                     ss = 0.0;
 #pragma unroll
-                    for (int w = 0; w < WPR; ++w) ss += s_ss[j & 1][group * WPR + w];
+                    for (int w = 0; w < WPR; ++w) ss += s_ss[j & 1][group * WPR + w][lane / SUB];
+                } else {
+                    ss = rows_sum<R>(ssr, lane);                // total of row lane / SUB
                 }
                 const float mine = inv_rms(__dmul_rn(ss, 0x1p822), K, p.inv_k, p.eps);
 #pragma unroll
@@ -351,10 +391,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                         }
                     }
                 }
-                // this group is done with the slot
-                if (WPR == 1) __syncwarp();
-                else named_sync(1 + group, GT);
-                if (leader) refill(j, st);
+                // a single warp is done with the slot; a wider group refills it at its next step
+                if (WPR == 1) {
+                    __syncwarp();
+                    if (leader) refill(j, st);
+                }
             } else {
                 // ---- pass B: y = (x * inv_rms) * c  (or x * c, or x) as element pairs, row maxima
                 uint64_t y[R][VPL][4];
@@ -384,11 +425,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                 }
                 float mrow = rows_max<R>(m, lane);               // maximum of row lane / SUB
                 if (WPR > 1) {
-                    if (lane == 0) s_mx[j & 1][warp] = mrow;
+                    if (lane % SUB == 0) s_mx[j & 1][warp][lane / SUB] = mrow;
                     named_sync(1 + group, GT);
                     mrow = 0.0f;
 #pragma unroll
-                    for (int w = 0; w < WPR; ++w) mrow = fmaxf(mrow, s_mx[j & 1][group * WPR + w]);
+                    for (int w = 0; w < WPR; ++w) mrow = fmaxf(mrow, s_mx[j & 1][group * WPR + w][lane / SUB]);
                 }
                 // step and reciprocal of the row this lane holds; one lane per row stores the step
                 const float delta = mrow > 0.0f ? __fdiv_rn(mrow, kQmax) : 0.0f;
@@ -496,33 +537,30 @@ __global__ void k_scales(const float *__restrict__ ax, const float *__restrict__
 // Launch geometry and dispatch.
 
 struct Geo {
-    int wpr, vpl, rpu, groups, stages;   // warps per row group, vectors per lane, rows per unit
-    size_t smem;
+    int wpr, vpl, rpu, groups;   // warps per row group, vectors per lane, rows per unit
 };
 
-// A lane covers 8 vectors (64 elements) of a row, or of R rows of a narrow input.
-constexpr size_t kSmemBudget = 225u * 1024u;   // ring + column table (the static part stays below 2 KB)
-
-Geo row_geo(int K, int mode) {
-    const int nvec = K / 8;
-    Geo g;
-    g.wpr = nvec <= 256 ? 1 : nvec <= 512 ? 2 : nvec <= 1024 ? 4 : 8;
-    if (g.wpr == 1) {
-        const int per = (nvec + 31) / 32;
-        g.vpl = per <= 1 ? 1 : per <= 2 ? 2 : per <= 4 ? 4 : 8;
-        g.rpu = 8 / g.vpl;
-    } else {
-        g.vpl = 8;
-        g.rpu = 1;
-    }
-    g.groups = kWarps / g.wpr;
+// Dynamic shared memory of a launch with `stages` ring slots per group.
+size_t rows_smem(int K, int mode, const Geo &g, int stages) {
     const size_t slotbytes = static_cast<size_t>(K) * 2 * g.rpu;
     const size_t ctab = mode == MODE_QUANT ? static_cast<size_t>(K) * 4 : 0;
-    long st = static_cast<long>((kSmemBudget - ctab) / (g.groups * slotbytes));
-    g.stages = static_cast<int>(st < 2 ? 2 : st > kMaxStages ? kMaxStages : st);
-    const size_t ring = static_cast<size_t>(g.groups) * g.stages * slotbytes;
+    const size_t ring = static_cast<size_t>(g.groups) * stages * slotbytes;
     const size_t red = mode == MODE_ABSMAX ? static_cast<size_t>(g.groups) * K * 4 : 0;
-    g.smem = (ring > red ? ring : red) + ctab;
+    return (ring > red ? ring : red) + ctab;
+}
+
+// A lane covers 8 vectors (64 elements) of a row, or of R rows of a narrow input.
+Geo row_geo(int K) {
+    const int nvec = K / 8;
+    Geo g;
+    // Rows of up to 2048 elements take one warp each (R = 8 / VPL rows per unit), wider rows a
+    // group of 2, 4 or 8 warps with one row per unit. (Groups of 4 warps over 2-row units of
+    // 4096-element rows gave larger copies but lost more to the wider group barrier.)
+    g.wpr = nvec <= 256 ? 1 : nvec <= 512 ? 2 : nvec <= 1024 ? 4 : 8;
+    const int per = (nvec + 32 * g.wpr - 1) / (32 * g.wpr);
+    g.vpl = per <= 1 ? 1 : per <= 2 ? 2 : per <= 4 ? 4 : 8;
+    g.rpu = 8 / g.vpl;
+    g.groups = kWarps / g.wpr;
     return g;
 }
 
@@ -533,21 +571,35 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
     static size_t configured_smem[64];
     static int per_sm[64];
     static int cluster_size[64], cluster_ctas[64];
+    static size_t smem_cap[64];    // opt-in maximum minus this kernel's static shared memory
+    if (smem_cap[dev] == 0) {
+        int optin = 0;
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return sq::cuda_status(e, "shared memory limits (rows)");
+        smem_cap[dev] = static_cast<size_t>(optin) - fa.sharedSizeBytes;
+    }
+    // as many ring slots per group as fit (2 .. kMaxStages)
+    int stages = kMaxStages;
+    while (stages > 2 && rows_smem(a.K, MODE, geo, stages) > smem_cap[dev]) --stages;
+    const size_t smem = rows_smem(a.K, MODE, geo, stages);
+    if (smem > smem_cap[dev]) return sq::fail(SQ_ERR_UNSUPPORTED, "row kernel needs %zu bytes of shared memory", smem);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = geo.smem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (configured_smem[dev] < geo.smem) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(geo.smem));
+    if (configured_smem[dev] < smem) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
         if (e != cudaSuccess) return sq::cuda_status(e, "cudaFuncSetAttribute(rows)");
         int nb = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, geo.smem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, smem);
         if (e != cudaSuccess) return sq::cuda_status(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor(rows)");
         per_sm[dev] = nb > 0 ? nb : 1;
         if (MODE == MODE_ABSMAX) {
@@ -564,19 +616,20 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
             }
             if (cluster_ctas[dev] == 0) return sq::fail(SQ_ERR_CUDA, "no cluster configuration fits the abs-max kernel");
         }
-        configured_smem[dev] = geo.smem;
+        configured_smem[dev] = smem;
     }
     const int64_t full = static_cast<int64_t>(sq::sm_count(dev)) * per_sm[dev];
-    a.stages = geo.stages;
+    a.stages = stages;
     a.inv_k = (a.K & (a.K - 1)) == 0 ? 1.0 / static_cast<double>(a.K) : 0.0;
     a.status = sq::device_status_word(dev);
     a.limit_ns = sq::wait_timeout_ns(dev);
+    a.stream_once = static_cast<double>(a.rows) * static_cast<double>(a.ld_bytes) > 0.5 * sq::l2_bytes(dev) ? 1 : 0;
     if (a.status == nullptr) return sq::fail(SQ_ERR_CUDA, "device status word unavailable");
     const int64_t units = (a.rows + R - 1) / R;
     if (MODE == MODE_QUANT) {
         int64_t ctas = (units + G - 1) / G;
         if (ctas > full) ctas = full;
-        kern<<<static_cast<unsigned>(ctas), kThreads, geo.smem, st>>>(a);
+        kern<<<static_cast<unsigned>(ctas), kThreads, smem, st>>>(a);
         return sq::cuda_status(cudaGetLastError(), "launch(rowquant)");
     }
     // one wave of resident clusters at most, at least ~4 units per group
@@ -605,7 +658,7 @@ sq_status dispatch_rows_f(const RowArgs &a, const Geo &g, int dev, cudaStream_t 
 // FULL: the row is exactly VPL vectors per lane of the group (no bounds checks per vector).
 template <int MODE, bool NORM>
 sq_status dispatch_rows(const RowArgs &a, int dev, cudaStream_t st) {
-    const Geo g = row_geo(a.K, MODE);
+    const Geo g = row_geo(a.K);
     const bool full = (a.K / 8) == g.vpl * 32 * g.wpr;
     return full ? dispatch_rows_f<MODE, NORM, true>(a, g, dev, st) : dispatch_rows_f<MODE, NORM, false>(a, g, dev, st);
 }
