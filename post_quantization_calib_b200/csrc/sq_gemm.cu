@@ -46,31 +46,17 @@ __device__ unsigned int g_sq_status;
 std::atomic<int> g_cta_pair{0};
 
 constexpr int BM = 128;            // tokens per tile (MMA M)
-constexpr int BN = 256;            // output channels per tile (MMA N)
+constexpr int BN = 256;            // output channels per tile of the wide forms (MMA N)
 constexpr int BK = 128;            // K bytes per pipeline stage (one 128-byte swizzle row)
 constexpr int UMMA_K = 32;         // K per tcgen05.mma.kind::i8
-constexpr int STAGES = 4;
 constexpr int A_STAGE = BM * BK;   // 16 KB
-constexpr int B_STAGE = BN * BK;   // 32 KB
 constexpr int EPI_WARPS = 4;
 constexpr int OUT_COLS = 32;       // bf16 columns per TMA store box (64 bytes, 64-byte swizzle)
 constexpr int OUT_ROWS = 32;       // rows per box: one warp's TMEM lane quarter
 constexpr int OUT_BOX = OUT_COLS * 2 * OUT_ROWS;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
-constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int BAND = 16;           // M tiles per raster band
-
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
-constexpr int OFF_OUT = OFF_B + STAGES * B_STAGE;
-constexpr int COL_TAB = 2 * BN * 4;   // w_scale and bias (binary32) of one tile's columns
-constexpr int OFF_COL = OFF_OUT + EPI_WARPS * 2 * OUT_BOX;
-constexpr int OFF_BAR = OFF_COL + 2 * COL_TAB;   // one table per accumulator buffer
-constexpr int NBARS = 2 * STAGES + 5;   // full[S], empty[S], tfull[2], tempty[2], done
-constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
-constexpr int SMEM_USED = OFF_MISC + 16;
-constexpr int SMEM_TOTAL = SMEM_USED + 1024;    // slack to align the base to 1024 bytes
-static_assert(SMEM_TOTAL <= 232448, "shared memory budget of one sm_100 CTA");
+constexpr int COL_TAB = 2 * BN * 4;   // w_scale and bias (binary32) of up to 256 columns
 
 // Instruction descriptor of tcgen05.mma.kind::i8: D = s32, A and B signed 8-bit, both K-major,
 // N >> 3 at bits 17..22, M >> 4 at bits 24..28.
@@ -78,7 +64,28 @@ constexpr uint32_t make_idesc(int M, int N) {
     return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);
 }
-constexpr uint32_t IDESC = make_idesc(BM, BN);
+
+// Shared-memory plan of the single-SM kernel for tiles of TN output channels. The 256-wide form
+// serves token counts that fill the SMs with tiles; the 64-wide form serves few tokens (decode),
+// where the weight stream dominates: four times as many tiles, and a deeper ring (8 stages of
+// 24 KB) keeps more weight bytes in flight per SM.
+template <int TN>
+struct Tile {
+    static constexpr int STAGES = TN == 256 ? 4 : 8;
+    static constexpr int B_STAGE = TN * BK;
+    static constexpr uint32_t TMEM_COLS = 2 * TN;          // two accumulators; a power of two >= 32
+    static constexpr int OFF_A = 0;
+    static constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
+    static constexpr int OFF_OUT = OFF_B + STAGES * B_STAGE;
+    static constexpr int OFF_COL = OFF_OUT + EPI_WARPS * 2 * OUT_BOX;
+    static constexpr int OFF_BAR = OFF_COL + 2 * COL_TAB;   // one column table per accumulator
+    static constexpr int NBARS = 2 * STAGES + 5;            // full[S], empty[S], tfull[2], tempty[2], done
+    static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+    static constexpr int SMEM_TOTAL = OFF_MISC + 16 + 1024; // slack to align the base to 1024 bytes
+    static constexpr uint32_t IDESC = make_idesc(BM, TN);
+    static_assert(SMEM_TOTAL <= 232448, "shared memory budget of one sm_100 CTA");
+    static_assert(TN % OUT_COLS == 0 && TN >= 32 && TN <= 256 && (TN & (TN - 1)) == 0, "tile width");
+};
 
 // ------------------------------------------------------------------------------------------------
 // PTX wrappers.
@@ -234,20 +241,25 @@ struct ColShare {
     uint32_t b;
 };
 
+// The tile's TN columns: thread ep fetches columns n0 + 2 ep and n0 + 2 ep + 1 (threads beyond
+// TN / 2 fetch nothing).
+template <int TN>
 __device__ __forceinline__ void cols_fetch(ColShare &p, int n0, int ep, const float *__restrict__ w_scale,
                                            const __nv_bfloat16 *__restrict__ bias, int N) {
     const int col = n0 + 2 * ep;
     p.w = make_float2(0.f, 0.f);
     p.b = 0u;
-    if (col < N) {      // N is even: both columns are in range or both beyond it
+    if (2 * ep < TN && col < N) {      // N is even: both columns are in range or both beyond it
         p.w = __ldg(reinterpret_cast<const float2 *>(w_scale + col));
         if (bias != nullptr) p.b = __ldg(reinterpret_cast<const unsigned int *>(bias + col));
     }
 }
 
+template <int TN>
 __device__ __forceinline__ void cols_store(const ColShare &p, float *tab, int ep) {
+    if (2 * ep >= TN) return;
     *reinterpret_cast<float2 *>(tab + 2 * ep) = p.w;
-    *reinterpret_cast<float2 *>(tab + BN + 2 * ep) = make_float2(__uint_as_float(p.b << 16), __uint_as_float(p.b & 0xFFFF0000u));
+    *reinterpret_cast<float2 *>(tab + TN + 2 * ep) = make_float2(__uint_as_float(p.b << 16), __uint_as_float(p.b & 0xFFFF0000u));
 }
 
 // Two packed pairs (four consecutive binary32 values) from shared memory, same address in every lane.
@@ -281,13 +293,14 @@ __device__ __forceinline__ void regs_after_wait(uint32_t *r) {
 }
 
 // Epilogue of one warp for one output tile: reads its 32 TMEM lanes (token rows row0 .. row0+31) for
-// columns n0 .. n0+255 of accumulator buffer `tcol` (TMEM column offset), applies
+// columns n0 .. n0+TN-1 of accumulator buffer `tcol` (TMEM column offset), applies
 // y = bf16(float(acc) * (x_scale * w_scale) + bias) in binary32 (each operation rounded once, two
 // columns per packed instruction), stages 32 x 32 boxes in 64-byte-swizzled shared memory and writes
 // them with TMA stores; optionally writes the raw accumulators. `tab` is the tile's column table,
 // `xs` the x_scale of this lane's row. The TMEM read of the next 32 columns is in flight while the
 // current 32 are converted. `stage_buf` holds two boxes that alternate; `nstores` counts this warp's
 // stores.
+template <int TN>
 __device__ __forceinline__ void epilogue_rows(uint32_t tmem_base, int quad, int lane, uint32_t tcol, int row0, int n0,
                                               float xs, const float *tab, bool has_bias, int32_t *__restrict__ acc_out,
                                               int T, int N, const CUtensorMap *tmY, uint8_t *stage_buf, int &nstores)
@@ -299,12 +312,12 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tmem_base, int quad, int 
     uint32_t ra[32], rb[32];
     tmem_ld32p(tl, ra);
 #pragma unroll
-    for (int c = 0; c < BN / OUT_COLS; ++c) {
+    for (int c = 0; c < TN / OUT_COLS; ++c) {
         uint32_t *cur = (c & 1) ? rb : ra;
         uint32_t *nxt = (c & 1) ? ra : rb;
         tmem_ld_wait();
         regs_after_wait(cur);
-        if (c + 1 < BN / OUT_COLS) tmem_ld32p(tl + (c + 1) * OUT_COLS, nxt);
+        if (c + 1 < TN / OUT_COLS) tmem_ld32p(tl + (c + 1) * OUT_COLS, nxt);
         const int col0 = n0 + c * OUT_COLS;
         if (col0 >= N) continue;
         if (acc_out != nullptr && row < T) {
@@ -327,7 +340,7 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tmem_base, int quad, int 
             uint64_t v23 = mul2_rn(a23, mul2_rn(xs2, w23));
             if (has_bias) {
                 uint64_t b01, b23;
-                lds_pairs(tab + BN + c * OUT_COLS + 4 * g, b01, b23);
+                lds_pairs(tab + TN + c * OUT_COLS + 4 * g, b01, b23);
                 v01 = add2_rn(v01, b01);
                 v23 = add2_rn(v23, b23);
             }
@@ -358,27 +371,30 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tmem_base, int quad, int 
 
 // ------------------------------------------------------------------------------------------------
 
+template <int TN>
 __global__ void __launch_bounds__(THREADS, 1)
 k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmY, const float *__restrict__ x_scale,
               const float *__restrict__ w_scale, const __nv_bfloat16 *__restrict__ bias,
-              int32_t *__restrict__ acc_out, int T, int N, int K, int m_tiles, int n_tiles,
+              int32_t *__restrict__ acc_out, int T, int N, int K, int m_tiles, int n_tiles, int a_rows,
               uint64_t limit_ns)
 {
+    using L = Tile<TN>;
+    constexpr int STAGES = L::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sA = smem + OFF_A;
-    uint8_t *sB = smem + OFF_B;
-    uint8_t *sOut = smem + OFF_OUT;
-    float *sCol = reinterpret_cast<float *>(smem + OFF_COL);
-    const uint32_t bar0 = smem_u32(smem + OFF_BAR);
+    uint8_t *sA = smem + L::OFF_A;
+    uint8_t *sB = smem + L::OFF_B;
+    uint8_t *sOut = smem + L::OFF_OUT;
+    float *sCol = reinterpret_cast<float *>(smem + L::OFF_COL);
+    const uint32_t bar0 = smem_u32(smem + L::OFF_BAR);
     auto full = [&](int s) { return bar0 + 8u * s; };
     auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
     auto tfull = [&](int b) { return bar0 + 8u * (2 * STAGES + b); };
     auto tempty = [&](int b) { return bar0 + 8u * (2 * STAGES + 2 + b); };
     const uint32_t done_bar = bar0 + 8u * (2 * STAGES + 4);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::OFF_MISC + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -392,7 +408,18 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         fence_async_smem();
     }
     if (warp == 0 && lane == 0) { prefetch_map(&tmA); prefetch_map(&tmB); prefetch_map(&tmY); }
-    if (warp == 1) { tmem_alloc(smem_u32(tmem_slot), TMEM_COLS); tmem_relinquish(); }
+    if (warp == 1) { tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS); tmem_relinquish(); }
+    // Fewer than 128 tokens: only the first a_rows rows of each A slot are loaded; the rest hold
+    // zeros, written once here (their products land in accumulator rows that are never stored).
+    if (a_rows < BM) {
+        const int per_slot = (BM - a_rows) * BK / 16;
+        for (int i = threadIdx.x; i < STAGES * per_slot; i += THREADS) {
+            const int st = i / per_slot;
+            uint8_t *dst = sA + st * A_STAGE + a_rows * BK + (i - st * per_slot) * 16;
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_async_smem();     // visible to the tensor cores (async proxy)
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -400,6 +427,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 
     const int k_blocks = (K + BK - 1) / BK;
     const int num_tiles = m_tiles * n_tiles;
+    const uint32_t stage_tx = static_cast<uint32_t>(a_rows * BK + L::B_STAGE);
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -413,9 +441,9 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 tile_coords(t, m_tiles, n_tiles, m, n);
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait(empty(stage), phase ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
-                    mbar_expect_tx(full(stage), A_STAGE + B_STAGE);
+                    mbar_expect_tx(full(stage), stage_tx);
                     tma_load_2d(smem_u32(sA + stage * A_STAGE), &tmA, full(stage), kb * BK, m * BM);
-                    tma_load_2d(smem_u32(sB + stage * B_STAGE), &tmB, full(stage), kb * BK, n * BN);
+                    tma_load_2d(smem_u32(sB + stage * L::B_STAGE), &tmB, full(stage), kb * BK, n * TN);
                     ++fills;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -442,15 +470,15 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 const uint32_t use = static_cast<uint32_t>(lt >> 1);
                 if (!mbar_wait(tempty(buf), (use & 1u) ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * TN);
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait(full(stage), phase, limit_ns, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sA + stage * A_STAGE);
-                    const uint32_t b0 = smem_u32(sB + stage * B_STAGE);
+                    const uint32_t b0 = smem_u32(sB + stage * L::B_STAGE);
 #pragma unroll
                     for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-                        mma_i8(d_tmem, kmajor_sw128_desc(a0 + kk * UMMA_K), kmajor_sw128_desc(b0 + kk * UMMA_K), IDESC,
+                        mma_i8(d_tmem, kmajor_sw128_desc(a0 + kk * UMMA_K), kmajor_sw128_desc(b0 + kk * UMMA_K), L::IDESC,
                                (kb | kk) != 0 ? 1u : 0u);
                     }
                     issued = true;
@@ -481,7 +509,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             if (t >= num_tiles) return;
             int m, n;
             tile_coords(t, m_tiles, n_tiles, m, n);
-            cols_fetch(cols, n * BN, ep, w_scale, bias, N);
+            cols_fetch<TN>(cols, n * TN, ep, w_scale, bias, N);
             const int row = m * BM + quad * 32 + lane;
             xs = row < T ? __ldg(x_scale + row) : 0.0f;
         };
@@ -491,7 +519,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             const uint32_t use = static_cast<uint32_t>(lt >> 1);
             const bool ok = mbar_wait(tfull(buf), use & 1u, limit_ns, abort_flag);
             float *tab = sCol + buf * (COL_TAB / 4);
-            if (ok) cols_store(cols, tab, ep);
+            if (ok) cols_store<TN>(cols, tab, ep);
             // every epilogue thread arrives (its wait is bounded); the table is complete after it
             if (named_sync_or(EPI_BAR, EPI_THREADS, !ok)) { give_up(abort_flag); break; }
             tc_fence_after();
@@ -499,7 +527,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             tile_coords(t, m_tiles, n_tiles, m, n);
             const float xs_t = xs;
             prefetch(t + gridDim.x);
-            epilogue_rows(tmem_base, quad, lane, static_cast<uint32_t>(buf * BN), m * BM + quad * 32, n * BN, xs_t, tab,
+            epilogue_rows<TN>(tmem_base, quad, lane, static_cast<uint32_t>(buf * TN), m * BM + quad * 32, n * TN, xs_t, tab,
                           bias != nullptr, acc_out, T, N, &tmY, stage_buf, nstores);
             tc_fence_before();
             mbar_arrive(tempty(buf));
@@ -511,7 +539,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
+    if (warp == 1) tmem_dealloc(tmem_base, L::TMEM_COLS);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -535,6 +563,7 @@ constexpr int P_OFF_MISC = P_OFF_BAR + P_NBARS * 8;
 constexpr int P_SMEM_TOTAL = P_OFF_MISC + 16 + 1024;
 static_assert(P_SMEM_TOTAL <= 232448, "shared memory budget of one sm_100 CTA");
 constexpr uint32_t P_IDESC = make_idesc(2 * BM, BN);
+constexpr uint32_t P_TMEM_COLS = 2 * BN;
 
 __global__ void __launch_bounds__(THREADS, 1)
 k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -573,7 +602,7 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         fence_async_smem();
     }
     if (warp == 0 && lane == 0) { prefetch_map(&tmA); prefetch_map(&tmB); prefetch_map(&tmY); }
-    if (warp == 1) { tmem_alloc2(smem_u32(tmem_slot), TMEM_COLS); tmem_relinquish2(); }
+    if (warp == 1) { tmem_alloc2(smem_u32(tmem_slot), P_TMEM_COLS); tmem_relinquish2(); }
     tc_fence_before();
     __syncthreads();
     cluster_sync_all();                                 // both CTAs' barriers exist before any remote use
@@ -667,7 +696,7 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             if (t >= num_tiles) return;
             int m, n;
             tile_coords(t, m_tiles, n_tiles, m, n);
-            cols_fetch(cols, n * BN, ep, w_scale, bias, N);
+            cols_fetch<BN>(cols, n * BN, ep, w_scale, bias, N);
             const int row = m * 2 * BM + static_cast<int>(rank) * BM + quad * 32 + lane;
             xs = row < T ? __ldg(x_scale + row) : 0.0f;
         };
@@ -677,14 +706,14 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             const uint32_t use = static_cast<uint32_t>(lt >> 1);
             const bool ok = mbar_wait_cluster(tfull(buf), use & 1u, limit_ns, abort_flag);
             float *tab = sCol + buf * (COL_TAB / 4);
-            if (ok) cols_store(cols, tab, ep);
+            if (ok) cols_store<BN>(cols, tab, ep);
             if (named_sync_or(EPI_BAR, EPI_THREADS, !ok)) { give_up(abort_flag); break; }
             tc_fence_after();
             int m, n;
             tile_coords(t, m_tiles, n_tiles, m, n);
             const float xs_t = xs;
             prefetch(t + ncl);
-            epilogue_rows(tmem_base, quad, lane, static_cast<uint32_t>(buf * BN),
+            epilogue_rows<BN>(tmem_base, quad, lane, static_cast<uint32_t>(buf * BN),
                           m * 2 * BM + static_cast<int>(rank) * BM + quad * 32, n * BN, xs_t, tab, bias != nullptr, acc_out,
                           T, N, &tmY, stage_buf, nstores);
             tc_fence_before();
@@ -705,7 +734,7 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     }
     cluster_sync_all();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc2(tmem_base, TMEM_COLS);
+    if (warp == 1) tmem_dealloc2(tmem_base, P_TMEM_COLS);
 }
 
 // One thread waits, with the same bounded wait as the GEMM, on a barrier nothing completes.
@@ -754,6 +783,28 @@ sq_status encode_2d(EncodeTiledFn enc, CUtensorMap *map, CUtensorMapDataType dt,
     return SQ_OK;
 }
 
+// Single-SM form with TN-channel tiles: one persistent CTA per SM at most.
+template <int TN>
+sq_status launch_single(const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mY, const float *x_scale,
+                        const float *w_scale, const void *bias, int32_t *acc_out, int64_t T, int64_t N, int64_t K,
+                        int a_rows, int dev, void *stream) {
+    static int configured[64];
+    if (!configured[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(k_w8a8_linear<TN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<TN>::SMEM_TOTAL);
+        if (e != cudaSuccess) return sq::cuda_status(e, "cudaFuncSetAttribute(w8a8_linear)");
+        configured[dev] = 1;
+    }
+    const int m_tiles = static_cast<int>((T + BM - 1) / BM);
+    const int n_tiles = static_cast<int>((N + TN - 1) / TN);
+    const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
+    if (tiles > 0x7FFFFFFF) return sq::fail(SQ_ERR_UNSUPPORTED, "sq_w8a8_linear: too many tiles");
+    const int grid = static_cast<int>(tiles < sq::sm_count(dev) ? tiles : sq::sm_count(dev));
+    k_w8a8_linear<TN><<<grid, THREADS, Tile<TN>::SMEM_TOTAL, sq::as_stream(stream)>>>(
+        mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out, static_cast<int>(T),
+        static_cast<int>(N), static_cast<int>(K), m_tiles, n_tiles, a_rows, sq::wait_timeout_ns(dev));
+    return sq::cuda_status(cudaGetLastError(), "launch(w8a8_linear)");
+}
+
 }  // namespace
 
 namespace sq {
@@ -798,9 +849,15 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, cons
     sq_status st = get_encoder(&enc);
     if (st != SQ_OK) return st;
     const bool pair = g_cta_pair.load(std::memory_order_relaxed) != 0 && T >= 2 * BM;   // 256-row tiles on CTA pairs
+    // 64-channel tiles when 256-channel tiles would leave SMs idle (few tokens: the weight stream
+    // then bounds the call, and more tiles spread it over more SMs)
+    const int64_t wide_tiles = ((T + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const bool narrow = !pair && wide_tiles < sq::sm_count(dev);
     CUtensorMap mA, mB, mY;
-    st = encode_2d(enc, &mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, T, K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B, "xq");
-    if (st == SQ_OK) st = encode_2d(enc, &mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, K, N, K, BK, pair ? 128 : BN, CU_TENSOR_MAP_SWIZZLE_128B, "wq");
+    // one M tile of fewer than 128 tokens: load only the token rows (rounded up to 8)
+    const int a_rows = T < BM ? static_cast<int>((T + 7) / 8 * 8) : BM;
+    st = encode_2d(enc, &mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, T, K, BK, pair ? BM : a_rows, CU_TENSOR_MAP_SWIZZLE_128B, "xq");
+    if (st == SQ_OK) st = encode_2d(enc, &mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, K, N, K, BK, pair ? 128 : narrow ? 64 : BN, CU_TENSOR_MAP_SWIZZLE_128B, "wq");
     if (st == SQ_OK) st = encode_2d(enc, &mY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, T, N * 2, OUT_COLS, OUT_ROWS, CU_TENSOR_MAP_SWIZZLE_64B, "y");
     if (st != SQ_OK) return st;
     if (pair) {
@@ -840,21 +897,8 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, cons
             "launch(w8a8_linear_pair)");
     }
 
-    static int configured[64];
-    if (!configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_w8a8_linear, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_TOTAL);
-        if (e != cudaSuccess) return sq::cuda_status(e, "cudaFuncSetAttribute(w8a8_linear)");
-        configured[dev] = 1;
-    }
-    const int m_tiles = static_cast<int>((T + BM - 1) / BM);
-    const int n_tiles = static_cast<int>((N + BN - 1) / BN);
-    const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
-    if (tiles > 0x7FFFFFFF) return fail(SQ_ERR_UNSUPPORTED, "sq_w8a8_linear: too many tiles");
-    const int grid = static_cast<int>(tiles < sq::sm_count(dev) ? tiles : sq::sm_count(dev));
-    k_w8a8_linear<<<grid, THREADS, SMEM_TOTAL, sq::as_stream(stream)>>>(
-        mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out, static_cast<int>(T),
-        static_cast<int>(N), static_cast<int>(K), m_tiles, n_tiles, sq::wait_timeout_ns(dev));
-    return sq::cuda_status(cudaGetLastError(), "launch(w8a8_linear)");
+    return narrow ? launch_single<64>(mA, mB, mY, x_scale, w_scale, bias, acc_out, T, N, K, a_rows, dev, stream)
+                  : launch_single<BN>(mA, mB, mY, x_scale, w_scale, bias, acc_out, T, N, K, a_rows, dev, stream);
 }
 
 sq_status sq_set_gemm_cta_pair(int enable) {

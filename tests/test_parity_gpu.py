@@ -171,6 +171,9 @@ EDGE = [
     (128, 256, 128, True, False),
     (255, 512, 4096, False, False),
     (777, 1288, 2064, True, True),
+    # enough 256-channel tiles to take the wide form, with ragged T, N and K
+    (2000, 2312, 1040, True, True),
+    (64, 37888, 64, False, True),
 ]
 
 
