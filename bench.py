@@ -130,9 +130,9 @@ def stage_work(w, T, N, K, calib_rows):
     }
 
 
-KERNEL_OF = {"calib_absmax": ("k_rows<ABSMAX,NORM>", "sq_rowwise.cu"), "weight_absmax": ("k_rows<ABSMAX>", "sq_rowwise.cu"),
-             "scales": ("k_scales", "sq_rowwise.cu"), "weight_quant": ("k_rows<QUANT>", "sq_rowwise.cu"),
-             "act_quant": ("k_rows<QUANT,NORM>", "sq_rowwise.cu"), "gemm": ("k_w8a8_linear", "sq_gemm.cu")}
+KERNEL_OF = {"calib_absmax": ("k_rows<2,8,1,ABSMAX,NORM>", "sq_rowwise.cu"), "weight_absmax": ("k_rows<2,8,1,ABSMAX>", "sq_rowwise.cu"),
+             "scales": ("k_scales", "sq_rowwise.cu"), "weight_quant": ("k_rows<2,8,1,QUANT>", "sq_rowwise.cu"),
+             "act_quant": ("k_rows<2,8,1,QUANT,NORM>", "sq_rowwise.cu"), "gemm": ("k_w8a8_linear<256>", "sq_gemm.cu")}
 LAUNCHES = {"calib_absmax": 2, "weight_absmax": 2, "scales": 1, "weight_quant": 1, "act_quant": 1, "gemm": 1}
 
 
