@@ -15,6 +15,7 @@ from . import build as _build
 
 __all__ = [
     "calibrate_absmax", "compute_scales", "smooth_quantize_weight", "rmsnorm_smooth_quant",
+    "static_scale", "rmsnorm_smooth_quant_static",
     "gemm_s8", "dequant", "w8a8_linear", "f32_to_bf16", "bf16_to_f32", "set_threads", "lib",
 ]
 
@@ -36,6 +37,8 @@ def lib() -> ctypes.CDLL:
             L.orc_compute_scales.argtypes = [_p, _p, _i64, ctypes.c_float, _p, _p, _p]
             L.orc_smooth_quantize_weight.argtypes = [_p, _i64, _i64, _p, _p, _p, _p]
             L.orc_rmsnorm_smooth_quant.argtypes = [_p, _i64, _i64, _p, ctypes.c_float, ctypes.c_int, _p, _p, _p]
+            L.orc_static_scale.argtypes = [_p, _i64, _p]
+            L.orc_rmsnorm_smooth_quant_static.argtypes = [_p, _i64, _i64, _p, ctypes.c_float, ctypes.c_int, _p, _p, _p]
             L.orc_gemm_s8.argtypes = [_p, _i64, _p, _i64, _i64, _p, _i64, _p, _i64, _p]
             L.orc_dequant.argtypes = [_p, _p, _p, _p, _p, _i64, _p, _i64, _p]
             L.orc_f32_to_bf16.argtypes = [ctypes.c_float]
@@ -118,6 +121,29 @@ def rmsnorm_smooth_quant(x, fold, eps=1e-6, apply_norm=True):
     work = np.empty(K, np.float32)
     lib().orc_rmsnorm_smooth_quant(_ptr(x), T, K, _ptr(f), float(eps), int(bool(apply_norm)),
                                    _ptr(xq), _ptr(xs), _ptr(work))
+    return xq, xs
+
+
+def static_scale(amax_y):
+    """Static per-tensor scale from the calibration maximum of the smoothed activation
+    ([W8A8] "One layer, measured"). Returns float32 [2] = (delta, 127 / m)."""
+    a = _need(amax_y, np.float32, "amax_y")
+    out = np.empty(2, np.float32)
+    lib().orc_static_scale(_ptr(a), a.shape[0], _ptr(out))
+    return out
+
+
+def rmsnorm_smooth_quant_static(x, fold, scale2, eps=1e-6, apply_norm=True):
+    """(RMSNorm with folded weight, or x*fold) then INT8 with the one static scale (clipping past the
+    calibrated maximum). Returns (xq, x_scale) with x_scale[t] = delta for every token."""
+    x = _need(x, np.uint16, "x")
+    T, K = x.shape
+    f = _need(fold, np.float32, "fold")
+    s2 = _need(scale2, np.float32, "scale2")
+    xq = np.empty((T, K), np.int8)
+    xs = np.empty(T, np.float32)
+    lib().orc_rmsnorm_smooth_quant_static(_ptr(x), T, K, _ptr(f), float(eps), int(bool(apply_norm)), _ptr(s2),
+                                          _ptr(xq), _ptr(xs))
     return xq, xs
 
 

@@ -207,6 +207,54 @@ void orc_rmsnorm_smooth_quant(const uint16_t *x, int64_t T, int64_t K, const flo
 }
 
 /*
+ * Static per-tensor activation scale, [W8A8] "One layer, measured" (one static scale per tensor,
+ * taken from the calibration tokens' maximum) and "Gotchas" (values past the calibrated maximum are
+ * clipped). amax_y[k] is the per-channel maximum, over the calibration tokens, of the smoothed
+ * activation exactly as the online quantiser forms it (the calibration abs-max with the fold in
+ * place of gamma). The tensor maximum is m = max_k amax_y[k]; scale2[0] = delta = m / 127 and
+ * scale2[1] = 127 / m, the same two values the per-token quantiser derives from a row maximum
+ * (m == 0 gives 0 and 0).
+ */
+void orc_static_scale(const float *amax_y, int64_t K, float *scale2)
+{
+    float m = 0.0f;
+    for (int64_t k = 0; k < K; ++k)
+        if (amax_y[k] > m) m = amax_y[k];
+    if (m == 0.0f) {
+        scale2[0] = 0.0f;
+        scale2[1] = 0.0f;
+        return;
+    }
+    scale2[0] = m / (float)ORC_QMAX;
+    scale2[1] = (float)ORC_QMAX / m;
+}
+
+/*
+ * Online activation quantisation with the static per-tensor scale: the smoothed (and, with
+ * apply_norm, normalised) activation y is formed exactly as in orc_rmsnorm_smooth_quant, then
+ * every value is coded with the one calibrated scale: q = clamp(round_half_away(y * scale2[1]),
+ * -127, 127) (values beyond the calibrated maximum saturate), and every token's scale is
+ * scale2[0], so the dequantisation is the scalar step times the per-channel weight scale.
+ *   [W8A8] "One layer, measured" and "Gotchas"; the quantiser of [TAMING] "Why Outliers Break
+ *   Quantization".
+ */
+void orc_rmsnorm_smooth_quant_static(const uint16_t *x, int64_t T, int64_t K, const float *fold,
+                                     float eps, int apply_norm, const float *scale2, int8_t *xq,
+                                     float *x_scale)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        const uint16_t *row = x + t * K;
+        float ir = apply_norm ? row_inv_rms(row, K, eps) : 1.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = bf16_to_f32(row[k]);
+            float y = apply_norm ? (v * ir) * fold[k] : v * fold[k];
+            xq[t * K + k] = quantize_one(y, scale2[1]);
+        }
+        x_scale[t] = scale2[0];
+    }
+}
+
+/*
  * INT8 x INT8 -> INT32 product of the quantised activations xq[T, K] and weights wq[N, K]
  * (both stored with K contiguous): acc[t, n] = sum_k xq[t, k] * wq[n, k].
  * [MIGRATE] section 7 (an integer product accumulated in 32 bits on the tensor cores); the GEMM

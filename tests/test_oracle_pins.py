@@ -225,6 +225,57 @@ def test_rmsnorm_constant_rows_and_scale_invariance(orc):
 
 
 # --------------------------------------------------------------------------------------------
+# Static per-tensor activation scale ("SmoothQuant and W8A8...", "One layer, measured" and
+# "Gotchas"): one scale from the calibration maximum, values past it clipped. Pinned against the
+# per-token quantiser (pinned above) through relations that hold exactly.
+
+@pytest.mark.parametrize("norm", [False, True])
+def test_static_scale_equals_dynamic_on_its_own_calibration_token(orc, norm):
+    # calibrating on a single token and quantising that token gives the per-token result exactly
+    K = 96
+    fold = (0.5 + np.random.default_rng(21).random(K)).astype(np.float32)
+    for seed in range(5):
+        x = rand_bf16((1, K), 40 + seed, scale=3.0)
+        amax_y = orc.calibrate_absmax(x, norm_gamma=fold if norm else None, eps=1e-6)
+        if not norm:
+            amax_y = (amax_y * fold).astype(np.float32)    # exact: one binary32 product per channel
+        s2 = orc.static_scale(amax_y)
+        q_s, xs_s = orc.rmsnorm_smooth_quant_static(x, fold, s2, eps=1e-6, apply_norm=norm)
+        q_d, xs_d = orc.rmsnorm_smooth_quant(x, fold, eps=1e-6, apply_norm=norm)
+        assert np.array_equal(q_s, q_d) and np.array_equal(xs_s, xs_d)
+
+
+def test_static_step_is_the_largest_per_token_step(orc):
+    # delta = m / 127 is monotone in m, and m is the largest row maximum of the calibration set
+    K = 200
+    x = rand_bf16((64, K), 50, scale=2.0)
+    fold = (0.25 + np.random.default_rng(50).random(K)).astype(np.float32)
+    amax_y = orc.calibrate_absmax(x, norm_gamma=fold, eps=1e-6)
+    s2 = orc.static_scale(amax_y)
+    _, xs_d = orc.rmsnorm_smooth_quant(x, fold, eps=1e-6, apply_norm=True)
+    assert s2[0] == xs_d.max()
+    assert s2[1] == np.float32(127) / amax_y.max()          # numpy binary32 division: one IEEE rounding
+
+
+def test_static_codes_clip_and_stay_within_half_a_step(orc):
+    K = 64
+    scale2 = np.array([np.float32(2.0) / np.float32(127), np.float32(127) / np.float32(2.0)], np.float32)
+    fold = np.ones(K, np.float32)
+    v = np.linspace(-6.0, 6.0, K).astype(np.float32)        # the calibrated maximum is 2
+    x = bf16_bits(torch.from_numpy(v[None, :]).to(torch.bfloat16))
+    q, xs = orc.rmsnorm_smooth_quant_static(x, fold, scale2, apply_norm=False)
+    y = bits_to_f64(x)[0]
+    assert np.all(q[0][y >= 2.0] == 127) and np.all(q[0][y <= -2.0] == -127)
+    inside = np.abs(y) < 2.0
+    assert np.all(np.abs(q[0][inside] * float(scale2[0]) - y[inside]) <= float(scale2[0]) * (0.5 + 1e-5))
+    assert np.all(xs == scale2[0])
+    z = orc.static_scale(np.zeros(8, np.float32))
+    assert z[0] == 0 and z[1] == 0
+    qz, xz = orc.rmsnorm_smooth_quant_static(x, fold, z, apply_norm=False)
+    assert not qz.any() and not xz.any()
+
+
+# --------------------------------------------------------------------------------------------
 # INT8 GEMM ("06 -- SmoothQuant...", section 7): numpy int64 matmul is the independent check.
 
 def test_gemm_matches_numpy_int64(orc):
