@@ -123,6 +123,34 @@ sq_status sq_rmsnorm_smooth_quant(const void *x, int64_t T, int64_t K, const flo
                                   int apply_norm, int8_t *xq, float *x_scale, void *stream);
 
 /*
+ * Static per-tensor activation scale (the alternative to per-token scales):
+ *   [W8A8] "One layer, measured" (one static scale per tensor, from the calibration tokens' maximum)
+ *   and "Gotchas" (values past the calibrated maximum are clipped).
+ *   m = max_k fl32(amax[k] * |factor[k]|)  (factor null: m = max_k amax[k]);
+ *   scale2[0] = fl32(m / 127), scale2[1] = fl32(127 / m); both 0 when m = 0.
+ * amax is the per-channel calibration maximum of the activation as the quantiser will form it:
+ *   norm-fed layer: sq_calibrate_absmax(calibration tokens, norm_gamma = fold) (the RMSNorm output
+ *   times the folded weight), factor = NULL;
+ *   layer fed directly: sq_calibrate_absmax(calibration tokens) and factor = fold (= 1/s).
+ * Rounding is monotone, so either way m equals the largest |y| the quantiser would form on the
+ * calibration tokens. amax fp32 [K]; factor nullable fp32 [K]; scale2 fp32 [2] out (device memory).
+ * K >= 1.
+ */
+sq_status sq_static_scale(const float *amax, const float *factor, int64_t K, float *scale2, void *stream);
+
+/*
+ * Online activation quantisation with the static per-tensor scale: y as in
+ * sq_rmsnorm_smooth_quant, then xq[t,k] = clamp(round_half_away(y * scale2[1]), -127, 127) (values
+ * beyond the calibrated maximum saturate) and x_scale[t] = scale2[0] for every token, so
+ * sq_w8a8_linear dequantises with the scalar step times the per-channel weight scale. No per-token
+ * maximum is taken. scale2 fp32 [2] from sq_static_scale (device memory, read by the kernel).
+ * Same arguments and requirements as sq_rmsnorm_smooth_quant otherwise; scale2 4-byte aligned.
+ */
+sq_status sq_rmsnorm_smooth_quant_static(const void *x, int64_t T, int64_t K, const float *fold, float eps,
+                                         int apply_norm, const float *scale2, int8_t *xq, float *x_scale,
+                                         void *stream);
+
+/*
  * W8A8 linear: INT8 x INT8 -> INT32 GEMM with the dequantisation fused into its epilogue.
  *   [MIGRATE] section 7 (the integer product accumulated in 32 bits on the tensor cores, then
  *   scaled by the activation and weight scales); [TAMING] "System Architecture" (the flowchart's

@@ -69,14 +69,28 @@ constexpr uint32_t make_idesc(int M, int N) {
 // serves token counts that fill the SMs with tiles; the 64-wide form serves few tokens (decode),
 // where the weight stream dominates: four times as many tiles, and a deeper ring (8 stages of
 // 24 KB) keeps more weight bytes in flight per SM.
-template <int TN>
+//
+// SWAP: the decode form for at most 128 tokens. The operands trade places: the weight is the MMA's
+// 128-row A operand and the tokens its TN-column (16 .. 128) B operand, so every ring slot carries 16 KB
+// of weight rows and the ring (6 .. 11 stages) keeps up to ~180 KB of the weight stream in flight per
+// SM; the accumulator lanes are output channels and its columns tokens.
+constexpr int DECODE_KS = 2;       // 128-byte K slices per stage of the decode form
+
+template <int TN, bool SWAP = false>
 struct Tile {
-    static constexpr int STAGES = TN == 256 ? 4 : 8;
-    static constexpr int B_STAGE = TN * BK;
+    // K slices per stage: the decode form reads DECODE_KS consecutive 128-byte pieces of every weight
+    // row per stage (longer contiguous DRAM reads); the other forms one.
+    static constexpr int KS = SWAP ? DECODE_KS : 1;
+    static constexpr int A_SLOT = KS * A_STAGE;
+    static constexpr int B_SLICE = TN * BK;
+    static constexpr int B_SLOT = KS * B_SLICE;
+    static constexpr int SPARE = 232448 - 1024 - EPI_WARPS * 2 * OUT_BOX - 2 * COL_TAB - 512;
+    static constexpr int STAGES = SWAP ? (SPARE / (A_SLOT + B_SLOT) > 11 ? 11 : SPARE / (A_SLOT + B_SLOT))
+                                       : TN == 256 ? 4 : 8;
     static constexpr uint32_t TMEM_COLS = 2 * TN;          // two accumulators; a power of two >= 32
     static constexpr int OFF_A = 0;
-    static constexpr int OFF_B = OFF_A + STAGES * A_STAGE;
-    static constexpr int OFF_OUT = OFF_B + STAGES * B_STAGE;
+    static constexpr int OFF_B = OFF_A + STAGES * A_SLOT;
+    static constexpr int OFF_OUT = OFF_B + STAGES * B_SLOT;
     static constexpr int OFF_COL = OFF_OUT + EPI_WARPS * 2 * OUT_BOX;
     static constexpr int OFF_BAR = OFF_COL + 2 * COL_TAB;   // one column table per accumulator
     static constexpr int NBARS = 2 * STAGES + 5;            // full[S], empty[S], tfull[2], tempty[2], done
@@ -84,7 +98,8 @@ struct Tile {
     static constexpr int SMEM_TOTAL = OFF_MISC + 16 + 1024; // slack to align the base to 1024 bytes
     static constexpr uint32_t IDESC = make_idesc(BM, TN);
     static_assert(SMEM_TOTAL <= 232448, "shared memory budget of one sm_100 CTA");
-    static_assert(TN % OUT_COLS == 0 && TN >= 32 && TN <= 256 && (TN & (TN - 1)) == 0, "tile width");
+    static_assert(SWAP ? (TN >= 16 && TN <= 128 && (TN & (TN - 1)) == 0)
+                       : (TN % OUT_COLS == 0 && TN >= 32 && TN <= 256 && (TN & (TN - 1)) == 0), "tile width");
 };
 
 // ------------------------------------------------------------------------------------------------
@@ -369,17 +384,69 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tmem_base, int quad, int 
     tmem_ld_wait();     // nothing of this tile's accumulator is still being read
 }
 
+// 16 columns of this warp's TMEM lane quarter into r[0..15] (asynchronous until tmem_ld_wait).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+// Epilogue of the swapped (decode) form for one tile: thread (quad, lane) owns output channel
+// n = n_base + 32 quad + lane and writes y[t][n] = bf16(float(acc) * (x_scale[t] * w_scale[n]) + bias[n])
+// (each operation rounded once, the same steps as the other forms) for the tile's tokens t < T; a warp
+// writes 32 consecutive channels of a token per store. Optionally writes the raw accumulators.
+template <int TN>
+__device__ __forceinline__ void epilogue_swap(uint32_t tmem_base, int quad, int lane, uint32_t tcol, int n_base, int t0,
+                                              const float *__restrict__ x_scale, const float *__restrict__ w_scale,
+                                              const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ y,
+                                              int32_t *__restrict__ acc_out, int T, int N)
+{
+    const int nq = n_base + quad * 32;
+    if (nq >= N) return;                    // the whole quarter lies beyond N
+    const int n = nq + lane;
+    const bool okn = n < N;
+    const float ws = okn ? __ldg(w_scale + n) : 0.0f;
+    float b = 0.0f;
+    if (bias != nullptr && okn)
+        b = __uint_as_float(static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short *>(bias) + n)) << 16);
+    const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tcol;
+#pragma unroll
+    for (int c = 0; c < TN; c += 16) {
+        if (t0 + c >= T) break;             // uniform in the warp
+        uint32_t r[16];
+        tmem_ld16(tl + c, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) asm volatile("" : "+r"(r[i]));
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int t = t0 + c + j;
+            if (t < T && okn) {
+                const int acc = static_cast<int>(r[j]);
+                const int64_t o = static_cast<int64_t>(t) * N + n;
+                if (acc_out != nullptr) acc_out[o] = acc;
+                float v = __fmul_rn(__int2float_rn(acc), __fmul_rn(__ldg(x_scale + t), ws));
+                if (bias != nullptr) v = __fadd_rn(v, b);
+                y[o] = __float2bfloat16_rn(v);
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------------------------------------
 
-template <int TN>
+template <int TN, bool SWAP>
 __global__ void __launch_bounds__(THREADS, 1)
 k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmY, const float *__restrict__ x_scale,
               const float *__restrict__ w_scale, const __nv_bfloat16 *__restrict__ bias,
-              int32_t *__restrict__ acc_out, int T, int N, int K, int m_tiles, int n_tiles, int a_rows,
-              uint64_t limit_ns)
+              int32_t *__restrict__ acc_out, __nv_bfloat16 *__restrict__ y, int T, int N, int K, int m_tiles,
+              int n_tiles, uint64_t limit_ns)
 {
-    using L = Tile<TN>;
+    using L = Tile<TN, SWAP>;
     constexpr int STAGES = L::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -409,25 +476,15 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     }
     if (warp == 0 && lane == 0) { prefetch_map(&tmA); prefetch_map(&tmB); prefetch_map(&tmY); }
     if (warp == 1) { tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS); tmem_relinquish(); }
-    // Fewer than 128 tokens: only the first a_rows rows of each A slot are loaded; the rest hold
-    // zeros, written once here (their products land in accumulator rows that are never stored).
-    if (a_rows < BM) {
-        const int per_slot = (BM - a_rows) * BK / 16;
-        for (int i = threadIdx.x; i < STAGES * per_slot; i += THREADS) {
-            const int st = i / per_slot;
-            uint8_t *dst = sA + st * A_STAGE + a_rows * BK + (i - st * per_slot) * 16;
-            *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_async_smem();     // visible to the tensor cores (async proxy)
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    const int k_blocks = (K + BK - 1) / BK;
+    constexpr int KS = L::KS;
+    const int k_blocks = (K + KS * BK - 1) / (KS * BK);   // slices beyond K are zero-filled by the TMA
     const int num_tiles = m_tiles * n_tiles;
-    const uint32_t stage_tx = static_cast<uint32_t>(a_rows * BK + L::B_STAGE);
+    constexpr uint32_t stage_tx = static_cast<uint32_t>(L::A_SLOT + L::B_SLOT);
 
     if (warp == 0) {
         // ---------------- TMA producer ----------------
@@ -442,8 +499,11 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait(empty(stage), phase ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
                     mbar_expect_tx(full(stage), stage_tx);
-                    tma_load_2d(smem_u32(sA + stage * A_STAGE), &tmA, full(stage), kb * BK, m * BM);
-                    tma_load_2d(smem_u32(sB + stage * L::B_STAGE), &tmB, full(stage), kb * BK, n * TN);
+#pragma unroll
+                    for (int ks = 0; ks < KS; ++ks) {
+                        tma_load_2d(smem_u32(sA + stage * L::A_SLOT + ks * A_STAGE), &tmA, full(stage), (kb * KS + ks) * BK, m * BM);
+                        tma_load_2d(smem_u32(sB + stage * L::B_SLOT + ks * L::B_SLICE), &tmB, full(stage), (kb * KS + ks) * BK, n * TN);
+                    }
                     ++fills;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -474,12 +534,15 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait(full(stage), phase, limit_ns, abort_flag)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sA + stage * A_STAGE);
-                    const uint32_t b0 = smem_u32(sB + stage * L::B_STAGE);
 #pragma unroll
-                    for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-                        mma_i8(d_tmem, kmajor_sw128_desc(a0 + kk * UMMA_K), kmajor_sw128_desc(b0 + kk * UMMA_K), L::IDESC,
-                               (kb | kk) != 0 ? 1u : 0u);
+                    for (int ks = 0; ks < KS; ++ks) {
+                        const uint32_t a0 = smem_u32(sA + stage * L::A_SLOT + ks * A_STAGE);
+                        const uint32_t b0 = smem_u32(sB + stage * L::B_SLOT + ks * L::B_SLICE);
+#pragma unroll
+                        for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+                            mma_i8(d_tmem, kmajor_sw128_desc(a0 + kk * UMMA_K), kmajor_sw128_desc(b0 + kk * UMMA_K), L::IDESC,
+                                   (kb | ks | kk) != 0 ? 1u : 0u);
+                        }
                     }
                     issued = true;
                     tc_commit(empty(stage));
@@ -498,6 +561,21 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     } else {
         // ---------------- epilogue ----------------
         const int quad = warp & 3;                  // TMEM lanes this warp may read: 32*quad .. +31
+      if constexpr (SWAP) {
+        int lt = 0;
+        for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++lt) {
+            const int buf = lt & 1;
+            const uint32_t use = static_cast<uint32_t>(lt >> 1);
+            if (!mbar_wait(tfull(buf), use & 1u, limit_ns, abort_flag)) { give_up(abort_flag); break; }
+            tc_fence_after();
+            int m, n;
+            tile_coords(t, m_tiles, n_tiles, m, n);
+            epilogue_swap<TN>(tmem_base, quad, lane, static_cast<uint32_t>(buf * TN), m * BM, n * TN, x_scale, w_scale,
+                              bias, y, acc_out, T, N);
+            tc_fence_before();
+            mbar_arrive(tempty(buf));
+        }
+      } else {
         uint8_t *stage_buf = sOut + (warp - 2) * 2 * OUT_BOX;
         const int ep = threadIdx.x - 64;            // 0 .. 127 among the epilogue threads
         int nstores = 0;
@@ -534,6 +612,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         }
         if (lane == 0) bulk_wait_all();
         __syncwarp();
+      }
     }
 
     tc_fence_before();
@@ -783,25 +862,29 @@ sq_status encode_2d(EncodeTiledFn enc, CUtensorMap *map, CUtensorMapDataType dt,
     return SQ_OK;
 }
 
-// Single-SM form with TN-channel tiles: one persistent CTA per SM at most.
-template <int TN>
+// Single-SM forms: one persistent CTA per SM at most. Plain: tiles of 128 tokens x TN channels (A =
+// tokens, B = weight). SWAP: tiles of 128 channels x TN tokens (A = weight, B = tokens).
+template <int TN, bool SWAP>
 sq_status launch_single(const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mY, const float *x_scale,
-                        const float *w_scale, const void *bias, int32_t *acc_out, int64_t T, int64_t N, int64_t K,
-                        int a_rows, int dev, void *stream) {
+                        const float *w_scale, const void *bias, int32_t *acc_out, void *y, int64_t T, int64_t N, int64_t K,
+                        int dev, void *stream) {
+    using L = Tile<TN, SWAP>;
     static int configured[64];
     if (!configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_w8a8_linear<TN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Tile<TN>::SMEM_TOTAL);
+        cudaError_t e = cudaFuncSetAttribute(k_w8a8_linear<TN, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_TOTAL);
         if (e != cudaSuccess) return sq::cuda_status(e, "cudaFuncSetAttribute(w8a8_linear)");
         configured[dev] = 1;
     }
-    const int m_tiles = static_cast<int>((T + BM - 1) / BM);
-    const int n_tiles = static_cast<int>((N + TN - 1) / TN);
+    const int64_t rows = SWAP ? N : T, cols = SWAP ? T : N;
+    const int m_tiles = static_cast<int>((rows + BM - 1) / BM);
+    const int n_tiles = static_cast<int>((cols + TN - 1) / TN);
     const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
     if (tiles > 0x7FFFFFFF) return sq::fail(SQ_ERR_UNSUPPORTED, "sq_w8a8_linear: too many tiles");
     const int grid = static_cast<int>(tiles < sq::sm_count(dev) ? tiles : sq::sm_count(dev));
-    k_w8a8_linear<TN><<<grid, THREADS, Tile<TN>::SMEM_TOTAL, sq::as_stream(stream)>>>(
-        mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out, static_cast<int>(T),
-        static_cast<int>(N), static_cast<int>(K), m_tiles, n_tiles, a_rows, sq::wait_timeout_ns(dev));
+    k_w8a8_linear<TN, SWAP><<<grid, THREADS, L::SMEM_TOTAL, sq::as_stream(stream)>>>(
+        mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out,
+        static_cast<__nv_bfloat16 *>(y), static_cast<int>(T), static_cast<int>(N), static_cast<int>(K), m_tiles, n_tiles,
+        sq::wait_timeout_ns(dev));
     return sq::cuda_status(cudaGetLastError(), "launch(w8a8_linear)");
 }
 
@@ -854,9 +937,21 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, cons
     const int64_t wide_tiles = ((T + BM - 1) / BM) * ((N + BN - 1) / BN);
     const bool narrow = !pair && wide_tiles < sq::sm_count(dev);
     CUtensorMap mA, mB, mY;
-    // one M tile of fewer than 128 tokens: load only the token rows (rounded up to 8)
-    const int a_rows = T < BM ? static_cast<int>((T + 7) / 8 * 8) : BM;
-    st = encode_2d(enc, &mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, T, K, BK, pair ? BM : a_rows, CU_TENSOR_MAP_SWIZZLE_128B, "xq");
+    if (!pair && T <= BM) {
+        // Decode form: the weight streams as the 128-row operand, the tokens (padded to 16 .. 128
+        // with zeros by the TMA) are the narrow one.
+        const int tn = T <= 16 ? 16 : T <= 32 ? 32 : T <= 64 ? 64 : 128;
+        st = encode_2d(enc, &mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, K, N, K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B, "wq");
+        if (st == SQ_OK) st = encode_2d(enc, &mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, T, K, BK, tn, CU_TENSOR_MAP_SWIZZLE_128B, "xq");
+        if (st != SQ_OK) return st;
+        switch (tn) {
+            case 16: return launch_single<16, true>(mA, mB, mA, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+            case 32: return launch_single<32, true>(mA, mB, mA, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+            case 64: return launch_single<64, true>(mA, mB, mA, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+            default: return launch_single<128, true>(mA, mB, mA, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+        }
+    }
+    st = encode_2d(enc, &mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, T, K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B, "xq");
     if (st == SQ_OK) st = encode_2d(enc, &mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, K, N, K, BK, pair ? 128 : narrow ? 64 : BN, CU_TENSOR_MAP_SWIZZLE_128B, "wq");
     if (st == SQ_OK) st = encode_2d(enc, &mY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, T, N * 2, OUT_COLS, OUT_ROWS, CU_TENSOR_MAP_SWIZZLE_64B, "y");
     if (st != SQ_OK) return st;
@@ -897,8 +992,8 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, cons
             "launch(w8a8_linear_pair)");
     }
 
-    return narrow ? launch_single<64>(mA, mB, mY, x_scale, w_scale, bias, acc_out, T, N, K, a_rows, dev, stream)
-                  : launch_single<BN>(mA, mB, mY, x_scale, w_scale, bias, acc_out, T, N, K, a_rows, dev, stream);
+    return narrow ? launch_single<64, false>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream)
+                  : launch_single<BN, false>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
 }
 
 sq_status sq_set_gemm_cta_pair(int enable) {

@@ -67,7 +67,8 @@ constexpr int kMaxStages = 4;
 constexpr uint32_t kSqBias = 485u << 20;   // binary64 exponent bias mapping bf16 x to x * 2^-411
 constexpr unsigned kAll = 0xFFFFFFFFu;
 
-enum { MODE_ABSMAX = 0, MODE_QUANT = 1 };
+// MODE_QSTATIC: the quantiser with one static per-tensor scale (no row maximum; codes clamped).
+enum { MODE_ABSMAX = 0, MODE_QUANT = 1, MODE_QSTATIC = 2 };
 
 struct RowArgs {
     const uint8_t *src;     // row r starts at src + r * ld_bytes (16-byte aligned)
@@ -81,6 +82,7 @@ struct RowArgs {
     float *amax;            // ABSMAX output [K] (running maximum; pre-zeroed when overwriting)
     int8_t *q;              // QUANT output [rows, K]
     float *scale;           // QUANT output [rows]
+    const float *scale2;    // QSTATIC: {delta, 127 / m} of the static per-tensor scale
     unsigned int *status;   // device status word
     uint64_t limit_ns;      // bound of every wait
     int stream_once;        // input larger than half the L2: its lines are evicted first
@@ -186,6 +188,16 @@ __device__ __forceinline__ uint32_t codes2(uint64_t t) {
     return __byte_perm(static_cast<uint32_t>(ql), static_cast<uint32_t>(qh), 0x0040);   // bytes: ql, qh in 0, 1
 }
 
+// codes2 for values that may lie beyond the calibrated range (static scale): t is clamped to
+// [-127, 127] first, so a code saturates at +-127.
+__device__ __forceinline__ uint32_t codes2_clamped(uint64_t t) {
+    uint32_t tl, th;
+    unpack2(t, tl, th);
+    const float a = fminf(fmaxf(__uint_as_float(tl), -kQmax), kQmax);
+    const float b = fminf(fmaxf(__uint_as_float(th), -kQmax), kQmax);
+    return codes2(pack2(a, b));
+}
+
 // 3-input maximum (one instruction on sm_100)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float d;
@@ -223,6 +235,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
     float4 *c_lo = reinterpret_cast<float4 *>(smem + (ring_bytes > red_bytes ? ring_bytes : red_bytes));   // c[8v .. 8v+3]
     float4 *c_hi = c_lo + nvec;                                                                              // c[8v+4 .. 8v+7]
     const bool has_vec = p.vec != nullptr;
+    float sdelta = 0.0f;
+    uint64_t sinv2 = 0;
+    if (MODE == MODE_QSTATIC) {
+        sdelta = __ldg(p.scale2);
+        const float si = __ldg(p.scale2 + 1);
+        sinv2 = pack2(si, si);
+    }
 
     const int64_t units = (p.rows + R - 1) / R;
     const int64_t g0 = static_cast<int64_t>(blockIdx.x) * G + group;
@@ -234,7 +253,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
         for (int g = 0; g < G; ++g) s_abort[g] = 0;
         mbar_init_fence();
     }
-    if (MODE == MODE_QUANT && has_vec) {
+    if (MODE != MODE_ABSMAX && has_vec) {
         const float4 *cv = reinterpret_cast<const float4 *>(p.vec);
         for (int v = tid; v < nvec; v += kThreads) { c_lo[v] = __ldg(cv + 2 * v); c_hi[v] = __ldg(cv + 2 * v + 1); }
     }
@@ -313,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                     const bool in = (FULL || v < nvec) && r < nr;
                     if (MODE == MODE_ABSMAX && !NORM) continue;
                     const uint4 q = in ? rp[r * rv + v] : make_uint4(0u, 0u, 0u, 0u);
-                    if (MODE == MODE_QUANT) xr[r][i] = q;
+                    if (MODE != MODE_ABSMAX) xr[r][i] = q;
                     if (NORM) {
                         if (i & 1) { add_squares<MODE == MODE_ABSMAX>(q.x, a2, a3); add_squares<MODE == MODE_ABSMAX>(q.y, a2, a3); add_squares<MODE == MODE_ABSMAX>(q.z, a2, a3); add_squares<MODE == MODE_ABSMAX>(q.w, a2, a3); }
                         else { add_squares<MODE == MODE_ABSMAX>(q.x, a0, a1); add_squares<MODE == MODE_ABSMAX>(q.y, a0, a1); add_squares<MODE == MODE_ABSMAX>(q.z, a0, a1); add_squares<MODE == MODE_ABSMAX>(q.w, a0, a1); }
@@ -334,10 +353,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                     break;
                 }
                 if (leader) {
-                    if (MODE == MODE_QUANT) refill(j, st);
+                    if (MODE != MODE_ABSMAX) refill(j, st);
                     else if (j > 0) refill(j - 1, st == 0 ? stages - 1 : st - 1);
                 }
-            } else if (MODE == MODE_QUANT) {
+            } else if (MODE != MODE_ABSMAX) {
                 __syncwarp();                                   // the unit is in registers now
                 if (leader) refill(j, st);
             }
@@ -395,6 +414,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                 if (WPR == 1) {
                     __syncwarp();
                     if (leader) refill(j, st);
+                }
+            } else if (MODE == MODE_QSTATIC) {
+                // ---- one pass: y = (x * inv_rms) * c (or x * c, or x), coded with the static scale
+#pragma unroll
+                for (int r = 0; r < R; ++r) {
+                    if (r < nr) {
+                        const uint64_t ir2 = pack2(ir[r], ir[r]);
+                        uint2 *qrow = reinterpret_cast<uint2 *>(p.q + (r0 + r) * static_cast<int64_t>(K));
+#pragma unroll
+                        for (int i = 0; i < VPL; ++i) {
+                            const int v = i * GT + gtid;
+                            if (!(FULL || v < nvec)) continue;
+                            float4 cl = make_float4(1.f, 1.f, 1.f, 1.f), ch = cl;
+                            if (has_vec) { cl = c_lo[v]; ch = c_hi[v]; }
+                            const uint64_t c2[4] = {pack2(cl.x, cl.y), pack2(cl.z, cl.w), pack2(ch.x, ch.y), pack2(ch.z, ch.w)};
+                            uint32_t cc[4];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const uint64_t x2 = bf2_to_f2(word_of(xr[r][i], k));
+                                const uint64_t yy = NORM ? mul2_rn(mul2_rn(x2, ir2), c2[k]) : (has_vec ? mul2_rn(x2, c2[k]) : x2);
+                                cc[k] = codes2_clamped(mul2_rn(yy, sinv2));
+                            }
+                            qrow[v] = make_uint2(__byte_perm(cc[0], cc[1], 0x5410), __byte_perm(cc[2], cc[3], 0x5410));
+                        }
+                    }
+                }
+                if (gtid == 0) {
+#pragma unroll
+                    for (int r = 0; r < R; ++r)
+                        if (r < nr) p.scale[r0 + r] = sdelta;
                 }
             } else {
                 // ---- pass B: y = (x * inv_rms) * c  (or x * c, or x) as element pairs, row maxima
@@ -516,6 +565,30 @@ __global__ void k_fill_zero(float *__restrict__ p, int64_t n) {
 }
 
 // ---------------------------------------------------------------------------------------------
+// Static per-tensor activation scale, [W8A8] "One layer, measured" (one scale per tensor from the
+// calibration tokens' maximum): m = max_k fl(amax[k] * |f[k]|) (f null: max_k amax[k]); scale2 =
+// {m / 127, 127 / m} (zeros when m == 0). One CTA: per-thread maxima, then warp and block maxima.
+__global__ void k_static_scale(const float *__restrict__ amax, const float *__restrict__ f, int64_t K,
+                               float *__restrict__ scale2)
+{
+    __shared__ float s_w[32];
+    float m = 0.0f;
+    for (int64_t k = threadIdx.x; k < K; k += blockDim.x) {
+        const float a = __ldg(amax + k);
+        m = fmaxf(m, f != nullptr ? __fmul_rn(a, fabsf(__ldg(f + k))) : a);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kAll, m, o));
+    if ((threadIdx.x & 31) == 0) s_w[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float t = 0.0f;
+        for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) t = fmaxf(t, s_w[w]);
+        scale2[0] = t > 0.0f ? __fdiv_rn(t, kQmax) : 0.0f;
+        scale2[1] = t > 0.0f ? __fdiv_rn(kQmax, t) : 0.0f;
+    }
+}
+
 // Smoothing factors and fold, [MIGRATE] section 3 and [W8A8] "The trick: move the range into the
 // weights": s = max|X|^alpha / max|W|^(1-alpha) in binary64, rounded once, floored at 1e-5;
 // fold = gamma / s (or 1 / s).
@@ -543,7 +616,7 @@ struct Geo {
 // Dynamic shared memory of a launch with `stages` ring slots per group.
 size_t rows_smem(int K, int mode, const Geo &g, int stages) {
     const size_t slotbytes = static_cast<size_t>(K) * 2 * g.rpu;
-    const size_t ctab = mode == MODE_QUANT ? static_cast<size_t>(K) * 4 : 0;
+    const size_t ctab = mode != MODE_ABSMAX ? static_cast<size_t>(K) * 4 : 0;
     const size_t ring = static_cast<size_t>(g.groups) * stages * slotbytes;
     const size_t red = mode == MODE_ABSMAX ? static_cast<size_t>(g.groups) * K * 4 : 0;
     return (ring > red ? ring : red) + ctab;
@@ -626,7 +699,7 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
     a.stream_once = static_cast<double>(a.rows) * static_cast<double>(a.ld_bytes) > 0.5 * sq::l2_bytes(dev) ? 1 : 0;
     if (a.status == nullptr) return sq::fail(SQ_ERR_CUDA, "device status word unavailable");
     const int64_t units = (a.rows + R - 1) / R;
-    if (MODE == MODE_QUANT) {
+    if (MODE != MODE_ABSMAX) {
         int64_t ctas = (units + G - 1) / G;
         if (ctas > full) ctas = full;
         kern<<<static_cast<unsigned>(ctas), kThreads, smem, st>>>(a);
@@ -771,6 +844,51 @@ sq_status sq_rmsnorm_smooth_quant(const void *x, int64_t T, int64_t K, const flo
     ra.scale = x_scale;
     cudaStream_t st = sq::as_stream(stream);
     return apply_norm ? dispatch_rows<MODE_QUANT, true>(ra, dev, st) : dispatch_rows<MODE_QUANT, false>(ra, dev, st);
+}
+
+sq_status sq_static_scale(const float *amax, const float *factor, int64_t K, float *scale2, void *stream)
+{
+    using sq::fail;
+    if (!amax || !scale2) return fail(SQ_ERR_INVALID_ARG, "sq_static_scale: amax and scale2 are required");
+    if (K < 1) return fail(SQ_ERR_INVALID_ARG, "sq_static_scale: K must be >= 1");
+    if (!sq::aligned(amax, 4) || !sq::aligned(scale2, 4) || (factor && !sq::aligned(factor, 4)))
+        return fail(SQ_ERR_MISALIGNED, "sq_static_scale: fp32 arrays must be 4-byte aligned");
+    int dev = 0;
+    SQ_TRY_ARCH(dev);
+    k_static_scale<<<1, 1024, 0, sq::as_stream(stream)>>>(amax, factor, K, scale2);
+    return sq::cuda_status(cudaGetLastError(), "launch(static_scale)");
+}
+
+sq_status sq_rmsnorm_smooth_quant_static(const void *x, int64_t T, int64_t K, const float *fold, float eps,
+                                         int apply_norm, const float *scale2, int8_t *xq, float *x_scale,
+                                         void *stream)
+{
+    using sq::fail;
+    if (T < 0 || K < 8) return fail(SQ_ERR_INVALID_ARG, "sq_rmsnorm_smooth_quant_static: need T >= 0 and K >= 8");
+    if (!fold || !scale2) return fail(SQ_ERR_INVALID_ARG, "sq_rmsnorm_smooth_quant_static: fold and scale2 are required");
+    if (T > 0 && (!x || !xq || !x_scale))
+        return fail(SQ_ERR_INVALID_ARG, "sq_rmsnorm_smooth_quant_static: x, xq and x_scale are required");
+    if (K % 8 != 0) return fail(SQ_ERR_MISALIGNED, "sq_rmsnorm_smooth_quant_static: K must be a multiple of 8");
+    if (K > kMaxK) return fail(SQ_ERR_UNSUPPORTED, "sq_rmsnorm_smooth_quant_static: K must be <= %d", kMaxK);
+    if ((x && !sq::aligned(x, 16)) || (xq && !sq::aligned(xq, 8)) || !sq::aligned(fold, 16) || !sq::aligned(scale2, 4) ||
+        (x_scale && !sq::aligned(x_scale, 4)))
+        return fail(SQ_ERR_MISALIGNED,
+                    "sq_rmsnorm_smooth_quant_static: x and fold 16-byte, xq 8-byte, scale2 and x_scale 4-byte alignment required");
+    int dev = 0;
+    SQ_TRY_ARCH(dev);
+    if (T == 0) return SQ_OK;
+    RowArgs ra = {};
+    ra.src = static_cast<const uint8_t *>(x);
+    ra.rows = T;
+    ra.ld_bytes = K * 2;
+    ra.K = static_cast<int>(K);
+    ra.vec = fold;
+    ra.eps = eps;
+    ra.q = xq;
+    ra.scale = x_scale;
+    ra.scale2 = scale2;
+    cudaStream_t st = sq::as_stream(stream);
+    return apply_norm ? dispatch_rows<MODE_QSTATIC, true>(ra, dev, st) : dispatch_rows<MODE_QSTATIC, false>(ra, dev, st);
 }
 
 }  // extern "C"

@@ -16,7 +16,8 @@ import torch
 __all__ = [
     "SQError", "lib", "sq_calibrate_absmax", "sq_compute_scales", "sq_smooth_quantize_weight",
     "sq_rmsnorm_smooth_quant", "sq_w8a8_linear", "sq_w8a8_linear_workspace_size", "sq_device_status",
-    "sq_set_wait_timeout_ns", "sq_selftest_wait_timeout", "sq_set_gemm_cta_pair", "sq_status_string", "sq_last_error",
+    "sq_set_wait_timeout_ns", "sq_selftest_wait_timeout", "sq_set_gemm_cta_pair",
+    "sq_static_scale", "sq_rmsnorm_smooth_quant_static", "sq_status_string", "sq_last_error",
     "sq_version", "LIB_PATH", "EXPORTS",
 ]
 
@@ -44,6 +45,8 @@ EXPORTS = {
     "sq_set_wait_timeout_ns": (_i, [_u64]),
     "sq_selftest_wait_timeout": (_i, [_p]),
     "sq_set_gemm_cta_pair": (_i, [_i]),
+    "sq_static_scale": (_i, [_p, _p, _i64, _p, _p]),
+    "sq_rmsnorm_smooth_quant_static": (_i, [_p, _i64, _i64, _p, _f, _i, _p, _p, _p, _p]),
 }
 
 
@@ -180,6 +183,33 @@ def sq_rmsnorm_smooth_quant(x: torch.Tensor, fold: torch.Tensor, eps: float = 1e
     x_scale = torch.empty(T, dtype=torch.float32, device=x.device) if x_scale is None else _dev(x_scale, "x_scale", torch.float32)
     _check(_lib.sq_rmsnorm_smooth_quant(_ptr(x), T, K, _ptr(fold), float(eps), int(bool(apply_norm)), _ptr(xq),
                                         _ptr(x_scale), _stream(stream)), "sq_rmsnorm_smooth_quant")
+    return xq, x_scale
+
+
+def sq_static_scale(amax: torch.Tensor, factor: Optional[torch.Tensor] = None, scale2: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """Static per-tensor activation scale {delta, 127/m} from a calibration maximum; see sq.h."""
+    _dev(amax, "amax", torch.float32)
+    K = amax.shape[0]
+    if factor is not None:
+        _dev(factor, "factor", torch.float32)
+    scale2 = torch.empty(2, dtype=torch.float32, device=amax.device) if scale2 is None else _dev(scale2, "scale2", torch.float32)
+    _check(_lib.sq_static_scale(_ptr(amax), _ptr(factor), K, _ptr(scale2), _stream(stream)), "sq_static_scale")
+    return scale2
+
+
+def sq_rmsnorm_smooth_quant_static(x: torch.Tensor, fold: torch.Tensor, scale2: torch.Tensor, eps: float = 1e-6,
+                                   apply_norm: bool = True, xq: Optional[torch.Tensor] = None,
+                                   x_scale: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Fused RMSNorm (folded 1/s) + INT8 with the static per-tensor scale; see sq.h."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(fold, "fold", torch.float32)
+    _dev(scale2, "scale2", torch.float32)
+    T, K = x.shape
+    xq = torch.empty(T, K, dtype=torch.int8, device=x.device) if xq is None else _dev(xq, "xq", torch.int8)
+    x_scale = torch.empty(T, dtype=torch.float32, device=x.device) if x_scale is None else _dev(x_scale, "x_scale", torch.float32)
+    _check(_lib.sq_rmsnorm_smooth_quant_static(_ptr(x), T, K, _ptr(fold), float(eps), int(bool(apply_norm)), _ptr(scale2),
+                                               _ptr(xq), _ptr(x_scale), _stream(stream)), "sq_rmsnorm_smooth_quant_static")
     return xq, x_scale
 
 

@@ -93,6 +93,18 @@ def test_scales_argument_checks(sqmod):
     assert L.sq_compute_scales(FAKE + 2, FAKE, 16, 0.5, None, FAKE, None, None) == SQ_ERR_MISALIGNED
 
 
+def test_static_scale_argument_checks(sqmod):
+    L = sqmod.lib()
+    assert L.sq_static_scale(None, None, 16, FAKE, None) == SQ_ERR_INVALID_ARG
+    assert L.sq_static_scale(FAKE, None, 0, FAKE, None) == SQ_ERR_INVALID_ARG
+    assert L.sq_static_scale(FAKE + 2, None, 16, FAKE, None) == SQ_ERR_MISALIGNED
+    q = L.sq_rmsnorm_smooth_quant_static
+    assert q(FAKE, 4, 64, FAKE, 1e-6, 1, None, FAKE, FAKE, None) == SQ_ERR_INVALID_ARG       # no scale2
+    assert q(FAKE, 4, 12, FAKE, 1e-6, 1, FAKE, FAKE, FAKE, None) == SQ_ERR_MISALIGNED        # K % 8
+    assert q(FAKE, 4, 32768, FAKE, 1e-6, 1, FAKE, FAKE, FAKE, None) == SQ_ERR_UNSUPPORTED
+    assert q(FAKE + 8, 4, 64, FAKE, 1e-6, 1, FAKE, FAKE, FAKE, None) == SQ_ERR_MISALIGNED    # x alignment
+
+
 def test_quant_argument_checks(sqmod):
     L = sqmod.lib()
     assert L.sq_smooth_quantize_weight(FAKE, 4, 12, None, FAKE, FAKE, None) == SQ_ERR_MISALIGNED

@@ -269,6 +269,66 @@ def test_cta_pair_gemm_matches(sq, orc, T, N, K, bias):
     check_linear(sq, orc, xq, xs, wq, ws, b, outs[1][0], outs[1][1], rows=rows)
 
 
+# The decode form (weights as the 128-row MMA operand, tokens padded to 16, 32, 64 or 128 columns):
+# every padding bucket and its edges, N not a multiple of 128, K not a multiple of the 128-byte stage.
+@pytest.mark.parametrize("T", [16, 17, 33, 65, 100, 128])
+def test_decode_form_buckets(sq, orc, T):
+    dev = "cuda"
+    N, K = 1000, 2064
+    g = torch.Generator(device="cpu").manual_seed(5 * T)
+    xq = torch.randint(-127, 128, (T, K), dtype=torch.int8, generator=g).to(dev)
+    wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, generator=g).to(dev)
+    xs = (torch.rand(T, generator=g) * 1e-2).to(dev)
+    ws = (torch.rand(N, generator=g) * 1e-2).to(dev)
+    b = torch.randn(N, generator=g).to(torch.bfloat16).to(dev)
+    acc = torch.empty(T, N, dtype=torch.int32, device=dev)
+    y = sq.sq_w8a8_linear(xq, xs, wq, ws, bias=b, acc_out=acc)
+    ok_status(sq)
+    check_linear(sq, orc, xq, xs, wq, ws, b, y, acc)
+
+
+# Static per-tensor activation scale: the calibration maximum of the quantiser's own y, the per-tensor
+# step, and the clipping quantiser, against the oracle fed the same inputs; online tokens include
+# values well beyond the calibration range, so saturation is exercised.
+@pytest.mark.parametrize("K,norm", [(1024, True), (1040, False), (4096, True), (4096, False), (8192, True)])
+def test_static_scale_path(sq, orc, K, norm):
+    dev = "cuda"
+    Tc, T, N = 1500, 777, 264
+    ch = synth.outlier_channels(K, synth.OutlierSpec(max(1, K // 256), 10.0, 25.0), K)
+    Xc = synth.outlier_tokens(Tc, K, ch, K + 1, dev)
+    X = synth.outlier_tokens(T, K, ch, K + 2, dev)
+    W = synth.normal_weight(N, K, K + 3, dev)
+    gamma = synth.norm_gamma(K, K + 4, dev) if norm else None
+    amax = sq.sq_calibrate_absmax(Xc, norm_gamma=gamma)
+    s, fold = sq.sq_compute_scales(amax, sq.sq_calibrate_absmax(W), 0.5, gamma=gamma)
+    fold_h = hnp(fold)
+    # the first 40 tokens go beyond anything calibration saw, so their codes clip: one channel (the
+    # one with the largest fold) dominates each of them (scaling a whole token would not do it with
+    # the norm, which is scale free)
+    X[:40, int(np.argmax(np.abs(fold_h)))] = 1000.0
+    if norm:
+        amax_y = sq.sq_calibrate_absmax(Xc, norm_gamma=fold)
+        s2 = sq.sq_static_scale(amax_y)
+        amax_y_o = orc.calibrate_absmax(h16(Xc), norm_gamma=fold_h)
+    else:
+        amax_x = sq.sq_calibrate_absmax(Xc)
+        s2 = sq.sq_static_scale(amax_x, factor=fold)
+        amax_y_o = (orc.calibrate_absmax(h16(Xc)) * np.abs(fold_h)).astype(np.float32)
+    ok_status(sq)
+    s2_o = orc.static_scale(amax_y_o)
+    assert np.array_equal(hnp(s2), s2_o), f"static scale differs: {hnp(s2)} vs {s2_o}"
+    xq, xs = sq.sq_rmsnorm_smooth_quant_static(X, fold, s2, apply_norm=norm)
+    xq_o, xs_o = orc.rmsnorm_smooth_quant_static(h16(X), fold_h, hnp(s2), apply_norm=norm)
+    assert np.array_equal(hnp(xs), xs_o) and np.all(hnp(xs) == hnp(s2)[0])
+    assert np.array_equal(hnp(xq), xq_o), f"{int((hnp(xq) != xq_o).sum())} static codes differ"
+    assert np.all((np.abs(xq_o[:40]) == 127).sum(axis=1) >= 1)   # every planted token saturates
+    wq, ws = sq.sq_smooth_quantize_weight(W, s)
+    acc = torch.empty(T, N, dtype=torch.int32, device=dev)
+    y = sq.sq_w8a8_linear(xq, xs, wq, ws, acc_out=acc)
+    check_linear(sq, orc, xq, xs, wq, ws, None, y, acc)
+    ok_status(sq)
+
+
 def test_deterministic_bytes(sq):
     w = synth.WORKLOADS[1]
     d = synth.group_inputs(w, 0, "cuda", T=1000)
