@@ -15,7 +15,7 @@ from . import build as _build
 
 __all__ = [
     "calibrate_absmax", "compute_scales", "smooth_quantize_weight", "rmsnorm_smooth_quant",
-    "static_scale", "rmsnorm_smooth_quant_static",
+    "static_scale", "rmsnorm_smooth_quant_static", "fold_into_prev_linear", "fold_into_w_scale",
     "gemm_s8", "dequant", "w8a8_linear", "f32_to_bf16", "bf16_to_f32", "set_threads", "lib",
 ]
 
@@ -39,6 +39,8 @@ def lib() -> ctypes.CDLL:
             L.orc_rmsnorm_smooth_quant.argtypes = [_p, _i64, _i64, _p, ctypes.c_float, ctypes.c_int, _p, _p, _p]
             L.orc_static_scale.argtypes = [_p, _i64, _p]
             L.orc_rmsnorm_smooth_quant_static.argtypes = [_p, _i64, _i64, _p, ctypes.c_float, ctypes.c_int, _p, _p, _p]
+            L.orc_fold_into_prev_linear.argtypes = [_p, _p, _i64, _i64, _p, _p, _p]
+            L.orc_fold_into_w_scale.argtypes = [_p, _i64, _p, _p]
             L.orc_gemm_s8.argtypes = [_p, _i64, _p, _i64, _i64, _p, _i64, _p, _i64, _p]
             L.orc_dequant.argtypes = [_p, _p, _p, _p, _p, _i64, _p, _i64, _p]
             L.orc_f32_to_bf16.argtypes = [ctypes.c_float]
@@ -145,6 +147,28 @@ def rmsnorm_smooth_quant_static(x, fold, scale2, eps=1e-6, apply_norm=True):
     lib().orc_rmsnorm_smooth_quant_static(_ptr(x), T, K, _ptr(f), float(eps), int(bool(apply_norm)), _ptr(s2),
                                           _ptr(xq), _ptr(xs))
     return xq, xs
+
+
+def fold_into_prev_linear(w_prev, b_prev, fold):
+    """Previous bf16 linear [K, Kp] with its output channel j multiplied by fold[j] ([MIGRATE]
+    section 7). Returns (w_out, b_out) as bf16 bits (b_out None without a bias)."""
+    w = _need(w_prev, np.uint16, "w_prev")
+    K, Kp = w.shape
+    f = _need(fold, np.float32, "fold")
+    b = None if b_prev is None else _need(b_prev, np.uint16, "b_prev")
+    wo = np.empty((K, Kp), np.uint16)
+    bo = None if b is None else np.empty(K, np.uint16)
+    lib().orc_fold_into_prev_linear(_ptr(w), _ptr(b), K, Kp, _ptr(f), _ptr(wo), _ptr(bo))
+    return wo, bo
+
+
+def fold_into_w_scale(w_scale, fold):
+    """Per-output-channel dequantisation scale of an INT8 previous layer times fold (binary32)."""
+    ws = _need(w_scale, np.float32, "w_scale")
+    f = _need(fold, np.float32, "fold")
+    out = np.empty_like(ws)
+    lib().orc_fold_into_w_scale(_ptr(ws), ws.shape[0], _ptr(f), _ptr(out))
+    return out
 
 
 def gemm_s8(xq, wq, rows=None, cols=None):

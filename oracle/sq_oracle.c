@@ -255,6 +255,31 @@ void orc_rmsnorm_smooth_quant_static(const uint16_t *x, int64_t T, int64_t K, co
 }
 
 /*
+ * Fold of the smoothing into the previous linear layer, [MIGRATE] section 7 (the division X / s is
+ * absorbed by multiplying the previous layer's output-column-j weights by 1 / s_j, so the smoothed
+ * layer's input arrives already divided). The previous layer's weight is stored [K, Kp] (output
+ * channel j of that layer = input channel j of the smoothed one), bf16:
+ *   w_out[j, i] = bf16_rn(w[j, i] * f[j]),  b_out[j] = bf16_rn(b[j] * f[j]),  f = fl32(1 / s) (the
+ *   fold vector of orc_compute_scales without gamma).
+ * For an INT8 previous layer the same factor goes into its per-output-channel dequantisation:
+ *   w_scale_out[j] = w_scale[j] * f[j] (binary32); its bias as above.
+ */
+void orc_fold_into_prev_linear(const uint16_t *w, const uint16_t *b, int64_t K, int64_t Kp, const float *f,
+                               uint16_t *w_out, uint16_t *b_out)
+{
+    for (int64_t j = 0; j < K; ++j) {
+        for (int64_t i = 0; i < Kp; ++i)
+            w_out[j * Kp + i] = f32_to_bf16_rne(bf16_to_f32(w[j * Kp + i]) * f[j]);
+        if (b) b_out[j] = f32_to_bf16_rne(bf16_to_f32(b[j]) * f[j]);
+    }
+}
+
+void orc_fold_into_w_scale(const float *w_scale, int64_t K, const float *f, float *w_scale_out)
+{
+    for (int64_t j = 0; j < K; ++j) w_scale_out[j] = w_scale[j] * f[j];
+}
+
+/*
  * INT8 x INT8 -> INT32 product of the quantised activations xq[T, K] and weights wq[N, K]
  * (both stored with K contiguous): acc[t, n] = sum_k xq[t, k] * wq[n, k].
  * [MIGRATE] section 7 (an integer product accumulated in 32 bits on the tensor cores); the GEMM

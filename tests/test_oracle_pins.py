@@ -276,6 +276,42 @@ def test_static_codes_clip_and_stay_within_half_a_step(orc):
 
 
 # --------------------------------------------------------------------------------------------
+# Fold into the previous linear's output columns ("06 -- SmoothQuant...", section 7): with powers
+# of two the fold is exact and the chain is unchanged; otherwise each weight is within half a bf16
+# step of w / s.
+
+def test_fold_into_prev_linear_power_of_two_is_exact(orc):
+    K, Kp, N = 64, 48, 40
+    g = torch.Generator().manual_seed(60)
+    w_prev = bf16_bits((torch.randn(K, Kp, generator=g) * 0.05).to(torch.bfloat16))
+    b_prev = bf16_bits((torch.randn(K, generator=g) * 0.05).to(torch.bfloat16))
+    s = (2.0 ** torch.randint(-4, 5, (K,), generator=g).double()).numpy().astype(np.float32)
+    fold = (np.float32(1) / s).astype(np.float32)
+    wo, bo = orc.fold_into_prev_linear(w_prev, b_prev, fold)
+    assert np.array_equal(bits_to_f64(wo), bits_to_f64(w_prev) / s[:, None].astype(np.float64))
+    assert np.array_equal(bits_to_f64(bo), bits_to_f64(b_prev) / s.astype(np.float64))
+    # the method's invariance: (h W_prev^T + b) diag(1/s) diag(s) W^T = (h W_prev^T + b) W^T
+    h = torch.randn(7, Kp, generator=g).double().numpy()
+    w = torch.randn(N, K, generator=g).double().numpy()
+    y_prev = h @ bits_to_f64(w_prev).T + bits_to_f64(b_prev)
+    y_fold = h @ bits_to_f64(wo).T + bits_to_f64(bo)
+    assert np.allclose((y_fold * s) @ w.T, y_prev @ w.T, rtol=1e-12, atol=1e-12)
+
+
+def test_fold_into_prev_linear_rounding_and_w_scale(orc):
+    K, Kp = 32, 40
+    g = torch.Generator().manual_seed(61)
+    w_prev = bf16_bits(torch.randn(K, Kp, generator=g).to(torch.bfloat16))
+    fold = (0.3 + np.random.default_rng(61).random(K)).astype(np.float32)
+    wo, bo = orc.fold_into_prev_linear(w_prev, None, fold)
+    assert bo is None
+    exact = bits_to_f64(w_prev) * fold[:, None].astype(np.float64)
+    assert np.all(np.abs(bits_to_f64(wo) - exact) <= np.abs(exact) * 2.0 ** -8 + 1e-30)
+    ws = (np.random.default_rng(62).random(K) * 1e-2).astype(np.float32)
+    assert np.array_equal(orc.fold_into_w_scale(ws, fold), ws * fold)     # one binary32 product each
+
+
+# --------------------------------------------------------------------------------------------
 # INT8 GEMM ("06 -- SmoothQuant...", section 7): numpy int64 matmul is the independent check.
 
 def test_gemm_matches_numpy_int64(orc):
