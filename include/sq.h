@@ -151,6 +151,28 @@ sq_status sq_rmsnorm_smooth_quant_static(const void *x, int64_t T, int64_t K, co
                                          void *stream);
 
 /*
+ * Fold of the smoothing into the previous linear layer instead of a norm:
+ *   [MIGRATE] section 7 (multiply the previous layer's output-column-j weights by 1/s_j; the
+ *   smoothed layer's input then arrives divided by s, at no run-time cost).
+ * The previous layer's weight w is bf16 [K, Kp] row-major (row j = its output channel j = input
+ * channel j of the smoothed layer), its bias b nullable bf16 [K]; fold fp32 [K] = fl32(1/s) (from
+ * sq_compute_scales with gamma = NULL):
+ *   w_out[j, i] = bf16_rn(w[j, i] * fold[j]),  b_out[j] = bf16_rn(b[j] * fold[j]).
+ * The smoothed layer then quantises its input with fold = 1 (sq_rmsnorm_smooth_quant, apply_norm 0).
+ * w_out / b_out may equal w / b (in place). Requirements: K >= 0, Kp >= 8, Kp % 8 == 0; w, w_out
+ * 16-byte aligned; b_out required when b is given.
+ */
+sq_status sq_fold_into_prev_linear(const void *w, const void *b, int64_t K, int64_t Kp, const float *fold,
+                                   void *w_out, void *b_out, void *stream);
+
+/*
+ * The same fold for an INT8 previous layer: its per-output-channel dequantisation scale absorbs it,
+ * w_scale_out[j] = fl32(w_scale[j] * fold[j]) (its bf16 bias as in sq_fold_into_prev_linear).
+ * fp32 [K] arrays, K >= 1; w_scale_out may equal w_scale.
+ */
+sq_status sq_fold_into_w_scale(const float *w_scale, int64_t K, const float *fold, float *w_scale_out, void *stream);
+
+/*
  * W8A8 linear: INT8 x INT8 -> INT32 GEMM with the dequantisation fused into its epilogue.
  *   [MIGRATE] section 7 (the integer product accumulated in 32 bits on the tensor cores, then
  *   scaled by the activation and weight scales); [TAMING] "System Architecture" (the flowchart's

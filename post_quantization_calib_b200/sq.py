@@ -17,7 +17,7 @@ __all__ = [
     "SQError", "lib", "sq_calibrate_absmax", "sq_compute_scales", "sq_smooth_quantize_weight",
     "sq_rmsnorm_smooth_quant", "sq_w8a8_linear", "sq_w8a8_linear_workspace_size", "sq_device_status",
     "sq_set_wait_timeout_ns", "sq_selftest_wait_timeout", "sq_set_gemm_cta_pair",
-    "sq_static_scale", "sq_rmsnorm_smooth_quant_static", "sq_status_string", "sq_last_error",
+    "sq_static_scale", "sq_rmsnorm_smooth_quant_static", "sq_fold_into_prev_linear", "sq_fold_into_w_scale", "sq_status_string", "sq_last_error",
     "sq_version", "LIB_PATH", "EXPORTS",
 ]
 
@@ -47,6 +47,8 @@ EXPORTS = {
     "sq_set_gemm_cta_pair": (_i, [_i]),
     "sq_static_scale": (_i, [_p, _p, _i64, _p, _p]),
     "sq_rmsnorm_smooth_quant_static": (_i, [_p, _i64, _i64, _p, _f, _i, _p, _p, _p, _p]),
+    "sq_fold_into_prev_linear": (_i, [_p, _p, _i64, _i64, _p, _p, _p, _p]),
+    "sq_fold_into_w_scale": (_i, [_p, _i64, _p, _p, _p]),
 }
 
 
@@ -211,6 +213,33 @@ def sq_rmsnorm_smooth_quant_static(x: torch.Tensor, fold: torch.Tensor, scale2: 
     _check(_lib.sq_rmsnorm_smooth_quant_static(_ptr(x), T, K, _ptr(fold), float(eps), int(bool(apply_norm)), _ptr(scale2),
                                                _ptr(xq), _ptr(x_scale), _stream(stream)), "sq_rmsnorm_smooth_quant_static")
     return xq, x_scale
+
+
+def sq_fold_into_prev_linear(w: torch.Tensor, fold: torch.Tensor, b: Optional[torch.Tensor] = None,
+                             w_out: Optional[torch.Tensor] = None, b_out: Optional[torch.Tensor] = None,
+                             stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Previous bf16 linear [K, Kp] with output channel j multiplied by fold[j]; see sq.h."""
+    _dev(w, "w", torch.bfloat16)
+    _dev(fold, "fold", torch.float32)
+    K, Kp = w.shape
+    w_out = torch.empty_like(w) if w_out is None else _dev(w_out, "w_out", torch.bfloat16)
+    if b is not None:
+        _dev(b, "b", torch.bfloat16)
+        b_out = torch.empty_like(b) if b_out is None else _dev(b_out, "b_out", torch.bfloat16)
+    _check(_lib.sq_fold_into_prev_linear(_ptr(w), _ptr(b), K, Kp, _ptr(fold), _ptr(w_out), _ptr(b_out) if b is not None else None,
+                                         _stream(stream)), "sq_fold_into_prev_linear")
+    return w_out, (b_out if b is not None else None)
+
+
+def sq_fold_into_w_scale(w_scale: torch.Tensor, fold: torch.Tensor, out: Optional[torch.Tensor] = None,
+                         stream=None) -> torch.Tensor:
+    """INT8 previous layer: per-channel dequantisation scale times fold; see sq.h."""
+    _dev(w_scale, "w_scale", torch.float32)
+    _dev(fold, "fold", torch.float32)
+    out = torch.empty_like(w_scale) if out is None else _dev(out, "out", torch.float32)
+    _check(_lib.sq_fold_into_w_scale(_ptr(w_scale), w_scale.shape[0], _ptr(fold), _ptr(out), _stream(stream)),
+           "sq_fold_into_w_scale")
+    return out
 
 
 def sq_w8a8_linear(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,

@@ -105,6 +105,17 @@ def test_static_scale_argument_checks(sqmod):
     assert q(FAKE + 8, 4, 64, FAKE, 1e-6, 1, FAKE, FAKE, FAKE, None) == SQ_ERR_MISALIGNED    # x alignment
 
 
+def test_fold_argument_checks(sqmod):
+    L = sqmod.lib()
+    f = L.sq_fold_into_prev_linear
+    assert f(FAKE, None, 4, 64, None, FAKE, None, None) == SQ_ERR_INVALID_ARG      # no fold
+    assert f(FAKE, FAKE, 4, 64, FAKE, FAKE, None, None) == SQ_ERR_INVALID_ARG      # bias without b_out
+    assert f(FAKE, None, 4, 12, FAKE, FAKE, None, None) == SQ_ERR_MISALIGNED       # Kp % 8
+    assert f(FAKE + 8, None, 4, 64, FAKE, FAKE, None, None) == SQ_ERR_MISALIGNED   # w alignment
+    assert L.sq_fold_into_w_scale(FAKE, 0, FAKE, FAKE, None) == SQ_ERR_INVALID_ARG
+    assert L.sq_fold_into_w_scale(FAKE + 2, 8, FAKE, FAKE, None) == SQ_ERR_MISALIGNED
+
+
 def test_quant_argument_checks(sqmod):
     L = sqmod.lib()
     assert L.sq_smooth_quantize_weight(FAKE, 4, 12, None, FAKE, FAKE, None) == SQ_ERR_MISALIGNED

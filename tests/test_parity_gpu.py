@@ -329,6 +329,28 @@ def test_static_scale_path(sq, orc, K, norm):
     ok_status(sq)
 
 
+# Fold into the previous linear layer: bit-exact against the oracle, in place as well; then the
+# smoothed layer fed by the folded layer's output quantises with fold = 1 and matches the oracle.
+@pytest.mark.parametrize("K,Kp,bias", [(4096, 4096, True), (1000, 264, False), (8, 8, True)])
+def test_fold_into_prev_linear(sq, orc, K, Kp, bias):
+    dev = "cuda"
+    g = torch.Generator(device="cpu").manual_seed(K + Kp)
+    w = (torch.randn(K, Kp, generator=g) * 0.05).to(torch.bfloat16).to(dev)
+    b = (torch.randn(K, generator=g) * 0.05).to(torch.bfloat16).to(dev) if bias else None
+    fold = (0.2 + torch.rand(K, generator=g) * 5).to(dev)
+    wo, bo = sq.sq_fold_into_prev_linear(w, fold, b)
+    wo_o, bo_o = orc.fold_into_prev_linear(h16(w), h16(b) if bias else None, hnp(fold))
+    assert np.array_equal(h16(wo), wo_o)
+    if bias:
+        assert np.array_equal(h16(bo), bo_o)
+    w2, b2 = w.clone(), (b.clone() if bias else None)
+    sq.sq_fold_into_prev_linear(w2, fold, b2, w_out=w2, b_out=b2)          # in place
+    assert torch.equal(w2, wo) and (not bias or torch.equal(b2, bo))
+    ws = torch.rand(K, generator=g).to(dev) * 1e-2
+    assert np.array_equal(hnp(sq.sq_fold_into_w_scale(ws, fold)), orc.fold_into_w_scale(hnp(ws), hnp(fold)))
+    ok_status(sq)
+
+
 def test_deterministic_bytes(sq):
     w = synth.WORKLOADS[1]
     d = synth.group_inputs(w, 0, "cuda", T=1000)
