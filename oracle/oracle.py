@@ -16,6 +16,8 @@ from . import build as _build
 __all__ = [
     "calibrate_absmax", "compute_scales", "smooth_quantize_weight", "rmsnorm_smooth_quant",
     "static_scale", "rmsnorm_smooth_quant_static", "fold_into_prev_linear", "fold_into_w_scale",
+    "e4m3_encode", "e4m3_decode", "smooth_quantize_weight_f8", "rmsnorm_smooth_quant_f8", "gemm_f8", "dequant_f32",
+    "w8a8_linear_f8",
     "gemm_s8", "dequant", "w8a8_linear", "f32_to_bf16", "bf16_to_f32", "set_threads", "lib",
 ]
 
@@ -41,6 +43,14 @@ def lib() -> ctypes.CDLL:
             L.orc_rmsnorm_smooth_quant_static.argtypes = [_p, _i64, _i64, _p, ctypes.c_float, ctypes.c_int, _p, _p, _p]
             L.orc_fold_into_prev_linear.argtypes = [_p, _p, _i64, _i64, _p, _p, _p]
             L.orc_fold_into_w_scale.argtypes = [_p, _i64, _p, _p]
+            L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+            L.orc_e4m3_encode.restype = ctypes.c_uint8
+            L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+            L.orc_e4m3_decode.restype = ctypes.c_float
+            L.orc_smooth_quantize_weight_f8.argtypes = [_p, _i64, _i64, _p, _p, _p, _p]
+            L.orc_rmsnorm_smooth_quant_f8.argtypes = [_p, _i64, _i64, _p, ctypes.c_float, ctypes.c_int, _p, _p, _p]
+            L.orc_gemm_f8.argtypes = [_p, _i64, _p, _i64, _i64, _p, _i64, _p, _i64, _p]
+            L.orc_dequant_f32.argtypes = [_p, _p, _p, _p, _p, _i64, _p, _i64, _p]
             L.orc_gemm_s8.argtypes = [_p, _i64, _p, _i64, _i64, _p, _i64, _p, _i64, _p]
             L.orc_dequant.argtypes = [_p, _p, _p, _p, _p, _i64, _p, _i64, _p]
             L.orc_f32_to_bf16.argtypes = [ctypes.c_float]
@@ -169,6 +179,81 @@ def fold_into_w_scale(w_scale, fold):
     out = np.empty_like(ws)
     lib().orc_fold_into_w_scale(_ptr(ws), ws.shape[0], _ptr(f), _ptr(out))
     return out
+
+
+def e4m3_encode(a):
+    """binary32 -> E4M3 codes (nearest, ties to even, saturating at 448), element by element."""
+    a = np.asarray(a, np.float32)
+    f = lib().orc_e4m3_encode
+    return np.array([f(float(v)) for v in a.ravel()], np.uint8).reshape(a.shape)
+
+
+def e4m3_decode(c):
+    """E4M3 codes -> binary32 values."""
+    c = np.asarray(c, np.uint8)
+    f = lib().orc_e4m3_decode
+    return np.array([f(int(v)) for v in c.ravel()], np.float32).reshape(c.shape)
+
+
+def smooth_quantize_weight_f8(w, s=None):
+    """diag(s)*W then E4M3 per output row (scale max/448). Returns (wq uint8 codes, w_scale)."""
+    w = _need(w, np.uint16, "w")
+    N, K = w.shape
+    wq = np.empty((N, K), np.uint8)
+    ws = np.empty(N, np.float32)
+    work = np.empty(K, np.float32)
+    sv = None if s is None else _need(s, np.float32, "s")
+    lib().orc_smooth_quantize_weight_f8(_ptr(w), N, K, _ptr(sv), _ptr(wq), _ptr(ws), _ptr(work))
+    return wq, ws
+
+
+def rmsnorm_smooth_quant_f8(x, fold, eps=1e-6, apply_norm=True):
+    """(RMSNorm with folded weight, or x*fold) then E4M3 per token. Returns (xq uint8 codes, x_scale)."""
+    x = _need(x, np.uint16, "x")
+    T, K = x.shape
+    f = _need(fold, np.float32, "fold")
+    xq = np.empty((T, K), np.uint8)
+    xs = np.empty(T, np.float32)
+    work = np.empty(K, np.float32)
+    lib().orc_rmsnorm_smooth_quant_f8(_ptr(x), T, K, _ptr(f), float(eps), int(bool(apply_norm)), _ptr(xq), _ptr(xs),
+                                      _ptr(work))
+    return xq, xs
+
+
+def gemm_f8(xq, wq, rows=None, cols=None):
+    """Exact (binary64) sum of E4M3 products for the listed rows / columns."""
+    xq = _need(xq, np.uint8, "xq")
+    wq = _need(wq, np.uint8, "wq")
+    T, K = xq.shape
+    N = wq.shape[0]
+    ri = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    ci = None if cols is None else np.ascontiguousarray(cols, np.int64)
+    nr = T if ri is None else ri.shape[0]
+    nc = N if ci is None else ci.shape[0]
+    acc = np.empty((nr, nc), np.float64)
+    lib().orc_gemm_f8(_ptr(xq), T, _ptr(wq), N, K, _ptr(ri), nr, _ptr(ci), nc, _ptr(acc))
+    return acc
+
+
+def dequant_f32(acc, x_scale, w_scale, bias=None, rows=None, cols=None):
+    """bf16(acc * (x_scale[t] * w_scale[n]) + bias[n]) from binary32 accumulators (bf16 bits)."""
+    acc = _need(acc, np.float32, "acc")
+    xs = _need(x_scale, np.float32, "x_scale")
+    ws = _need(w_scale, np.float32, "w_scale")
+    b = None if bias is None else _need(bias, np.uint16, "bias")
+    ri = None if rows is None else np.ascontiguousarray(rows, np.int64)
+    ci = None if cols is None else np.ascontiguousarray(cols, np.int64)
+    nr, nc = acc.shape
+    y = np.empty((nr, nc), np.uint16)
+    lib().orc_dequant_f32(_ptr(acc), _ptr(xs), _ptr(ws), _ptr(b), _ptr(ri), nr, _ptr(ci), nc, _ptr(y))
+    return y
+
+
+def w8a8_linear_f8(xq, x_scale, wq, w_scale, bias=None, rows=None, cols=None):
+    """FP8 GEMM (exact accumulation) then the dequant epilogue on the accumulator rounded to binary32.
+    Returns (y bf16 bits, acc binary64)."""
+    acc = gemm_f8(xq, wq, rows, cols)
+    return dequant_f32(acc.astype(np.float32), x_scale, w_scale, bias, rows, cols), acc
 
 
 def gemm_s8(xq, wq, rows=None, cols=None):

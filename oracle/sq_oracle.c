@@ -279,6 +279,135 @@ void orc_fold_into_w_scale(const float *w_scale, int64_t K, const float *f, floa
     for (int64_t j = 0; j < K; ++j) w_scale_out[j] = w_scale[j] * f[j];
 }
 
+/* ---------------------------------------------------------------------------------------------
+ * FP8 E4M3 variant, [W8A8] "One layer, measured" (the same sweep in FP8 E4M3) and "FP8's exponent
+ * gives each value its own scale". E4M3 (the OCP "FN" form): 1 sign bit, 4 exponent bits with bias
+ * 7, 3 mantissa bits; normals (1 + m/8) * 2^(e-7) for e = 1..15 except the pattern S.1111.111
+ * (NaN), so the largest finite value is 448; subnormals (m/8) * 2^-6. Reading: scales are
+ * delta = max|v| / 448 with codes e4m3(v * fl32(448 / max|v|)), rounded to nearest (ties to even)
+ * with saturation to +-448, the FP8 counterpart of the INT8 quantiser above.
+ */
+#define ORC_F8MAX 448.0f
+
+/* Nearest E4M3 value to a (a >= 0, finite), ties to even, saturating at 448; returned as its code
+ * (exponent and mantissa bits, sign bit clear). */
+static uint8_t e4m3_code_abs(float a)
+{
+    if (a >= ORC_F8MAX) return 0x7E;                      /* 448 (anything above saturates) */
+    if (a < 0x1p-6f) {                                     /* subnormal grid, step 2^-9 */
+        float q = nearbyintf(a * 0x1p9f);                  /* exact scaling; default mode is nearest-even */
+        return (uint8_t)q;                                 /* q = 8 is the smallest normal, code 0x08 */
+    }
+    int e;
+    frexpf(a, &e);                                         /* a = f * 2^e, f in [0.5, 1) */
+    e -= 1;                                                /* a in [2^e, 2^(e+1)) */
+    float q = nearbyintf(ldexpf(a, 3 - e));                /* multiples of 2^(e-3): q in [8, 16] */
+    int ee = e + 7, m = (int)q - 8;
+    if (m == 8) { ee += 1; m = 0; }                        /* rounded up into the next binade */
+    if (ee > 15 || (ee == 15 && m > 6)) return 0x7E;       /* beyond 448 after rounding: saturate */
+    return (uint8_t)((ee << 3) | m);
+}
+
+static uint8_t e4m3_encode(float v)
+{
+    uint8_t c = e4m3_code_abs(fabsf(v));
+    return signbit(v) ? (uint8_t)(c | 0x80) : c;           /* the sign is kept, also on a zero */
+}
+
+static float e4m3_decode(uint8_t c)
+{
+    int e = (c >> 3) & 15, m = c & 7;
+    float a = e == 0 ? ldexpf((float)m, -9) : ldexpf((float)(8 + m), e - 10);
+    return (c & 0x80) ? -a : a;
+}
+
+uint8_t orc_e4m3_encode(float v) { return e4m3_encode(v); }
+float orc_e4m3_decode(uint8_t c) { return e4m3_decode(c); }
+
+/* One row of smoothed binary32 values to E4M3 with one scale: m = max|v|, delta = m / 448,
+ * codes e4m3(v * fl32(448 / m)); a zero row gives delta 0 and codes 0. */
+static void quantize_row_f8(const float *v, int64_t n, uint8_t *q, float *delta_out)
+{
+    float m = 0.0f;
+    for (int64_t k = 0; k < n; ++k) {
+        float a = fabsf(v[k]);
+        if (a > m) m = a;
+    }
+    if (m == 0.0f) {
+        for (int64_t k = 0; k < n; ++k) q[k] = 0;
+        *delta_out = 0.0f;
+        return;
+    }
+    float inv = ORC_F8MAX / m;
+    for (int64_t k = 0; k < n; ++k) q[k] = e4m3_encode(v[k] * inv);
+    *delta_out = m / ORC_F8MAX;
+}
+
+/* Smoothed weight in E4M3, one scale per output channel (the FP8 form of orc_smooth_quantize_weight). */
+void orc_smooth_quantize_weight_f8(const uint16_t *w, int64_t N, int64_t K, const float *s, uint8_t *wq,
+                                   float *w_scale, float *work)
+{
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            float v = bf16_to_f32(w[n * K + k]);
+            work[k] = s ? v * s[k] : v;
+        }
+        quantize_row_f8(work, K, wq + n * K, &w_scale[n]);
+    }
+}
+
+/* RMSNorm with the folded weight (or x * fold), then E4M3 with one dynamic scale per token. */
+void orc_rmsnorm_smooth_quant_f8(const uint16_t *x, int64_t T, int64_t K, const float *fold, float eps,
+                                 int apply_norm, uint8_t *xq, float *x_scale, float *work)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        const uint16_t *row = x + t * K;
+        float ir = apply_norm ? row_inv_rms(row, K, eps) : 1.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = bf16_to_f32(row[k]);
+            work[k] = apply_norm ? (v * ir) * fold[k] : v * fold[k];
+        }
+        quantize_row_f8(work, K, xq + t * K, &x_scale[t]);
+    }
+}
+
+/* FP8 product accumulated exactly: acc[t, n] = sum_k e4m3(xq[t,k]) * e4m3(wq[n,k]) in binary64.
+ * Each product has at most 8 significant bits and lies in [2^-18, 2^18], so for K <= 2^20 the
+ * binary64 sum is exact (the tensor cores accumulate in binary32; tests bound that difference). */
+void orc_gemm_f8(const uint8_t *xq, int64_t T, const uint8_t *wq, int64_t N, int64_t K, const int64_t *row_idx,
+                 int64_t nrows, const int64_t *col_idx, int64_t ncols, double *acc)
+{
+    if (!row_idx) nrows = T;
+    if (!col_idx) ncols = N;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t t = row_idx ? row_idx[i] : i;
+        for (int64_t c = 0; c < ncols; ++c) {
+            int64_t n = col_idx ? col_idx[c] : c;
+            double sum = 0.0;
+            for (int64_t k = 0; k < K; ++k) sum += (double)e4m3_decode(xq[t * K + k]) * (double)e4m3_decode(wq[n * K + k]);
+            acc[i * ncols + c] = sum;
+        }
+    }
+}
+
+/* Dequantisation of binary32 accumulators (the FP8 form): y = bf16(acc * (x_scale * w_scale) + bias),
+ * the same steps as orc_dequant. */
+void orc_dequant_f32(const float *acc, const float *x_scale, const float *w_scale, const uint16_t *bias,
+                     const int64_t *row_idx, int64_t nrows, const int64_t *col_idx, int64_t ncols, uint16_t *y)
+{
+    for (int64_t i = 0; i < nrows; ++i) {
+        int64_t t = row_idx ? row_idx[i] : i;
+        for (int64_t c = 0; c < ncols; ++c) {
+            int64_t n = col_idx ? col_idx[c] : c;
+            float sc = x_scale[t] * w_scale[n];
+            float v = acc[i * ncols + c] * sc;
+            if (bias) v = v + bf16_to_f32(bias[n]);
+            y[i * ncols + c] = f32_to_bf16_rne(v);
+        }
+    }
+}
+
 /*
  * INT8 x INT8 -> INT32 product of the quantised activations xq[T, K] and weights wq[N, K]
  * (both stored with K contiguous): acc[t, n] = sum_k xq[t, k] * wq[n, k].

@@ -312,6 +312,67 @@ def test_fold_into_prev_linear_rounding_and_w_scale(orc):
 
 
 # --------------------------------------------------------------------------------------------
+# FP8 E4M3 variant ("SmoothQuant and W8A8...", "One layer, measured"): torch's float8_e4m3fn type
+# is the independent check of the format (decode of every finite code, round-to-nearest-even
+# encode including exact ties and subnormals); saturation at 448 is the closed form.
+
+def _finite_e4m3_codes():
+    c = np.arange(256, dtype=np.uint8)
+    return c[(c & 0x7F) != 0x7F]
+
+
+def test_e4m3_decode_matches_torch(orc):
+    c = _finite_e4m3_codes()
+    ref = torch.from_numpy(c.copy()).view(torch.float8_e4m3fn).float().numpy()
+    assert np.array_equal(orc.e4m3_decode(c), ref)
+    assert orc.e4m3_decode(np.uint8(0x7E)) == 448.0 and orc.e4m3_decode(np.uint8(0x01)) == 2.0 ** -9
+
+
+def test_e4m3_encode_matches_torch_and_saturates(orc):
+    ref = torch.from_numpy(_finite_e4m3_codes().copy()).view(torch.float8_e4m3fn).float().numpy()
+    pos = np.sort(ref[ref > 0])
+    rng = np.random.default_rng(70)
+    vals = np.concatenate([ref, (pos[:-1] + pos[1:]) / 2, -(pos[:-1] + pos[1:]) / 2,   # every exact tie
+                           rng.uniform(-448, 448, 4000), rng.standard_normal(4000) * 2.0 ** -8]).astype(np.float32)
+    tref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(orc.e4m3_encode(vals), tref)
+    assert np.all(orc.e4m3_encode(np.array([448.5, 470.0, 1e9], np.float32)) == 0x7E)
+    assert np.all(orc.e4m3_encode(np.array([-448.5, -1e9], np.float32)) == 0xFE)
+
+
+def test_fp8_quantiser_invariants(orc):
+    x = rand_bf16((17, 256), 71, scale=3.0)
+    fold = (0.5 + np.random.default_rng(71).random(256)).astype(np.float32)
+    xq, xs = orc.rmsnorm_smooth_quant_f8(x, fold, apply_norm=True)
+    assert np.all((xq & 0x7F).max(axis=1) == 0x7E)               # the row maximum maps to +-448
+    wq, ws = orc.smooth_quantize_weight_f8(rand_bf16((9, 256), 72), fold)
+    assert np.all((wq & 0x7F).max(axis=1) == 0x7E)
+    y = bits_to_f64(x) * fold.astype(np.float64)                 # without the norm: y = x * fold
+    xq2, xs2 = orc.rmsnorm_smooth_quant_f8(x, fold, apply_norm=False)
+    t = y / xs2[:, None].astype(np.float64)                       # the value each code stands for
+    d = orc.e4m3_decode(xq2).astype(np.float64)
+    normal = np.abs(d) >= 2.0 ** -6
+    assert np.all(np.abs(d - t)[normal] <= np.abs(t)[normal] * 2.0 ** -4 * (1 + 1e-6))   # half a step of 3 bits
+    assert np.all(np.abs(d - t)[~normal] <= 2.0 ** -10 * (1 + 1e-6) + np.abs(t)[~normal] * 2.0 ** -20)
+
+
+def test_fp8_gemm_exact_and_dequant(orc):
+    rng = np.random.default_rng(73)
+    c = _finite_e4m3_codes()
+    xq = rng.choice(c, size=(11, 700)).astype(np.uint8)
+    wq = rng.choice(c, size=(13, 700)).astype(np.uint8)
+    dx = torch.from_numpy(xq).view(torch.float8_e4m3fn).double().numpy()
+    dw = torch.from_numpy(wq).view(torch.float8_e4m3fn).double().numpy()
+    acc = orc.gemm_f8(xq, wq)
+    assert np.array_equal(acc, dx @ dw.T)                       # both exact: every partial sum is representable
+    xs = (rng.random(11) * 1e-2).astype(np.float32)
+    ws = (rng.random(13) * 1e-2).astype(np.float32)
+    y, _ = orc.w8a8_linear_f8(xq, xs, wq, ws)
+    exact = acc * xs[:, None].astype(np.float64) * ws[None, :].astype(np.float64)
+    assert np.all(np.abs(bits_to_f64(y) - exact) <= np.abs(exact) * (2.0 ** -8 + 2.0 ** -22) + 1e-30)
+
+
+# --------------------------------------------------------------------------------------------
 # INT8 GEMM ("06 -- SmoothQuant...", section 7): numpy int64 matmul is the independent check.
 
 def test_gemm_matches_numpy_int64(orc):
