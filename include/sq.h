@@ -203,6 +203,32 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, cons
  */
 sq_status sq_set_gemm_cta_pair(int enable);
 
+/*
+ * FP8 E4M3 variant of the weight and activation quantisers and of the linear layer:
+ *   [W8A8] "One layer, measured" (the same layer quantised to FP8 E4M3, weights per output channel,
+ *   activations per token) and its explanation that FP8's exponent gives each value its own scale.
+ * E4M3 is the OCP "FN" form (largest finite value 448). Codes are e4m3(v * fl32(448 / m)) rounded to
+ * nearest (ties to even) with saturation at +-448, the sign kept on zeros; the scale is m / 448
+ * (m = the row maximum); an all-zero row gives scale 0 and codes +0 (0x00). Codes are stored one byte
+ * per value (uint8, the E4M3 bit pattern). Same arguments and requirements as the INT8 calls.
+ */
+sq_status sq_smooth_quantize_weight_fp8(const void *w, int64_t N, int64_t K, const float *s, uint8_t *wq,
+                                        float *w_scale, void *stream);
+sq_status sq_rmsnorm_smooth_quant_fp8(const void *x, int64_t T, int64_t K, const float *fold, float eps,
+                                      int apply_norm, uint8_t *xq, float *x_scale, void *stream);
+
+/*
+ * FP8 linear: E4M3 x E4M3 products accumulated in binary32 on the tensor cores
+ * (tcgen05.mma.kind::f8f6f4), then y[t,n] = bf16_rn(acc * (x_scale[t] * w_scale[n]) + bias[n]) in
+ * binary32 as in sq_w8a8_linear. The products are exact; the order and precision of the tensor-core
+ * accumulation are the hardware's, so acc differs from the exact sum by rounding only. acc_out
+ * nullable fp32 [T, N] (the accumulators). Same arguments and requirements as sq_w8a8_linear (the
+ * CTA-pair setting does not apply).
+ */
+sq_status sq_w8a8_linear_fp8(const uint8_t *xq, const float *x_scale, int64_t T, const uint8_t *wq,
+                             const float *w_scale, int64_t N, int64_t K, const void *bias, void *y,
+                             float *acc_out, void *workspace, size_t workspace_bytes, void *stream);
+
 /* Bytes of workspace sq_w8a8_linear needs for these sizes (0 in this build). */
 size_t sq_w8a8_linear_workspace_size(int64_t T, int64_t N, int64_t K);
 

@@ -379,13 +379,15 @@ void orc_gemm_f8(const uint8_t *xq, int64_t T, const uint8_t *wq, int64_t N, int
 {
     if (!row_idx) nrows = T;
     if (!col_idx) ncols = N;
+    double table[256];                                     /* the value of every code */
+    for (int c = 0; c < 256; ++c) table[c] = (double)e4m3_decode((uint8_t)c);
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < nrows; ++i) {
         int64_t t = row_idx ? row_idx[i] : i;
         for (int64_t c = 0; c < ncols; ++c) {
             int64_t n = col_idx ? col_idx[c] : c;
             double sum = 0.0;
-            for (int64_t k = 0; k < K; ++k) sum += (double)e4m3_decode(xq[t * K + k]) * (double)e4m3_decode(wq[n * K + k]);
+            for (int64_t k = 0; k < K; ++k) sum += table[xq[t * K + k]] * table[wq[n * K + k]];
             acc[i * ncols + c] = sum;
         }
     }

@@ -64,6 +64,16 @@ constexpr uint32_t make_idesc(int M, int N) {
     return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
            (static_cast<uint32_t>(M >> 4) << 24);
 }
+// kind::f8f6f4 with A and B E4M3 (format 0), D = f32 (format 1 at bits 4..5), both K-major.
+constexpr uint32_t make_idesc_f8(int M, int N) {
+    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+// Binary32 value of an accumulator word: the integer converted (INT8 form) or the f32 bits (FP8).
+template <bool F8>
+__device__ __forceinline__ float acc_value(uint32_t r) {
+    if (F8) return __uint_as_float(r);
+    return __int2float_rn(static_cast<int>(r));
+}
 
 // Shared-memory plan of the single-SM kernel for tiles of TN output channels. The 256-wide form
 // serves token counts that fill the SMs with tiles; the 64-wide form serves few tokens (decode),
@@ -97,6 +107,7 @@ struct Tile {
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM_TOTAL = OFF_MISC + 16 + 1024; // slack to align the base to 1024 bytes
     static constexpr uint32_t IDESC = make_idesc(BM, TN);
+    static constexpr uint32_t IDESC_F8 = make_idesc_f8(BM, TN);
     static_assert(SMEM_TOTAL <= 232448, "shared memory budget of one sm_100 CTA");
     static_assert(SWAP ? (TN >= 16 && TN <= 128 && (TN & (TN - 1)) == 0)
                        : (TN % OUT_COLS == 0 && TN >= 32 && TN <= 256 && (TN & (TN - 1)) == 0), "tile width");
@@ -151,6 +162,15 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// FP8 form: A and B both E4M3, binary32 accumulators (tcgen05.mma.kind::f8f6f4, K = 32 per instruction).
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc)
         : "memory");
 }
@@ -315,7 +335,7 @@ __device__ __forceinline__ void regs_after_wait(uint32_t *r) {
 // `xs` the x_scale of this lane's row. The TMEM read of the next 32 columns is in flight while the
 // current 32 are converted. `stage_buf` holds two boxes that alternate; `nstores` counts this warp's
 // stores.
-template <int TN>
+template <int TN, bool F8>
 __device__ __forceinline__ void epilogue_rows(uint32_t tmem_base, int quad, int lane, uint32_t tcol, int row0, int n0,
                                               float xs, const float *tab, bool has_bias, int32_t *__restrict__ acc_out,
                                               int T, int N, const CUtensorMap *tmY, uint8_t *stage_buf, int &nstores)
@@ -349,8 +369,8 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tmem_base, int quad, int 
         for (int g = 0; g < OUT_COLS / 4; ++g) {
             uint64_t w01, w23;
             lds_pairs(tab + c * OUT_COLS + 4 * g, w01, w23);
-            const uint64_t a01 = pack2(__int2float_rn(static_cast<int>(cur[4 * g])), __int2float_rn(static_cast<int>(cur[4 * g + 1])));
-            const uint64_t a23 = pack2(__int2float_rn(static_cast<int>(cur[4 * g + 2])), __int2float_rn(static_cast<int>(cur[4 * g + 3])));
+            const uint64_t a01 = pack2(acc_value<F8>(cur[4 * g]), acc_value<F8>(cur[4 * g + 1]));
+            const uint64_t a23 = pack2(acc_value<F8>(cur[4 * g + 2]), acc_value<F8>(cur[4 * g + 3]));
             uint64_t v01 = mul2_rn(a01, mul2_rn(xs2, w01));
             uint64_t v23 = mul2_rn(a23, mul2_rn(xs2, w23));
             if (has_bias) {
@@ -398,7 +418,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t *r) {
 // n = n_base + 32 quad + lane and writes y[t][n] = bf16(float(acc) * (x_scale[t] * w_scale[n]) + bias[n])
 // (each operation rounded once, the same steps as the other forms) for the tile's tokens t < T; a warp
 // writes 32 consecutive channels of a token per store. Optionally writes the raw accumulators.
-template <int TN>
+template <int TN, bool F8>
 __device__ __forceinline__ void epilogue_swap(uint32_t tmem_base, int quad, int lane, uint32_t tcol, int n_base, int t0,
                                               const float *__restrict__ x_scale, const float *__restrict__ w_scale,
                                               const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ y,
@@ -428,7 +448,7 @@ __device__ __forceinline__ void epilogue_swap(uint32_t tmem_base, int quad, int 
                 const int acc = static_cast<int>(r[j]);
                 const int64_t o = static_cast<int64_t>(t) * N + n;
                 if (acc_out != nullptr) acc_out[o] = acc;
-                float v = __fmul_rn(__int2float_rn(acc), __fmul_rn(__ldg(x_scale + t), ws));
+                float v = __fmul_rn(acc_value<F8>(r[j]), __fmul_rn(__ldg(x_scale + t), ws));
                 if (bias != nullptr) v = __fadd_rn(v, b);
                 y[o] = __float2bfloat16_rn(v);
             }
@@ -438,7 +458,7 @@ __device__ __forceinline__ void epilogue_swap(uint32_t tmem_base, int quad, int 
 
 // ------------------------------------------------------------------------------------------------
 
-template <int TN, bool SWAP>
+template <int TN, bool SWAP, bool F8>
 __global__ void __launch_bounds__(THREADS, 1)
 k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmY, const float *__restrict__ x_scale,
@@ -540,8 +560,12 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                         const uint32_t b0 = smem_u32(sB + stage * L::B_SLOT + ks * L::B_SLICE);
 #pragma unroll
                         for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-                            mma_i8(d_tmem, kmajor_sw128_desc(a0 + kk * UMMA_K), kmajor_sw128_desc(b0 + kk * UMMA_K), L::IDESC,
-                                   (kb | ks | kk) != 0 ? 1u : 0u);
+                            if (F8)
+                                mma_f8(d_tmem, kmajor_sw128_desc(a0 + kk * UMMA_K), kmajor_sw128_desc(b0 + kk * UMMA_K), L::IDESC_F8,
+                                       (kb | ks | kk) != 0 ? 1u : 0u);
+                            else
+                                mma_i8(d_tmem, kmajor_sw128_desc(a0 + kk * UMMA_K), kmajor_sw128_desc(b0 + kk * UMMA_K), L::IDESC,
+                                       (kb | ks | kk) != 0 ? 1u : 0u);
                         }
                     }
                     issued = true;
@@ -570,7 +594,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             tc_fence_after();
             int m, n;
             tile_coords(t, m_tiles, n_tiles, m, n);
-            epilogue_swap<TN>(tmem_base, quad, lane, static_cast<uint32_t>(buf * TN), m * BM, n * TN, x_scale, w_scale,
+            epilogue_swap<TN, F8>(tmem_base, quad, lane, static_cast<uint32_t>(buf * TN), m * BM, n * TN, x_scale, w_scale,
                               bias, y, acc_out, T, N);
             tc_fence_before();
             mbar_arrive(tempty(buf));
@@ -605,7 +629,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             tile_coords(t, m_tiles, n_tiles, m, n);
             const float xs_t = xs;
             prefetch(t + gridDim.x);
-            epilogue_rows<TN>(tmem_base, quad, lane, static_cast<uint32_t>(buf * TN), m * BM + quad * 32, n * TN, xs_t, tab,
+            epilogue_rows<TN, F8>(tmem_base, quad, lane, static_cast<uint32_t>(buf * TN), m * BM + quad * 32, n * TN, xs_t, tab,
                           bias != nullptr, acc_out, T, N, &tmY, stage_buf, nstores);
             tc_fence_before();
             mbar_arrive(tempty(buf));
@@ -792,7 +816,7 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             tile_coords(t, m_tiles, n_tiles, m, n);
             const float xs_t = xs;
             prefetch(t + ncl);
-            epilogue_rows<BN>(tmem_base, quad, lane, static_cast<uint32_t>(buf * BN),
+            epilogue_rows<BN, false>(tmem_base, quad, lane, static_cast<uint32_t>(buf * BN),
                           m * 2 * BM + static_cast<int>(rank) * BM + quad * 32, n * BN, xs_t, tab, bias != nullptr, acc_out,
                           T, N, &tmY, stage_buf, nstores);
             tc_fence_before();
@@ -864,14 +888,14 @@ sq_status encode_2d(EncodeTiledFn enc, CUtensorMap *map, CUtensorMapDataType dt,
 
 // Single-SM forms: one persistent CTA per SM at most. Plain: tiles of 128 tokens x TN channels (A =
 // tokens, B = weight). SWAP: tiles of 128 channels x TN tokens (A = weight, B = tokens).
-template <int TN, bool SWAP>
+template <int TN, bool SWAP, bool F8>
 sq_status launch_single(const CUtensorMap &mA, const CUtensorMap &mB, const CUtensorMap &mY, const float *x_scale,
                         const float *w_scale, const void *bias, int32_t *acc_out, void *y, int64_t T, int64_t N, int64_t K,
                         int dev, void *stream) {
     using L = Tile<TN, SWAP>;
     static int configured[64];
     if (!configured[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(k_w8a8_linear<TN, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_TOTAL);
+        cudaError_t e = cudaFuncSetAttribute(k_w8a8_linear<TN, SWAP, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_TOTAL);
         if (e != cudaSuccess) return sq::cuda_status(e, "cudaFuncSetAttribute(w8a8_linear)");
         configured[dev] = 1;
     }
@@ -881,49 +905,29 @@ sq_status launch_single(const CUtensorMap &mA, const CUtensorMap &mB, const CUte
     const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
     if (tiles > 0x7FFFFFFF) return sq::fail(SQ_ERR_UNSUPPORTED, "sq_w8a8_linear: too many tiles");
     const int grid = static_cast<int>(tiles < sq::sm_count(dev) ? tiles : sq::sm_count(dev));
-    k_w8a8_linear<TN, SWAP><<<grid, THREADS, L::SMEM_TOTAL, sq::as_stream(stream)>>>(
+    k_w8a8_linear<TN, SWAP, F8><<<grid, THREADS, L::SMEM_TOTAL, sq::as_stream(stream)>>>(
         mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out,
         static_cast<__nv_bfloat16 *>(y), static_cast<int>(T), static_cast<int>(N), static_cast<int>(K), m_tiles, n_tiles,
         sq::wait_timeout_ns(dev));
     return sq::cuda_status(cudaGetLastError(), "launch(w8a8_linear)");
 }
 
-}  // namespace
-
-namespace sq {
-
-unsigned int *device_status_word(int device) {
-    static unsigned int *addr[64];
-    if (device < 0 || device >= 64) return nullptr;
-    if (!addr[device]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_sq_status) != cudaSuccess) return nullptr;
-        addr[device] = static_cast<unsigned int *>(p);
-    }
-    return addr[device];
-}
-
-}  // namespace sq
-
-extern "C" {
-
-sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, const int8_t *wq,
-                         const float *w_scale, int64_t N, int64_t K, const void *bias, void *y,
-                         int32_t *acc_out, void *workspace, size_t workspace_bytes, void *stream)
+template <bool F8>
+sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const void *wq, const float *w_scale, int64_t N,
+                      int64_t K, const void *bias, void *y, void *acc_out_v, void *stream, const char *fn)
 {
+    int32_t *acc_out = static_cast<int32_t *>(acc_out_v);   // raw accumulator words (s32, or f32 bits)
     using sq::fail;
-    (void)workspace;
-    (void)workspace_bytes;
-    if (T < 0 || N < 8 || K < 16) return fail(SQ_ERR_INVALID_ARG, "sq_w8a8_linear: need T >= 0, N >= 8, K >= 16");
-    if (!wq || !w_scale) return fail(SQ_ERR_INVALID_ARG, "sq_w8a8_linear: wq and w_scale are required");
-    if (T > 0 && (!xq || !x_scale || !y)) return fail(SQ_ERR_INVALID_ARG, "sq_w8a8_linear: xq, x_scale and y are required");
-    if (N % 8 != 0 || K % 16 != 0) return fail(SQ_ERR_MISALIGNED, "sq_w8a8_linear: N must be a multiple of 8 and K of 16");
+    if (T < 0 || N < 8 || K < 16) return fail(SQ_ERR_INVALID_ARG, "%s: need T >= 0, N >= 8, K >= 16", fn);
+    if (!wq || !w_scale) return fail(SQ_ERR_INVALID_ARG, "%s: wq and w_scale are required", fn);
+    if (T > 0 && (!xq || !x_scale || !y)) return fail(SQ_ERR_INVALID_ARG, "%s: xq, x_scale and y are required", fn);
+    if (N % 8 != 0 || K % 16 != 0) return fail(SQ_ERR_MISALIGNED, "%s: N must be a multiple of 8 and K of 16", fn);
     if (K > 131072 || N > 0x7FFFFFFF || T > 0x7FFFFFFF)
-        return fail(SQ_ERR_UNSUPPORTED, "sq_w8a8_linear: K must be <= 131072 and T, N < 2^31");
+        return fail(SQ_ERR_UNSUPPORTED, "%s: K must be <= 131072 and T, N < 2^31", fn);
     if ((xq && !sq::aligned(xq, 16)) || !sq::aligned(wq, 16) || (y && !sq::aligned(y, 16)) ||
         (acc_out && !sq::aligned(acc_out, 16)) || !sq::aligned(w_scale, 16) || (x_scale && !sq::aligned(x_scale, 4)) ||
         (bias && !sq::aligned(bias, 8)))
-        return fail(SQ_ERR_MISALIGNED, "sq_w8a8_linear: xq, wq, y, acc_out, w_scale need 16-byte, bias 8-byte, x_scale 4-byte alignment");
+        return fail(SQ_ERR_MISALIGNED, "%s: xq, wq, y, acc_out, w_scale need 16-byte, bias 8-byte, x_scale 4-byte alignment", fn);
     int dev = 0;
     SQ_TRY_ARCH(dev);
     if (T == 0) return SQ_OK;
@@ -931,7 +935,7 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, cons
     EncodeTiledFn enc = nullptr;
     sq_status st = get_encoder(&enc);
     if (st != SQ_OK) return st;
-    const bool pair = g_cta_pair.load(std::memory_order_relaxed) != 0 && T >= 2 * BM;   // 256-row tiles on CTA pairs
+    const bool pair = !F8 && g_cta_pair.load(std::memory_order_relaxed) != 0 && T >= 2 * BM;   // 256-row tiles on CTA pairs
     // 64-channel tiles when 256-channel tiles would leave SMs idle (few tokens: the weight stream
     // then bounds the call, and more tiles spread it over more SMs)
     const int64_t wide_tiles = ((T + BM - 1) / BM) * ((N + BN - 1) / BN);
@@ -945,10 +949,10 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, cons
         if (st == SQ_OK) st = encode_2d(enc, &mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, T, K, BK, tn, CU_TENSOR_MAP_SWIZZLE_128B, "xq");
         if (st != SQ_OK) return st;
         switch (tn) {
-            case 16: return launch_single<16, true>(mA, mB, mA, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
-            case 32: return launch_single<32, true>(mA, mB, mA, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
-            case 64: return launch_single<64, true>(mA, mB, mA, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
-            default: return launch_single<128, true>(mA, mB, mA, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+            case 16: return launch_single<16, true, F8>(mA, mB, mA, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+            case 32: return launch_single<32, true, F8>(mA, mB, mA, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+            case 64: return launch_single<64, true, F8>(mA, mB, mA, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+            default: return launch_single<128, true, F8>(mA, mB, mA, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
         }
     }
     st = encode_2d(enc, &mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, T, K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B, "xq");
@@ -982,7 +986,7 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, cons
         const int m_tiles = static_cast<int>((T + 2 * BM - 1) / (2 * BM));
         const int n_tiles = static_cast<int>((N + BN - 1) / BN);
         const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
-        if (tiles > 0x7FFFFFFF) return fail(SQ_ERR_UNSUPPORTED, "sq_w8a8_linear: too many tiles");
+        if (tiles > 0x7FFFFFFF) return fail(SQ_ERR_UNSUPPORTED, "%s: too many tiles", fn);
         const int clusters = static_cast<int>(tiles < pclusters[dev] ? tiles : pclusters[dev]);
         cfg.gridDim = dim3(2 * clusters, 1, 1);
         return sq::cuda_status(
@@ -992,8 +996,46 @@ sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, cons
             "launch(w8a8_linear_pair)");
     }
 
-    return narrow ? launch_single<64, false>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream)
-                  : launch_single<BN, false>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+    return narrow ? launch_single<64, false, F8>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream)
+                  : launch_single<BN, false, F8>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+}
+
+
+}  // namespace
+
+namespace sq {
+
+unsigned int *device_status_word(int device) {
+    static unsigned int *addr[64];
+    if (device < 0 || device >= 64) return nullptr;
+    if (!addr[device]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_sq_status) != cudaSuccess) return nullptr;
+        addr[device] = static_cast<unsigned int *>(p);
+    }
+    return addr[device];
+}
+
+}  // namespace sq
+
+extern "C" {
+
+sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, const int8_t *wq,
+                         const float *w_scale, int64_t N, int64_t K, const void *bias, void *y,
+                         int32_t *acc_out, void *workspace, size_t workspace_bytes, void *stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    return linear_impl<false>(xq, x_scale, T, wq, w_scale, N, K, bias, y, acc_out, stream, "sq_w8a8_linear");
+}
+
+sq_status sq_w8a8_linear_fp8(const uint8_t *xq, const float *x_scale, int64_t T, const uint8_t *wq,
+                             const float *w_scale, int64_t N, int64_t K, const void *bias, void *y,
+                             float *acc_out, void *workspace, size_t workspace_bytes, void *stream)
+{
+    (void)workspace;
+    (void)workspace_bytes;
+    return linear_impl<true>(xq, x_scale, T, wq, w_scale, N, K, bias, y, acc_out, stream, "sq_w8a8_linear_fp8");
 }
 
 sq_status sq_set_gemm_cta_pair(int enable) {

@@ -68,7 +68,9 @@ constexpr uint32_t kSqBias = 485u << 20;   // binary64 exponent bias mapping bf1
 constexpr unsigned kAll = 0xFFFFFFFFu;
 
 // MODE_QSTATIC: the quantiser with one static per-tensor scale (no row maximum; codes clamped).
-enum { MODE_ABSMAX = 0, MODE_QUANT = 1, MODE_QSTATIC = 2 };
+// MODE_QF8: the per-row quantiser with FP8 E4M3 codes (scale max/448).
+enum { MODE_ABSMAX = 0, MODE_QUANT = 1, MODE_QSTATIC = 2, MODE_QF8 = 3 };
+constexpr float kF8Max = 448.0f;  // largest finite E4M3 value
 
 struct RowArgs {
     const uint8_t *src;     // row r starts at src + r * ld_bytes (16-byte aligned)
@@ -186,6 +188,16 @@ __device__ __forceinline__ uint32_t codes2(uint64_t t) {
     const int ql = __float2int_rz(__uint_as_float(vl));
     const int qh = __float2int_rz(__uint_as_float(vh));
     return __byte_perm(static_cast<uint32_t>(ql), static_cast<uint32_t>(qh), 0x0040);   // bytes: ql, qh in 0, 1
+}
+
+// E4M3 codes of the two values of t (round to nearest, ties to even, saturating at +-448, the sign
+// kept on a zero): the low element's code in the low byte.
+__device__ __forceinline__ uint32_t f8codes2(uint64_t t) {
+    uint32_t tl, th;
+    unpack2(t, tl, th);
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(__uint_as_float(th)), "f"(__uint_as_float(tl)));
+    return d;
 }
 
 // codes2 for values that may lie beyond the calibrated range (static scale): t is clamped to
@@ -481,8 +493,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                     for (int w = 0; w < WPR; ++w) mrow = fmaxf(mrow, s_mx[j & 1][group * WPR + w][lane / SUB]);
                 }
                 // step and reciprocal of the row this lane holds; one lane per row stores the step
-                const float delta = mrow > 0.0f ? __fdiv_rn(mrow, kQmax) : 0.0f;
-                const float inv_m = mrow > 0.0f ? __fdiv_rn(kQmax, mrow) : 0.0f;
+                constexpr float qmax = MODE == MODE_QF8 ? kF8Max : kQmax;
+                const float delta = mrow > 0.0f ? __fdiv_rn(mrow, qmax) : 0.0f;
+                const float inv_m = mrow > 0.0f ? __fdiv_rn(qmax, mrow) : 0.0f;
                 if (wig == 0 && (lane % SUB) == 0 && lane / SUB < nr) p.scale[r0 + lane / SUB] = delta;
                 // ---- pass C: codes
 #pragma unroll
@@ -495,9 +508,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                         for (int i = 0; i < VPL; ++i) {
                             const int v = i * GT + gtid;
                             if (FULL || v < nvec) {
-                                const uint32_t c01 = codes2(mul2_rn(y[r][i][0], inv2)), c23 = codes2(mul2_rn(y[r][i][1], inv2));
-                                const uint32_t c45 = codes2(mul2_rn(y[r][i][2], inv2)), c67 = codes2(mul2_rn(y[r][i][3], inv2));
-                                qrow[v] = make_uint2(__byte_perm(c01, c23, 0x5410), __byte_perm(c45, c67, 0x5410));
+                                uint32_t c01, c23, c45, c67;
+                                if (MODE == MODE_QF8) {
+                                    c01 = f8codes2(mul2_rn(y[r][i][0], inv2)); c23 = f8codes2(mul2_rn(y[r][i][1], inv2));
+                                    c45 = f8codes2(mul2_rn(y[r][i][2], inv2)); c67 = f8codes2(mul2_rn(y[r][i][3], inv2));
+                                } else {
+                                    c01 = codes2(mul2_rn(y[r][i][0], inv2)); c23 = codes2(mul2_rn(y[r][i][1], inv2));
+                                    c45 = codes2(mul2_rn(y[r][i][2], inv2)); c67 = codes2(mul2_rn(y[r][i][3], inv2));
+                                }
+                                uint2 out = make_uint2(__byte_perm(c01, c23, 0x5410), __byte_perm(c45, c67, 0x5410));
+                                if (MODE == MODE_QF8 && iv == 0.0f) out = make_uint2(0u, 0u);   // a zero row: codes +0
+                                qrow[v] = out;
                             }
                         }
                     }
@@ -844,6 +865,59 @@ sq_status sq_rmsnorm_smooth_quant(const void *x, int64_t T, int64_t K, const flo
     ra.scale = x_scale;
     cudaStream_t st = sq::as_stream(stream);
     return apply_norm ? dispatch_rows<MODE_QUANT, true>(ra, dev, st) : dispatch_rows<MODE_QUANT, false>(ra, dev, st);
+}
+
+sq_status sq_smooth_quantize_weight_fp8(const void *w, int64_t N, int64_t K, const float *s, uint8_t *wq,
+                                        float *w_scale, void *stream)
+{
+    using sq::fail;
+    if (N < 0 || K < 8) return fail(SQ_ERR_INVALID_ARG, "sq_smooth_quantize_weight_fp8: need N >= 0 and K >= 8");
+    if (N > 0 && (!w || !wq || !w_scale)) return fail(SQ_ERR_INVALID_ARG, "sq_smooth_quantize_weight_fp8: w, wq and w_scale are required");
+    if (K % 8 != 0) return fail(SQ_ERR_MISALIGNED, "sq_smooth_quantize_weight_fp8: K must be a multiple of 8");
+    if (K > kMaxK) return fail(SQ_ERR_UNSUPPORTED, "sq_smooth_quantize_weight_fp8: K must be <= %d", kMaxK);
+    if ((w && !sq::aligned(w, 16)) || (wq && !sq::aligned(wq, 8)) || (s && !sq::aligned(s, 16)) ||
+        (w_scale && !sq::aligned(w_scale, 4)))
+        return fail(SQ_ERR_MISALIGNED, "sq_smooth_quantize_weight_fp8: w and s 16-byte, wq 8-byte, w_scale 4-byte alignment required");
+    int dev = 0;
+    SQ_TRY_ARCH(dev);
+    if (N == 0) return SQ_OK;
+    RowArgs ra = {};
+    ra.src = static_cast<const uint8_t *>(w);
+    ra.rows = N;
+    ra.ld_bytes = K * 2;
+    ra.K = static_cast<int>(K);
+    ra.vec = s;
+    ra.q = reinterpret_cast<int8_t *>(wq);
+    ra.scale = w_scale;
+    return dispatch_rows<MODE_QF8, false>(ra, dev, sq::as_stream(stream));
+}
+
+sq_status sq_rmsnorm_smooth_quant_fp8(const void *x, int64_t T, int64_t K, const float *fold, float eps,
+                                      int apply_norm, uint8_t *xq, float *x_scale, void *stream)
+{
+    using sq::fail;
+    if (T < 0 || K < 8) return fail(SQ_ERR_INVALID_ARG, "sq_rmsnorm_smooth_quant_fp8: need T >= 0 and K >= 8");
+    if (!fold) return fail(SQ_ERR_INVALID_ARG, "sq_rmsnorm_smooth_quant_fp8: fold is required");
+    if (T > 0 && (!x || !xq || !x_scale)) return fail(SQ_ERR_INVALID_ARG, "sq_rmsnorm_smooth_quant_fp8: x, xq and x_scale are required");
+    if (K % 8 != 0) return fail(SQ_ERR_MISALIGNED, "sq_rmsnorm_smooth_quant_fp8: K must be a multiple of 8");
+    if (K > kMaxK) return fail(SQ_ERR_UNSUPPORTED, "sq_rmsnorm_smooth_quant_fp8: K must be <= %d", kMaxK);
+    if ((x && !sq::aligned(x, 16)) || (xq && !sq::aligned(xq, 8)) || !sq::aligned(fold, 16) ||
+        (x_scale && !sq::aligned(x_scale, 4)))
+        return fail(SQ_ERR_MISALIGNED, "sq_rmsnorm_smooth_quant_fp8: x and fold 16-byte, xq 8-byte, x_scale 4-byte alignment required");
+    int dev = 0;
+    SQ_TRY_ARCH(dev);
+    if (T == 0) return SQ_OK;
+    RowArgs ra = {};
+    ra.src = static_cast<const uint8_t *>(x);
+    ra.rows = T;
+    ra.ld_bytes = K * 2;
+    ra.K = static_cast<int>(K);
+    ra.vec = fold;
+    ra.eps = eps;
+    ra.q = reinterpret_cast<int8_t *>(xq);
+    ra.scale = x_scale;
+    cudaStream_t st = sq::as_stream(stream);
+    return apply_norm ? dispatch_rows<MODE_QF8, true>(ra, dev, st) : dispatch_rows<MODE_QF8, false>(ra, dev, st);
 }
 
 sq_status sq_static_scale(const float *amax, const float *factor, int64_t K, float *scale2, void *stream)

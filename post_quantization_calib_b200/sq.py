@@ -17,7 +17,8 @@ __all__ = [
     "SQError", "lib", "sq_calibrate_absmax", "sq_compute_scales", "sq_smooth_quantize_weight",
     "sq_rmsnorm_smooth_quant", "sq_w8a8_linear", "sq_w8a8_linear_workspace_size", "sq_device_status",
     "sq_set_wait_timeout_ns", "sq_selftest_wait_timeout", "sq_set_gemm_cta_pair",
-    "sq_static_scale", "sq_rmsnorm_smooth_quant_static", "sq_fold_into_prev_linear", "sq_fold_into_w_scale", "sq_status_string", "sq_last_error",
+    "sq_static_scale", "sq_rmsnorm_smooth_quant_static", "sq_fold_into_prev_linear", "sq_fold_into_w_scale",
+    "sq_smooth_quantize_weight_fp8", "sq_rmsnorm_smooth_quant_fp8", "sq_w8a8_linear_fp8", "sq_status_string", "sq_last_error",
     "sq_version", "LIB_PATH", "EXPORTS",
 ]
 
@@ -49,6 +50,9 @@ EXPORTS = {
     "sq_rmsnorm_smooth_quant_static": (_i, [_p, _i64, _i64, _p, _f, _i, _p, _p, _p, _p]),
     "sq_fold_into_prev_linear": (_i, [_p, _p, _i64, _i64, _p, _p, _p, _p]),
     "sq_fold_into_w_scale": (_i, [_p, _i64, _p, _p, _p]),
+    "sq_smooth_quantize_weight_fp8": (_i, [_p, _i64, _i64, _p, _p, _p, _p]),
+    "sq_rmsnorm_smooth_quant_fp8": (_i, [_p, _i64, _i64, _p, _f, _i, _p, _p, _p]),
+    "sq_w8a8_linear_fp8": (_i, [_p, _p, _i64, _p, _p, _i64, _i64, _p, _p, _p, _p, ctypes.c_size_t, _p]),
 }
 
 
@@ -240,6 +244,56 @@ def sq_fold_into_w_scale(w_scale: torch.Tensor, fold: torch.Tensor, out: Optiona
     _check(_lib.sq_fold_into_w_scale(_ptr(w_scale), w_scale.shape[0], _ptr(fold), _ptr(out), _stream(stream)),
            "sq_fold_into_w_scale")
     return out
+
+
+def sq_smooth_quantize_weight_fp8(w: torch.Tensor, s: Optional[torch.Tensor] = None, wq: Optional[torch.Tensor] = None,
+                                  w_scale: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """diag(s)*W quantised to FP8 E4M3 (uint8 codes) per output channel; see sq.h."""
+    _dev(w, "w", torch.bfloat16)
+    N, K = w.shape
+    if s is not None:
+        _dev(s, "s", torch.float32)
+    wq = torch.empty(N, K, dtype=torch.uint8, device=w.device) if wq is None else _dev(wq, "wq", torch.uint8)
+    w_scale = torch.empty(N, dtype=torch.float32, device=w.device) if w_scale is None else _dev(w_scale, "w_scale", torch.float32)
+    _check(_lib.sq_smooth_quantize_weight_fp8(_ptr(w), N, K, _ptr(s), _ptr(wq), _ptr(w_scale), _stream(stream)),
+           "sq_smooth_quantize_weight_fp8")
+    return wq, w_scale
+
+
+def sq_rmsnorm_smooth_quant_fp8(x: torch.Tensor, fold: torch.Tensor, eps: float = 1e-6, apply_norm: bool = True,
+                                xq: Optional[torch.Tensor] = None, x_scale: Optional[torch.Tensor] = None,
+                                stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Fused RMSNorm (folded 1/s) + per-token FP8 E4M3 (uint8 codes); see sq.h."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(fold, "fold", torch.float32)
+    T, K = x.shape
+    xq = torch.empty(T, K, dtype=torch.uint8, device=x.device) if xq is None else _dev(xq, "xq", torch.uint8)
+    x_scale = torch.empty(T, dtype=torch.float32, device=x.device) if x_scale is None else _dev(x_scale, "x_scale", torch.float32)
+    _check(_lib.sq_rmsnorm_smooth_quant_fp8(_ptr(x), T, K, _ptr(fold), float(eps), int(bool(apply_norm)), _ptr(xq),
+                                            _ptr(x_scale), _stream(stream)), "sq_rmsnorm_smooth_quant_fp8")
+    return xq, x_scale
+
+
+def sq_w8a8_linear_fp8(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
+                       bias: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                       acc_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """FP8 E4M3 GEMM (binary32 accumulation) with the dequant epilogue -> bf16 [T, N]; see sq.h."""
+    _dev(xq, "xq", torch.uint8)
+    _dev(x_scale, "x_scale", torch.float32)
+    _dev(wq, "wq", torch.uint8)
+    _dev(w_scale, "w_scale", torch.float32)
+    T, K = xq.shape
+    N, K2 = wq.shape
+    if K2 != K:
+        raise ValueError(f"inner sizes differ: xq has K={K}, wq has K={K2}")
+    if bias is not None:
+        _dev(bias, "bias", torch.bfloat16)
+    y = torch.empty(T, N, dtype=torch.bfloat16, device=xq.device) if y is None else _dev(y, "y", torch.bfloat16)
+    if acc_out is not None:
+        _dev(acc_out, "acc_out", torch.float32)
+    _check(_lib.sq_w8a8_linear_fp8(_ptr(xq), _ptr(x_scale), T, _ptr(wq), _ptr(w_scale), N, K, _ptr(bias), _ptr(y),
+                                   _ptr(acc_out), None, 0, _stream(stream)), "sq_w8a8_linear_fp8")
+    return y
 
 
 def sq_w8a8_linear(xq: torch.Tensor, x_scale: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,

@@ -116,6 +116,17 @@ def test_fold_argument_checks(sqmod):
     assert L.sq_fold_into_w_scale(FAKE + 2, 8, FAKE, FAKE, None) == SQ_ERR_MISALIGNED
 
 
+def test_fp8_argument_checks(sqmod):
+    L = sqmod.lib()
+    assert L.sq_smooth_quantize_weight_fp8(FAKE, 4, 12, None, FAKE, FAKE, None) == SQ_ERR_MISALIGNED
+    assert L.sq_smooth_quantize_weight_fp8(FAKE, 4, 32768, None, FAKE, FAKE, None) == SQ_ERR_UNSUPPORTED
+    assert L.sq_rmsnorm_smooth_quant_fp8(FAKE, 4, 64, None, 1e-6, 1, FAKE, FAKE, None) == SQ_ERR_INVALID_ARG
+    g = L.sq_w8a8_linear_fp8
+    assert g(FAKE, FAKE, 4, FAKE, FAKE, 4, 64, None, FAKE, None, None, 0, None) == SQ_ERR_INVALID_ARG   # N < 8
+    assert g(FAKE, FAKE, 4, FAKE, FAKE, 12, 64, None, FAKE, None, None, 0, None) == SQ_ERR_MISALIGNED   # N % 8
+    assert g(FAKE, FAKE, 4, None, FAKE, 16, 64, None, FAKE, None, None, 0, None) == SQ_ERR_INVALID_ARG  # no wq
+
+
 def test_quant_argument_checks(sqmod):
     L = sqmod.lib()
     assert L.sq_smooth_quantize_weight(FAKE, 4, 12, None, FAKE, FAKE, None) == SQ_ERR_MISALIGNED

@@ -351,6 +351,49 @@ def test_fold_into_prev_linear(sq, orc, K, Kp, bias):
     ok_status(sq)
 
 
+# FP8 E4M3 variant: codes and scales bit-exact against the oracle; the binary32 tensor-core
+# accumulators within the bound of binary32 summation (K * 2^-24 * sum |products|, K the terms) of
+# the exact sum; the epilogue bit-exact given those accumulators; the bf16 outputs within the
+# 1e-2 bar of the exact dequantised product. Shapes reach every GEMM form (decode, 64- and
+# 256-channel tiles) with ragged T, N and K.
+FP8_SHAPES = [(1, 264, 144, True, True), (33, 1000, 2064, False, False), (100, 520, 1040, True, True),
+              (300, 520, 272, False, True), (2000, 2312, 1040, True, False)]
+
+
+@pytest.mark.parametrize("T,N,K,norm,bias", FP8_SHAPES)
+def test_fp8_path(sq, orc, T, N, K, norm, bias):
+    dev = "cuda"
+    seed = 3 * T + N + K
+    ch = synth.outlier_channels(K, synth.OutlierSpec(max(1, K // 64), 10.0, 100.0), seed)
+    X = synth.outlier_tokens(T, K, ch, seed + 1, dev)
+    X[T // 2].zero_()
+    W = synth.normal_weight(N, K, seed + 2, dev)
+    gamma = synth.norm_gamma(K, seed + 3, dev) if norm else None
+    b = synth.bias_vector(N, seed + 4, dev) if bias else None
+    s, fold = sq.sq_compute_scales(sq.sq_calibrate_absmax(X, norm_gamma=gamma), sq.sq_calibrate_absmax(W), 0.5, gamma=gamma)
+    wq, ws = sq.sq_smooth_quantize_weight_fp8(W, s)
+    wq_o, ws_o = orc.smooth_quantize_weight_f8(h16(W), hnp(s))
+    assert np.array_equal(hnp(ws), ws_o) and np.array_equal(hnp(wq), wq_o), "fp8 weight codes differ"
+    xq, xs = sq.sq_rmsnorm_smooth_quant_fp8(X, fold, apply_norm=norm)
+    xq_o, xs_o = orc.rmsnorm_smooth_quant_f8(h16(X), hnp(fold), apply_norm=norm)
+    assert np.array_equal(hnp(xs), xs_o), "fp8 token scales differ"
+    assert np.array_equal(hnp(xq), xq_o), f"{int((hnp(xq) != xq_o).sum())} fp8 token codes differ"
+    assert hnp(xs)[T // 2] == 0 and not hnp(xq)[T // 2].any()
+    acc = torch.empty(T, N, dtype=torch.float32, device=dev)
+    y = sq.sq_w8a8_linear_fp8(xq, xs, wq, ws, bias=b, acc_out=acc)
+    ok_status(sq)
+    exact = orc.gemm_f8(hnp(xq), hnp(wq))
+    table = orc.e4m3_decode(np.arange(256, dtype=np.uint8)).astype(np.float64)
+    mag = np.abs(table[hnp(xq)]) @ np.abs(table[hnp(wq)]).T            # sum of |products|, exact
+    acc_h = hnp(acc).astype(np.float64)
+    assert np.all(np.abs(acc_h - exact) <= K * 2.0 ** -24 * mag + 1e-30), "fp8 accumulators beyond binary32 summation error"
+    b_h = h16(b) if bias else None
+    assert np.array_equal(h16(y), orc.dequant_f32(hnp(acc), hnp(xs), hnp(ws), b_h)), "fp8 epilogue differs"
+    ref = exact * hnp(xs)[:, None].astype(np.float64) * hnp(ws)[None, :] + (f64(b_h)[None, :] if bias else 0.0)
+    scale_mag = mag * hnp(xs)[:, None].astype(np.float64) * hnp(ws)[None, :]
+    assert np.all(np.abs(f64(h16(y)) - ref) <= 1e-2 * np.abs(ref) + 1e-2 * 2.0 ** -8 * (scale_mag + (np.abs(f64(b_h))[None, :] if bias else 0)) + 1e-30)
+
+
 def test_deterministic_bytes(sq):
     w = synth.WORKLOADS[1]
     d = synth.group_inputs(w, 0, "cuda", T=1000)
