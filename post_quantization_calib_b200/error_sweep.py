@@ -3,13 +3,15 @@
 "SmoothQuant and W8A8: Quantizing Activations Too", "One layer, measured": the migration strength
 alpha is swept from 0.1 to 1, plus a point without smoothing, with weights quantised per output
 channel and activations either with one static scale per tensor (from the calibration maximum) or
-one dynamic scale per token; the error is measured on the layer's output for held-out tokens as
+one dynamic scale per token, in INT8 and in FP8 E4M3; the error is measured on the layer's output
+for held-out tokens as
 ||X W - Q(X) Q(W)|| / ||X W|| (Frobenius norms).
 
 Every quantisation step runs through the library (``sq``): calibration abs-maxima, smoothing factors
 and fold, the smoothed INT8 weight, the activation quantiser (per token, or the static per-tensor
 scale with its clipping quantiser) and the INT8 GEMM, whose exact INT32 accumulators give
-Q(X) Q(W) = acc * x_scale[t] * w_scale[n] in binary64. The reference X W is the layer's input (the
+Q(X) Q(W) = acc * x_scale[t] * w_scale[n] in binary64; the FP8 points use the E4M3 quantisers and the
+FP8 GEMM (binary32 accumulators). The reference X W is the layer's input (the
 RMSNorm output times gamma for a norm-fed layer, else x) times the weight, in binary64. The error of
 the bf16 output the layer actually returns is reported beside it.
 
@@ -45,8 +47,8 @@ def relative_error(ref: torch.Tensor, out: torch.Tensor) -> float:
 def sweep(workload: str = "qproj_t8192_k4096_n4096", holdout: int = 2048, alphas: Sequence[float] = ALPHAS,
           device: str = "cuda") -> List[Dict]:
     """One row per (smoothing point, activation scheme): alpha (None = unsmoothed), scheme
-    ("per_token" | "per_tensor"), error (from the exact accumulators) and error_bf16 (the bf16
-    output)."""
+    ("per_token" | "per_tensor" INT8, "fp8_per_token" E4M3), error (from the accumulators: exact for
+    INT8, binary32 for FP8) and error_bf16 (the bf16 output)."""
     from . import sq
 
     w = synth.workload(workload)
@@ -65,6 +67,7 @@ def sweep(workload: str = "qproj_t8192_k4096_n4096", holdout: int = 2048, alphas
     aw = sq.sq_calibrate_absmax(W)
 
     acc = torch.empty(T, N, dtype=torch.int32, device=device)
+    accf = torch.empty(T, N, dtype=torch.float32, device=device)
     rows: List[Dict] = []
     points: List[Optional[float]] = [None] + [float(a) for a in alphas]
     for a in points:
@@ -74,7 +77,15 @@ def sweep(workload: str = "qproj_t8192_k4096_n4096", holdout: int = 2048, alphas
         else:
             s, fold = sq.sq_compute_scales(amax, aw, a, gamma=gamma)
         wq, ws = sq.sq_smooth_quantize_weight(W, s)
-        for scheme in ("per_token", "per_tensor"):
+        wq8, ws8 = sq.sq_smooth_quantize_weight_fp8(W, s)
+        for scheme in ("per_token", "per_tensor", "fp8_per_token"):
+            if scheme == "fp8_per_token":
+                xq8, xs8 = sq.sq_rmsnorm_smooth_quant_fp8(X, fold, eps=w.eps, apply_norm=w.norm)
+                y = sq.sq_w8a8_linear_fp8(xq8, xs8, wq8, ws8, acc_out=accf)
+                qq = accf.to(torch.float64) * xs8.to(torch.float64)[:, None] * ws8.to(torch.float64)[None, :]
+                rows.append({"workload": workload, "alpha": a, "scheme": scheme, "tokens": T,
+                             "error": relative_error(ref, qq), "error_bf16": relative_error(ref, y)})
+                continue
             if scheme == "per_token":
                 xq, xs = sq.sq_rmsnorm_smooth_quant(X, fold, eps=w.eps, apply_norm=w.norm)
             else:
@@ -98,7 +109,7 @@ def sweep(workload: str = "qproj_t8192_k4096_n4096", holdout: int = 2048, alphas
 def summary(rows: List[Dict]) -> Dict:
     """Unsmoothed vs best smoothed error per scheme, and the alpha that gives it."""
     out = {}
-    for scheme in ("per_token", "per_tensor"):
+    for scheme in ("per_token", "per_tensor", "fp8_per_token"):
         r = [x for x in rows if x["scheme"] == scheme]
         base = next(x for x in r if x["alpha"] is None)
         best = min((x for x in r if x["alpha"] is not None), key=lambda x: x["error"])

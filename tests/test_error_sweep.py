@@ -1,9 +1,10 @@
 """The layer-error harness ("SmoothQuant and W8A8...", "One layer, measured").
 
 CPU: the reference output and the error metric against closed forms. GPU: the sweep on the single
-linear workload reproduces the qualitative findings the page reports (smoothing lowers both errors on
-outlier data; a static per-tensor scale is worse than per-token scales without smoothing), and its
-quantised product agrees with the bf16 output the layer returns.
+linear workload reproduces the qualitative findings the page reports (smoothing lowers both INT8
+errors on outlier data; a static per-tensor scale is worse than per-token scales without smoothing;
+FP8 E4M3 barely needs smoothing, and smoothed INT8 beats it), and its quantised product agrees with
+the bf16 output the layer returns.
 """
 import numpy as np
 import pytest
@@ -46,3 +47,6 @@ def test_sweep_single_linear_findings():
     assert get[(None, "per_tensor")]["error"] > get[(None, "per_token")]["error"]
     s = error_sweep.summary(rows)
     assert s["per_tensor"]["reduction"] > 1.5 and s["per_token"]["reduction"] > 1.2
+    # FP8: smoothing changes little, and smoothed INT8 per token beats the best FP8 point
+    assert s["fp8_per_token"]["reduction"] < 1.3
+    assert s["per_token"]["best"] < s["fp8_per_token"]["best"]
