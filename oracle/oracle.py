@@ -17,7 +17,7 @@ __all__ = [
     "calibrate_absmax", "compute_scales", "smooth_quantize_weight", "rmsnorm_smooth_quant",
     "static_scale", "rmsnorm_smooth_quant_static", "fold_into_prev_linear", "fold_into_w_scale",
     "e4m3_encode", "e4m3_decode", "smooth_quantize_weight_f8", "rmsnorm_smooth_quant_f8", "gemm_f8", "dequant_f32",
-    "w8a8_linear_f8",
+    "w8a8_linear_f8", "calibrate_absmax_layernorm", "fold_layernorm_bias", "layernorm_smooth_quant",
     "gemm_s8", "dequant", "w8a8_linear", "f32_to_bf16", "bf16_to_f32", "set_threads", "lib",
 ]
 
@@ -51,6 +51,9 @@ def lib() -> ctypes.CDLL:
             L.orc_rmsnorm_smooth_quant_f8.argtypes = [_p, _i64, _i64, _p, ctypes.c_float, ctypes.c_int, _p, _p, _p]
             L.orc_gemm_f8.argtypes = [_p, _i64, _p, _i64, _i64, _p, _i64, _p, _i64, _p]
             L.orc_dequant_f32.argtypes = [_p, _p, _p, _p, _p, _i64, _p, _i64, _p]
+            L.orc_calibrate_absmax_layernorm.argtypes = [_p, _i64, _i64, _i64, _p, _p, ctypes.c_float, _p, ctypes.c_int, _p]
+            L.orc_fold_layernorm_bias.argtypes = [_p, _p, _i64, _p]
+            L.orc_layernorm_smooth_quant.argtypes = [_p, _i64, _i64, _p, _p, ctypes.c_float, _p, _p, _p]
             L.orc_gemm_s8.argtypes = [_p, _i64, _p, _i64, _i64, _p, _i64, _p, _i64, _p]
             L.orc_dequant.argtypes = [_p, _p, _p, _p, _p, _i64, _p, _i64, _p]
             L.orc_f32_to_bf16.argtypes = [ctypes.c_float]
@@ -254,6 +257,42 @@ def w8a8_linear_f8(xq, x_scale, wq, w_scale, bias=None, rows=None, cols=None):
     Returns (y bf16 bits, acc binary64)."""
     acc = gemm_f8(xq, wq, rows, cols)
     return dequant_f32(acc.astype(np.float32), x_scale, w_scale, bias, rows, cols), acc
+
+
+def calibrate_absmax_layernorm(a, gamma, beta, eps=1e-5, amax=None, accumulate=False):
+    """Per-column abs-max of LayerNorm(a) * gamma + beta ([WOVS] "Integration with Transformers"). Returns amax (float32 [cols])."""
+    a = _need(a, np.uint16, "a")
+    rows, cols = a.shape
+    if amax is None:
+        amax = np.zeros(cols, np.float32)
+    g = _need(np.asarray(gamma), np.float32, "gamma")
+    b = _need(np.asarray(beta), np.float32, "beta")
+    work = np.empty(cols, np.float32)
+    lib().orc_calibrate_absmax_layernorm(_ptr(a), rows, cols, cols, _ptr(g), _ptr(b), float(eps), _ptr(amax),
+                                         int(bool(accumulate)), _ptr(work))
+    return amax
+
+
+def fold_layernorm_bias(beta, s):
+    """beta / s (binary32): the LayerNorm bias with S^-1 folded in ([WOVS] "Integration with Transformers")."""
+    b = _need(np.asarray(beta), np.float32, "beta")
+    sv = _need(np.asarray(s), np.float32, "s")
+    out = np.empty_like(b)
+    lib().orc_fold_layernorm_bias(_ptr(b), _ptr(sv), b.shape[0], _ptr(out))
+    return out
+
+
+def layernorm_smooth_quant(x, fold, beta_fold, eps=1e-5):
+    """LayerNorm with the folded scale and bias, then per-token INT8. Returns (xq, x_scale)."""
+    x = _need(x, np.uint16, "x")
+    T, K = x.shape
+    f = _need(fold, np.float32, "fold")
+    bf = _need(beta_fold, np.float32, "beta_fold")
+    xq = np.empty((T, K), np.int8)
+    xs = np.empty(T, np.float32)
+    work = np.empty(2 * K, np.float32)
+    lib().orc_layernorm_smooth_quant(_ptr(x), T, K, _ptr(f), _ptr(bf), float(eps), _ptr(xq), _ptr(xs), _ptr(work))
+    return xq, xs
 
 
 def gemm_s8(xq, wq, rows=None, cols=None):

@@ -280,6 +280,66 @@ void orc_fold_into_w_scale(const float *w_scale, int64_t K, const float *f, floa
 }
 
 /* ---------------------------------------------------------------------------------------------
+ * LayerNorm-fed layers, [WOVS] "Integration with Transformers" (the run-time division by S costs
+ * nothing: S^-1 is folded into the scale gamma and the bias beta of the preceding LayerNorm, so
+ * activations leave the norm already smoothed). LayerNorm is not printed on the pages; the standard form is used:
+ *   mu = (sum_k x_k) / K in binary64, m = fl32(mu);  c_k = fl32(x_k - m);
+ *   var = (sum_k c_k^2) / K in binary64 (each square exact), ms = fl32(var);
+ *   r = fl32(sqrt(fl32(ms + eps))), ir = fl32(1 / r);
+ *   y_k = fl32(fl32(fl32(c_k * ir) * g_k) + b_k)
+ * with g = gamma, b = beta for calibration, and g = fold = fl32(gamma / s), b = fl32(beta / s) online.
+ */
+static float row_layernorm(const uint16_t *x, int64_t K, float eps, float *c)
+{
+    double sum = 0.0;
+    for (int64_t k = 0; k < K; ++k) sum += (double)bf16_to_f32(x[k]);
+    float m = (float)(sum / (double)K);
+    double ss = 0.0;
+    for (int64_t k = 0; k < K; ++k) {
+        c[k] = bf16_to_f32(x[k]) - m;
+        ss += (double)c[k] * (double)c[k];
+    }
+    float ms = (float)(ss / (double)K);
+    float r = sqrtf(ms + eps);
+    return 1.0f / r;
+}
+
+/* Per-channel abs-max of the LayerNorm output y = LN(x) * gamma + beta over the rows (running maximum
+ * with accumulate != 0). work holds K floats. */
+void orc_calibrate_absmax_layernorm(const uint16_t *a, int64_t rows, int64_t cols, int64_t ld, const float *gamma,
+                                    const float *beta, float eps, float *amax, int accumulate, float *work)
+{
+    if (!accumulate)
+        for (int64_t j = 0; j < cols; ++j) amax[j] = 0.0f;
+    for (int64_t r = 0; r < rows; ++r) {
+        float ir = row_layernorm(a + r * ld, cols, eps, work);
+        for (int64_t j = 0; j < cols; ++j) {
+            float y = (work[j] * ir) * gamma[j] + beta[j];
+            float v = fabsf(y);
+            if (v > amax[j]) amax[j] = v;
+        }
+    }
+}
+
+/* The LayerNorm bias with S^-1 folded in: beta_fold[k] = fl32(beta[k] / s[k]). */
+void orc_fold_layernorm_bias(const float *beta, const float *s, int64_t K, float *beta_fold)
+{
+    for (int64_t k = 0; k < K; ++k) beta_fold[k] = beta[k] / s[k];
+}
+
+/* LayerNorm with the folded scale and bias, then per-token symmetric INT8 (the quantiser above). */
+void orc_layernorm_smooth_quant(const uint16_t *x, int64_t T, int64_t K, const float *fold, const float *beta_fold,
+                                float eps, int8_t *xq, float *x_scale, float *work /* [2K] */)
+{
+    float *c = work, *y = work + K;
+    for (int64_t t = 0; t < T; ++t) {
+        float ir = row_layernorm(x + t * K, K, eps, c);
+        for (int64_t k = 0; k < K; ++k) y[k] = (c[k] * ir) * fold[k] + beta_fold[k];
+        quantize_row(y, K, xq + t * K, &x_scale[t]);
+    }
+}
+
+/* ---------------------------------------------------------------------------------------------
  * FP8 E4M3 variant, [W8A8] "One layer, measured" (the same sweep in FP8 E4M3) and "FP8's exponent
  * gives each value its own scale". E4M3 (the OCP "FN" form): 1 sign bit, 4 exponent bits with bias
  * 7, 3 mantissa bits; normals (1 + m/8) * 2^(e-7) for e = 1..15 except the pattern S.1111.111

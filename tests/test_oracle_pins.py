@@ -312,6 +312,58 @@ def test_fold_into_prev_linear_rounding_and_w_scale(orc):
 
 
 # --------------------------------------------------------------------------------------------
+# LayerNorm fold ("SmoothQuant: Weight-Only vs W8A8", "Integration with Transformers": S^-1 into the
+# LayerNorm's gamma and beta): the oracle's LayerNorm against numpy binary64, scale freedom, constant rows, and the fold
+# giving y / s.
+
+def _ln64(x64, g, b, eps):
+    mu = x64.mean(axis=1, keepdims=True)
+    c = x64 - mu
+    return c / np.sqrt((c * c).mean(axis=1, keepdims=True) + eps) * g + b, mu
+
+
+def test_layernorm_calibration_against_fp64(orc):
+    x = rand_bf16((40, 128), 80, scale=2.0)
+    x64 = bits_to_f64(x) + 0.0
+    g = (1 + 0.1 * np.random.default_rng(80).standard_normal(128)).astype(np.float32)
+    b = (0.05 * np.random.default_rng(81).standard_normal(128)).astype(np.float32)
+    amax = orc.calibrate_absmax_layernorm(x, g, b, eps=1e-5)
+    y64, mu = _ln64(x64, g.astype(np.float64), b.astype(np.float64), 1e-5)
+    ref = np.abs(y64).max(axis=0)
+    assert np.all(np.abs(amax - ref) <= 16 * 2.0 ** -24 * (ref + np.abs(b)) + 4 * 2.0 ** -24 * np.abs(mu).max() * np.abs(g) * 10)
+    # running maximum over two batches equals the maximum over their concatenation
+    a2 = orc.calibrate_absmax_layernorm(x[20:], g, b, eps=1e-5, amax=orc.calibrate_absmax_layernorm(x[:20], g, b, eps=1e-5).copy(),
+                                        accumulate=True)
+    assert np.array_equal(a2, amax)
+
+
+def test_layernorm_quant_fold_and_invariances(orc):
+    K = 96
+    x = rand_bf16((12, K), 82, scale=1.5)
+    rng = np.random.default_rng(82)
+    g = (1 + 0.1 * rng.standard_normal(K)).astype(np.float32)
+    b = (0.1 * rng.standard_normal(K)).astype(np.float32)
+    s = (0.5 + rng.random(K) * 4).astype(np.float32)
+    fold = (g / s).astype(np.float32)
+    bf = orc.fold_layernorm_bias(b, s)
+    assert np.array_equal(bf, (b / s).astype(np.float32))
+    xq, xs = orc.layernorm_smooth_quant(x, fold, bf, eps=1e-5)
+    y64, _ = _ln64(bits_to_f64(x), g.astype(np.float64), b.astype(np.float64), 1e-5)
+    t = y64 / s.astype(np.float64)                           # the smoothed activation the codes stand for
+    err = np.abs(xq * xs[:, None].astype(np.float64) - t)
+    assert np.all(err <= xs[:, None] * (0.5 + 1e-4) + 1e-6 * np.abs(t))
+    assert np.all(np.abs(xq).max(axis=1) == 127)
+    # doubling a row (exact) leaves LayerNorm, so the codes, unchanged
+    x2 = bf16_bits(torch.from_numpy(bits_to_f64(x).astype(np.float32) * 2).to(torch.bfloat16))
+    assert np.array_equal(orc.layernorm_smooth_quant(x2, fold, bf, eps=0.0)[0], orc.layernorm_smooth_quant(x, fold, bf, eps=0.0)[0])
+    # a constant row normalises to zero: what remains is the folded bias
+    c = bf16_bits(torch.full((1, K), 0.75).to(torch.bfloat16))
+    qc, sc = orc.layernorm_smooth_quant(c, fold, bf, eps=1e-5)
+    qb, sb = orc.rmsnorm_smooth_quant(bf16_bits(torch.ones(1, K).to(torch.bfloat16)), bf, apply_norm=False)
+    assert np.array_equal(qc, qb) and np.array_equal(sc, sb)
+
+
+# --------------------------------------------------------------------------------------------
 # FP8 E4M3 variant ("SmoothQuant and W8A8...", "One layer, measured"): torch's float8_e4m3fn type
 # is the independent check of the format (decode of every finite code, round-to-nearest-even
 # encode including exact ties and subnormals); saturation at 448 is the closed form.
