@@ -173,6 +173,33 @@ sq_status sq_fold_into_prev_linear(const void *w, const void *b, int64_t K, int6
 sq_status sq_fold_into_w_scale(const float *w_scale, int64_t K, const float *fold, float *w_scale_out, void *stream);
 
 /*
+ * LayerNorm-fed layers: the fold of S^-1 into the scale gamma and the bias beta of the LayerNorm in
+ * front of the smoothed layer ([WOVS] "Integration with Transformers": its output then leaves the
+ * norm already smoothed, at no run-time cost). The pages do not write LayerNorm out; the standard
+ * per-token form is used, each step rounded as listed (fl32 = round to nearest binary32):
+ *   m = fl32(sum_k x_k / K);  c_k = fl32(x_k - m);  ms = fl32(sum_k c_k^2 / K)   (sums in binary64)
+ *   ir = fl32(1 / fl32(sqrt(fl32(ms + eps))));   y_k = fl32(fl32(fl32(c_k * ir) * g_k) + b_k)
+ *
+ * sq_calibrate_absmax_layernorm: per-column abs-max of y over the rows of bf16 a [rows, cols]
+ *   (row stride ld elements) with g = gamma, b = beta (fp32 [cols]; beta nullable = no bias), into
+ *   amax fp32 [cols]; accumulate != 0 keeps the running maximum (amax must then hold non-negative
+ *   values). Requirements as sq_calibrate_absmax; gamma and beta 16-byte aligned; cols <= 16384.
+ * sq_fold_layernorm_bias: beta_fold[k] = fl32(beta[k] / s[k]), fp32 [K], K >= 1 (the scale side,
+ *   fl32(gamma / s), is the fold sq_compute_scales writes when given gamma).
+ * sq_layernorm_smooth_quant: y with g = fold, b = beta_fold (nullable = no bias), then per-token
+ *   symmetric INT8 exactly as sq_rmsnorm_smooth_quant: x bf16 [T, K] -> xq int8 [T, K], x_scale fp32
+ *   [T]. Requirements: T >= 0, 8 <= K <= 16384, K % 8 == 0; x, fold, beta_fold 16-byte aligned, xq
+ *   8-byte aligned.
+ * The binary64 sums are taken in a tree order (see the library's LayerNorm source for when that can
+ * differ from index order).
+ */
+sq_status sq_calibrate_absmax_layernorm(const void *a, int64_t rows, int64_t cols, int64_t ld, const float *gamma,
+                                        const float *beta, float eps, float *amax, int accumulate, void *stream);
+sq_status sq_fold_layernorm_bias(const float *beta, const float *s, int64_t K, float *beta_fold, void *stream);
+sq_status sq_layernorm_smooth_quant(const void *x, int64_t T, int64_t K, const float *fold, const float *beta_fold,
+                                    float eps, int8_t *xq, float *x_scale, void *stream);
+
+/*
  * W8A8 linear: INT8 x INT8 -> INT32 GEMM with the dequantisation fused into its epilogue.
  *   [MIGRATE] section 7 (the integer product accumulated in 32 bits on the tensor cores, then
  *   scaled by the activation and weight scales); [TAMING] "System Architecture" (the flowchart's

@@ -18,7 +18,8 @@ __all__ = [
     "sq_rmsnorm_smooth_quant", "sq_w8a8_linear", "sq_w8a8_linear_workspace_size", "sq_device_status",
     "sq_set_wait_timeout_ns", "sq_selftest_wait_timeout", "sq_set_gemm_cta_pair",
     "sq_static_scale", "sq_rmsnorm_smooth_quant_static", "sq_fold_into_prev_linear", "sq_fold_into_w_scale",
-    "sq_smooth_quantize_weight_fp8", "sq_rmsnorm_smooth_quant_fp8", "sq_w8a8_linear_fp8", "sq_status_string", "sq_last_error",
+    "sq_smooth_quantize_weight_fp8", "sq_rmsnorm_smooth_quant_fp8", "sq_w8a8_linear_fp8", "sq_calibrate_absmax_layernorm", "sq_fold_layernorm_bias",
+    "sq_layernorm_smooth_quant", "sq_status_string", "sq_last_error",
     "sq_version", "LIB_PATH", "EXPORTS",
 ]
 
@@ -53,6 +54,9 @@ EXPORTS = {
     "sq_smooth_quantize_weight_fp8": (_i, [_p, _i64, _i64, _p, _p, _p, _p]),
     "sq_rmsnorm_smooth_quant_fp8": (_i, [_p, _i64, _i64, _p, _f, _i, _p, _p, _p]),
     "sq_w8a8_linear_fp8": (_i, [_p, _p, _i64, _p, _p, _i64, _i64, _p, _p, _p, _p, ctypes.c_size_t, _p]),
+    "sq_calibrate_absmax_layernorm": (_i, [_p, _i64, _i64, _i64, _p, _p, _f, _p, _i, _p]),
+    "sq_fold_layernorm_bias": (_i, [_p, _p, _i64, _p, _p]),
+    "sq_layernorm_smooth_quant": (_i, [_p, _i64, _i64, _p, _p, _f, _p, _p, _p]),
 }
 
 
@@ -244,6 +248,56 @@ def sq_fold_into_w_scale(w_scale: torch.Tensor, fold: torch.Tensor, out: Optiona
     _check(_lib.sq_fold_into_w_scale(_ptr(w_scale), w_scale.shape[0], _ptr(fold), _ptr(out), _stream(stream)),
            "sq_fold_into_w_scale")
     return out
+
+
+def sq_calibrate_absmax_layernorm(a: torch.Tensor, gamma: torch.Tensor, beta: Optional[torch.Tensor] = None,
+                                  eps: float = 1e-5, amax: Optional[torch.Tensor] = None, accumulate: bool = False,
+                                  stream=None) -> torch.Tensor:
+    """Per-column abs-max of LayerNorm(a) * gamma + beta (a bf16, rows may be strided); see sq.h."""
+    _dev(a, "a", torch.bfloat16, contiguous=False)
+    if a.dim() != 2 or a.stride(1) != 1:
+        raise ValueError("a must be 2-D with unit column stride")
+    rows, cols = a.shape
+    if amax is None:
+        amax = torch.empty(cols, dtype=torch.float32, device=a.device)
+        accumulate = False
+    _dev(amax, "amax", torch.float32)
+    _dev(gamma, "gamma", torch.float32)
+    if beta is not None:
+        _dev(beta, "beta", torch.float32)
+    ld = a.stride(0) if a.stride(0) >= cols else cols
+    _check(_lib.sq_calibrate_absmax_layernorm(_ptr(a), rows, cols, ld, _ptr(gamma), _ptr(beta), float(eps), _ptr(amax),
+                                              int(bool(accumulate)), _stream(stream)), "sq_calibrate_absmax_layernorm")
+    return amax
+
+
+def sq_fold_layernorm_bias(beta: torch.Tensor, s: torch.Tensor, out: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    """LayerNorm bias with S^-1 folded in, beta / s; see sq.h."""
+    _dev(beta, "beta", torch.float32)
+    _dev(s, "s", torch.float32)
+    if s.numel() != beta.numel():
+        raise ValueError("beta and s must have the same length")
+    out = torch.empty_like(beta) if out is None else _dev(out, "out", torch.float32)
+    _check(_lib.sq_fold_layernorm_bias(_ptr(beta), _ptr(s), beta.numel(), _ptr(out), _stream(stream)),
+           "sq_fold_layernorm_bias")
+    return out
+
+
+def sq_layernorm_smooth_quant(x: torch.Tensor, fold: torch.Tensor, beta_fold: Optional[torch.Tensor] = None,
+                              eps: float = 1e-5, xq: Optional[torch.Tensor] = None,
+                              x_scale: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Fused LayerNorm (gamma / s, beta / s folded in) + per-token INT8 quantisation; see sq.h."""
+    _dev(x, "x", torch.bfloat16)
+    _dev(fold, "fold", torch.float32)
+    if beta_fold is not None:
+        _dev(beta_fold, "beta_fold", torch.float32)
+    T, K = x.shape
+    xq = torch.empty(T, K, dtype=torch.int8, device=x.device) if xq is None else _dev(xq, "xq", torch.int8)
+    x_scale = torch.empty(T, dtype=torch.float32, device=x.device) if x_scale is None else _dev(x_scale, "x_scale", torch.float32)
+    _check(_lib.sq_layernorm_smooth_quant(_ptr(x), T, K, _ptr(fold), _ptr(beta_fold), float(eps), _ptr(xq), _ptr(x_scale),
+                                          _stream(stream)), "sq_layernorm_smooth_quant")
+    return xq, x_scale
 
 
 def sq_smooth_quantize_weight_fp8(w: torch.Tensor, s: Optional[torch.Tensor] = None, wq: Optional[torch.Tensor] = None,

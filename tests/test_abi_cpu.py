@@ -116,6 +116,24 @@ def test_fold_argument_checks(sqmod):
     assert L.sq_fold_into_w_scale(FAKE + 2, 8, FAKE, FAKE, None) == SQ_ERR_MISALIGNED
 
 
+def test_layernorm_argument_checks(sqmod):
+    L = sqmod.lib()
+    c = L.sq_calibrate_absmax_layernorm
+    assert c(FAKE, 4, 64, 64, None, None, 1e-5, FAKE, 0, None) == SQ_ERR_INVALID_ARG       # no gamma
+    assert c(FAKE, 4, 64, 32, FAKE, None, 1e-5, FAKE, 0, None) == SQ_ERR_INVALID_ARG       # ld < cols
+    assert c(FAKE, 4, 12, 12, FAKE, None, 1e-5, FAKE, 0, None) == SQ_ERR_MISALIGNED        # cols % 8
+    assert c(FAKE, 4, 64, 64, FAKE, FAKE + 4, 1e-5, FAKE, 0, None) == SQ_ERR_MISALIGNED    # beta alignment
+    assert c(FAKE, 4, 32768, 32768, FAKE, None, 1e-5, FAKE, 0, None) == SQ_ERR_UNSUPPORTED
+    assert L.sq_fold_layernorm_bias(FAKE, None, 8, FAKE, None) == SQ_ERR_INVALID_ARG
+    assert L.sq_fold_layernorm_bias(FAKE, FAKE, 0, FAKE, None) == SQ_ERR_INVALID_ARG
+    assert L.sq_fold_layernorm_bias(FAKE + 2, FAKE, 8, FAKE, None) == SQ_ERR_MISALIGNED
+    q = L.sq_layernorm_smooth_quant
+    assert q(FAKE, 4, 64, None, None, 1e-5, FAKE, FAKE, None) == SQ_ERR_INVALID_ARG         # no fold
+    assert q(FAKE, 4, 64, FAKE, FAKE + 4, 1e-5, FAKE, FAKE, None) == SQ_ERR_MISALIGNED      # beta_fold alignment
+    assert q(FAKE, 4, 32768, FAKE, None, 1e-5, FAKE, FAKE, None) == SQ_ERR_UNSUPPORTED
+    assert q(FAKE, -1, 64, FAKE, None, 1e-5, FAKE, FAKE, None) == SQ_ERR_INVALID_ARG
+
+
 def test_fp8_argument_checks(sqmod):
     L = sqmod.lib()
     assert L.sq_smooth_quantize_weight_fp8(FAKE, 4, 12, None, FAKE, FAKE, None) == SQ_ERR_MISALIGNED

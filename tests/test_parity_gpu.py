@@ -394,6 +394,57 @@ def test_fp8_path(sq, orc, T, N, K, norm, bias):
     assert np.all(np.abs(f64(h16(y)) - ref) <= 1e-2 * np.abs(ref) + 1e-2 * 2.0 ** -8 * (scale_mag + (np.abs(f64(b_h))[None, :] if bias else 0)) + 1e-30)
 
 
+# LayerNorm fold: the calibration abs-max of LayerNorm(x) * gamma + beta, the folded bias beta / s and
+# the fused LayerNorm + INT8 quantiser, bit-exact against the oracle. Tokens carry a common offset
+# (so the centring matters); one row is zero and one constant (both normalise to c = 0, so y is the
+# folded bias alone); calibration reads strided rows in two batches (running maximum). Widths reach
+# every block shape of the kernel (1, 2 and 4 vectors per thread; 32..512 threads) with ragged ones.
+LN_SHAPES = [(300, 64, True), (777, 1040, False), (1000, 4096, True), (513, 8192, True), (129, 12288, False),
+             (64, 16384, True)]
+
+
+@pytest.mark.parametrize("T,K,bias", LN_SHAPES)
+def test_layernorm_fold_path(sq, orc, T, K, bias):
+    dev = "cuda"
+    seed = 7 * T + K
+    ch = synth.outlier_channels(K, synth.OutlierSpec(max(1, K // 128), 10.0, 60.0), seed)
+    Xc = (synth.outlier_tokens(2 * T, K, ch, seed + 1, dev).float() + 3.0).to(torch.bfloat16)
+    X = (synth.outlier_tokens(T, K, ch, seed + 2, dev).float() + 3.0).to(torch.bfloat16)
+    X[T // 2].zero_()
+    X[T // 3] = 0.75
+    g = torch.Generator(device="cpu").manual_seed(seed + 3)
+    gamma = (1 + 0.2 * torch.randn(K, generator=g)).to(dev)
+    beta = (0.1 * torch.randn(K, generator=g)).to(dev) if bias else None
+    zeros = np.zeros(K, np.float32)
+    big = torch.zeros(2 * T, K + 16, dtype=torch.bfloat16, device=dev)
+    big[:, :K] = Xc
+    amax = sq.sq_calibrate_absmax_layernorm(big[:T, :K], gamma, beta)
+    sq.sq_calibrate_absmax_layernorm(big[T:, :K], gamma, beta, amax=amax, accumulate=True)
+    ok_status(sq)
+    amax_o = orc.calibrate_absmax_layernorm(h16(Xc), hnp(gamma), hnp(beta) if bias else zeros)
+    assert np.array_equal(hnp(amax), amax_o), f"{int((hnp(amax) != amax_o).sum())} LayerNorm abs-maxima differ"
+    N = 264
+    W = synth.normal_weight(N, K, seed + 4, dev)
+    s, fold = sq.sq_compute_scales(amax, sq.sq_calibrate_absmax(W), 0.5, gamma=gamma)
+    bf = sq.sq_fold_layernorm_bias(beta, s) if bias else None
+    if bias:
+        assert np.array_equal(hnp(bf), orc.fold_layernorm_bias(hnp(beta), hnp(s)))
+    xq, xs = sq.sq_layernorm_smooth_quant(X, fold, bf)
+    ok_status(sq)
+    xq_o, xs_o = orc.layernorm_smooth_quant(h16(X), hnp(fold), hnp(bf) if bias else zeros)
+    assert np.array_equal(hnp(xs), xs_o), f"{int((hnp(xs) != xs_o).sum())} LayerNorm token scales differ"
+    assert np.array_equal(hnp(xq), xq_o), f"{int((hnp(xq) != xq_o).sum())} LayerNorm codes differ"
+    if bias:   # a zero row and a constant row both quantise the folded bias alone
+        assert np.array_equal(hnp(xq)[T // 2], hnp(xq)[T // 3]) and hnp(xs)[T // 2] == hnp(xs)[T // 3] > 0
+    else:
+        assert hnp(xs)[T // 2] == 0 and hnp(xs)[T // 3] == 0 and not hnp(xq)[T // 3].any()
+    wq, ws = sq.sq_smooth_quantize_weight(W, s)
+    acc = torch.empty(T, N, dtype=torch.int32, device=dev)
+    y = sq.sq_w8a8_linear(xq, xs, wq, ws, acc_out=acc)
+    check_linear(sq, orc, xq, xs, wq, ws, None, y, acc)
+    ok_status(sq)
+
+
 def test_deterministic_bytes(sq):
     w = synth.WORKLOADS[1]
     d = synth.group_inputs(w, 0, "cuda", T=1000)
