@@ -144,6 +144,15 @@ static __device__ __forceinline__ uint64_t add2_rn(uint64_t a, uint64_t b) {
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
     return d;
 }
+// fl(a + b) for both halves with scalar round-to-nearest adds, which the compiler never contracts
+// with a preceding multiply into a fused multiply-add (a packed add after a packed multiply can be
+// contracted, so a sum that must be rounded on its own uses this form).
+static __device__ __forceinline__ uint64_t add2_scalar(uint64_t a, uint64_t b) {
+    uint32_t al, ah, bl, bh;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(al), "=r"(ah) : "l"(a));
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(bl), "=r"(bh) : "l"(b));
+    return pack2(__fadd_rn(__uint_as_float(al), __uint_as_float(bl)), __fadd_rn(__uint_as_float(ah), __uint_as_float(bh)));
+}
 static __device__ __forceinline__ uint64_t add2_rz(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("add.rz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));

@@ -1,9 +1,11 @@
 // sq_fold.cu -- fold of the smoothing factor 1/s into the previous linear layer, the alternative to
 // folding it into a norm's weight.
 //
-// Page cited: [MIGRATE] "06 -- SmoothQuant: Migrating Difficulty from Activations to Weights",
+// Pages cited: [MIGRATE] "06 -- SmoothQuant: Migrating Difficulty from Activations to Weights",
 // section 7 (the division X / s is absorbed by multiplying the previous layer's output-column-j
-// weights by 1 / s_j; zero run-time cost).
+// weights by 1 / s_j; zero run-time cost); [WOVS] "SmoothQuant: Weight-Only vs W8A8", "Integration
+// with Transformers" (S^-1 folded into a LayerNorm's gamma and beta: beta / s here, gamma / s is
+// the fold the smoothing-factor kernel writes).
 //
 // The previous layer's weight is bf16 [K, Kp] (its output channel j feeds input channel j of the
 // smoothed layer): row j is multiplied by fold[j] = fl32(1 / s_j) and rounded to bf16 (nearest,
@@ -52,6 +54,15 @@ __global__ void k_fold_w_scale(const float *ws, int64_t K, const float *__restri
         out[j] = __fmul_rn(ws[j], fold[j]);
 }
 
+// beta_fold[k] = fl32(beta[k] / s[k]): the LayerNorm bias with S^-1 folded in.
+__global__ void k_fold_ln_bias(const float *__restrict__ beta, const float *__restrict__ s, int64_t K,
+                               float *__restrict__ out)
+{
+    for (int64_t k = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; k < K;
+         k += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        out[k] = __fdiv_rn(beta[k], s[k]);
+}
+
 }  // namespace
 
 extern "C" {
@@ -88,6 +99,19 @@ sq_status sq_fold_into_w_scale(const float *w_scale, int64_t K, const float *fol
     k_fold_w_scale<<<static_cast<unsigned>((K + 255) / 256 < 1024 ? (K + 255) / 256 : 1024), 256, 0, sq::as_stream(stream)>>>(
         w_scale, K, fold, w_scale_out);
     return sq::cuda_status(cudaGetLastError(), "launch(fold_w_scale)");
+}
+
+sq_status sq_fold_layernorm_bias(const float *beta, const float *s, int64_t K, float *beta_fold, void *stream)
+{
+    using sq::fail;
+    if (K < 1 || !beta || !s || !beta_fold) return fail(SQ_ERR_INVALID_ARG, "sq_fold_layernorm_bias: need K >= 1 and all arrays");
+    if (!sq::aligned(beta, 4) || !sq::aligned(s, 4) || !sq::aligned(beta_fold, 4))
+        return fail(SQ_ERR_MISALIGNED, "sq_fold_layernorm_bias: fp32 arrays must be 4-byte aligned");
+    int dev = 0;
+    SQ_TRY_ARCH(dev);
+    k_fold_ln_bias<<<static_cast<unsigned>((K + 255) / 256 < 1024 ? (K + 255) / 256 : 1024), 256, 0, sq::as_stream(stream)>>>(
+        beta, s, K, beta_fold);
+    return sq::cuda_status(cudaGetLastError(), "launch(fold_layernorm_bias)");
 }
 
 }  // extern "C"

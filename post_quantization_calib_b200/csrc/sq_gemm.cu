@@ -374,10 +374,12 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tmem_base, int quad, int 
             uint64_t v01 = mul2_rn(a01, mul2_rn(xs2, w01));
             uint64_t v23 = mul2_rn(a23, mul2_rn(xs2, w23));
             if (has_bias) {
+                // scalar round-to-nearest adds: never contracted with the multiply before them into
+                // a fused multiply-add (a packed add after a packed multiply can be)
                 uint64_t b01, b23;
                 lds_pairs(tab + TN + c * OUT_COLS + 4 * g, b01, b23);
-                v01 = add2_rn(v01, b01);
-                v23 = add2_rn(v23, b23);
+                v01 = add2_scalar(v01, b01);
+                v23 = add2_scalar(v23, b23);
             }
             packed[2 * g] = bf16x2_rn(v01);
             packed[2 * g + 1] = bf16x2_rn(v23);

@@ -7,6 +7,7 @@
 //   [MIGRATE] "06 -- SmoothQuant: Migrating Difficulty from Activations to Weights"
 //   [TAMING]  "Taming the Outliers: A Deep Dive into SmoothQuant for LLM Quantization"
 //   [W8A8]    "SmoothQuant and W8A8: Quantizing Activations Too"
+//   [WOVS]    "SmoothQuant: Weight-Only vs W8A8"
 //
 // Design (B200). One kernel template serves the abs-max (MODE_ABSMAX) and the quantisers
 // (MODE_QUANT). A CTA (one per SM) has 16 warps, 4 per scheduler. Rows of up to 2048 elements are
@@ -69,7 +70,9 @@ constexpr unsigned kAll = 0xFFFFFFFFu;
 
 // MODE_QSTATIC: the quantiser with one static per-tensor scale (no row maximum; codes clamped).
 // MODE_QF8: the per-row quantiser with FP8 E4M3 codes (scale max/448).
-enum { MODE_ABSMAX = 0, MODE_QUANT = 1, MODE_QSTATIC = 2, MODE_QF8 = 3 };
+// MODE_QLN / MODE_ALN: the per-row quantiser and the column abs-max of a LayerNorm's output
+// y = fl(fl(fl(c * inv_std) * g) + b), c = fl(x - mean) (g from vec, b from vec2).
+enum { MODE_ABSMAX = 0, MODE_QUANT = 1, MODE_QSTATIC = 2, MODE_QF8 = 3, MODE_QLN = 4, MODE_ALN = 5 };
 constexpr float kF8Max = 448.0f;  // largest finite E4M3 value
 
 struct RowArgs {
@@ -79,6 +82,7 @@ struct RowArgs {
     int K;                  // bf16 elements per row (multiple of 8)
     int stages;             // ring slots per row group
     const float *vec;       // ABSMAX: norm gamma (NORM) ; QUANT: per-column factor c (nullable)
+    const float *vec2;      // LayerNorm modes: per-column bias b (nullable = none)
     float eps;
     double inv_k;           // 1 / K when K is a power of two (exact), else 0
     float *amax;            // ABSMAX output [K] (running maximum; pre-zeroed when overwriting)
@@ -144,8 +148,9 @@ __device__ __forceinline__ float rows_max(float (&v)[R], int lane) {
     return v[0];
 }
 
-// |x| * 2^-411 in binary64 for the bf16 x held (sign cleared) in bits 30..16 of `a`: one 64-bit
-// multiply-add a * 2^29 + (485 << 52) writes both halves of the register pair (low half zero).
+// |x| * 2^-411 in binary64 for the binary32 bits of |x| in `a` (a bf16 x: its bits in 30..16, the
+// low half zero): one 64-bit multiply-add a * 2^29 + (485 << 52) writes both halves of the
+// register pair.
 __device__ __forceinline__ double sq_operand(uint32_t a) {
     double d;
     asm("{\n\t.reg .u64 t;\n\tmad.wide.u32 t, %1, 536870912, %2;\n\tmov.b64 %0, t;\n\t}"
@@ -176,6 +181,24 @@ __device__ __forceinline__ uint32_t word_of(const uint4 &v, int k) {
 
 // bf16 pair -> packed binary32 pair (exact)
 __device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) { return pack2u(w << 16, w & 0xFFFF0000u); }
+
+// Adds the two bf16 values of `w` (exactly converted) to the binary64 sums a and b.
+__device__ __forceinline__ void add_values(uint32_t w, double &a, double &b) {
+    a = __dadd_rn(a, static_cast<double>(__uint_as_float(w << 16)));
+    b = __dadd_rn(b, static_cast<double>(__uint_as_float(w & 0xFFFF0000u)));
+}
+
+// Adds the squares of c = fl(x - m) for the two bf16 values x of `w` (nm2 = {-m, -m}) to the
+// scaled binary64 accumulators a and b: one 64-bit multiply-add places the binary32 |c| in the
+// binary64 fields with exponent bias +485, i.e. |c| * 2^-411, exact for normal |c| >= 2^-100 (a zero
+// becomes 2^-538, whose square rounds away in the fused multiply-add).
+__device__ __forceinline__ void add_centred_squares(uint32_t w, uint64_t nm2, double &a, double &b) {
+    uint32_t cl, ch;
+    unpack2(add2_rn(bf2_to_f2(w), nm2), cl, ch);
+    const double dl = sq_operand(cl & 0x7FFFFFFFu), dh = sq_operand(ch & 0x7FFFFFFFu);
+    a = __fma_rn(dl, dl, a);
+    b = __fma_rn(dh, dh, b);
+}
 
 // Signed INT8 codes of the two values of t: round half away from zero. v = rz(t + copysign(1/2, t))
 // has the integer part of the exactly rounded value, and the conversion truncates it.
@@ -210,6 +233,27 @@ __device__ __forceinline__ uint32_t codes2_clamped(uint64_t t) {
     return codes2(pack2(a, b));
 }
 
+// LayerNorm parameters of vector v (8 columns) as binary32 pairs: g from the shared-memory table,
+// b from global memory (nullable: zeros).
+__device__ __forceinline__ void ln_params(const float4 *c_lo, const float4 *c_hi, const float *b, int v,
+                                          uint64_t (&g2)[4], uint64_t (&b2)[4]) {
+    const float4 gl = c_lo[v], gh = c_hi[v];
+    g2[0] = pack2(gl.x, gl.y); g2[1] = pack2(gl.z, gl.w); g2[2] = pack2(gh.x, gh.y); g2[3] = pack2(gh.z, gh.w);
+    float4 bl = make_float4(0.f, 0.f, 0.f, 0.f), bh = bl;
+    if (b != nullptr) {
+        bl = __ldg(reinterpret_cast<const float4 *>(b) + 2 * v);
+        bh = __ldg(reinterpret_cast<const float4 *>(b) + 2 * v + 1);
+    }
+    b2[0] = pack2(bl.x, bl.y); b2[1] = pack2(bl.z, bl.w); b2[2] = pack2(bh.x, bh.y); b2[3] = pack2(bh.z, bh.w);
+}
+
+// y = fl(fl(fl(c * ir) * g) + b) with c = fl(x - m), for the two bf16 values x of `w` (nm2 = {-m, -m}).
+// The bias goes in with scalar adds (add2_scalar): a packed add here was contracted with the
+// multiply before it, which rounds y once instead of twice.
+__device__ __forceinline__ uint64_t ln_y2(uint32_t w, uint64_t nm2, uint64_t ir2, uint64_t g2, uint64_t b2) {
+    return add2_scalar(mul2_rn(mul2_rn(add2_rn(bf2_to_f2(w), nm2), ir2), g2), b2);
+}
+
 // 3-input maximum (one instruction on sm_100)
 __device__ __forceinline__ float max3f(float a, float b, float c) {
     float d;
@@ -227,9 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
     constexpr int GT = 32 * WPR;      // consumer threads per row group
     constexpr int SUB = 32 / R;       // lanes that hold one row's total after a butterfly
     static_assert(R >= 1 && R <= 8 && VPL * R <= 8, "a unit gives a lane at most 64 element-rows");
+    constexpr bool LN = MODE == MODE_QLN || MODE == MODE_ALN;       // LayerNorm: mean removed, bias added
+    constexpr bool ABS = MODE == MODE_ABSMAX || MODE == MODE_ALN;   // column abs-max: rows re-read from the slot
+    static_assert(!LN || NORM, "the LayerNorm modes normalise");
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[G * kMaxStages];
     __shared__ double s_ss[2][kWarps][R];
+    __shared__ double s_ss2[LN ? 2 : 1][kWarps][LN ? R : 1];   // LayerNorm: the centred sums of squares
     __shared__ float s_mx[2][kWarps][R];
     __shared__ int s_abort[G];
 
@@ -243,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
     const int stages = p.stages;
     uint8_t *ring = smem;
     const size_t ring_bytes = static_cast<size_t>(G) * stages * slotbytes;
-    const size_t red_bytes = MODE == MODE_ABSMAX ? static_cast<size_t>(G) * K * 4 : 0;
+    const size_t red_bytes = ABS ? static_cast<size_t>(G) * K * 4 : 0;
     float4 *c_lo = reinterpret_cast<float4 *>(smem + (ring_bytes > red_bytes ? ring_bytes : red_bytes));   // c[8v .. 8v+3]
     float4 *c_hi = c_lo + nvec;                                                                              // c[8v+4 .. 8v+7]
     const bool has_vec = p.vec != nullptr;
@@ -344,8 +392,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                     const bool in = (FULL || v < nvec) && r < nr;
                     if (MODE == MODE_ABSMAX && !NORM) continue;
                     const uint4 q = in ? rp[r * rv + v] : make_uint4(0u, 0u, 0u, 0u);
-                    if (MODE != MODE_ABSMAX) xr[r][i] = q;
-                    if (NORM) {
+                    if (!ABS) xr[r][i] = q;
+                    if (LN) {                                   // the row sums of x (absent: zeros)
+                        if (i & 1) { add_values(q.x, a2, a3); add_values(q.y, a2, a3); add_values(q.z, a2, a3); add_values(q.w, a2, a3); }
+                        else { add_values(q.x, a0, a1); add_values(q.y, a0, a1); add_values(q.z, a0, a1); add_values(q.w, a0, a1); }
+                    } else if (NORM) {
                         if (i & 1) { add_squares<MODE == MODE_ABSMAX>(q.x, a2, a3); add_squares<MODE == MODE_ABSMAX>(q.y, a2, a3); add_squares<MODE == MODE_ABSMAX>(q.z, a2, a3); add_squares<MODE == MODE_ABSMAX>(q.w, a2, a3); }
                         else { add_squares<MODE == MODE_ABSMAX>(q.x, a0, a1); add_squares<MODE == MODE_ABSMAX>(q.y, a0, a1); add_squares<MODE == MODE_ABSMAX>(q.z, a0, a1); add_squares<MODE == MODE_ABSMAX>(q.w, a0, a1); }
                     }
@@ -365,16 +416,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                     break;
                 }
                 if (leader) {
-                    if (MODE != MODE_ABSMAX) refill(j, st);
+                    if (!ABS) refill(j, st);
                     else if (j > 0) refill(j - 1, st == 0 ? stages - 1 : st - 1);
                 }
-            } else if (MODE != MODE_ABSMAX) {
+            } else if (!ABS) {
                 __syncwarp();                                   // the unit is in registers now
                 if (leader) refill(j, st);
             }
 
-            // ---- 1 / rms of every row of the unit, broadcast to all lanes
+            // ---- 1 / rms (LayerNorm: the mean, then 1 / standard deviation) of every row of the
+            // unit, broadcast to all lanes
             float ir[R];
+            float mu[R];
             if (NORM) {
                 double ss;
                 if (WPR > 1) {
@@ -384,6 +437,39 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                 } else {
                     ss = rows_sum<R>(ssr, lane);                // total of row lane / SUB
                 }
+                if (LN) {
+                    // ss is the row's sum of x: its mean, then the scaled sum of the squares of
+                    // c = fl(x - mean) (a second group step when the row spans several warps)
+                    const float mean = __double2float_rn(p.inv_k != 0.0 ? __dmul_rn(ss, p.inv_k)
+                                                                        : __ddiv_rn(ss, static_cast<double>(K)));
+#pragma unroll
+                    for (int r = 0; r < R; ++r) mu[r] = __shfl_sync(kAll, mean, r * SUB);
+                    double sq2[R];
+#pragma unroll
+                    for (int r = 0; r < R; ++r) {
+                        const uint64_t nm2 = pack2(-mu[r], -mu[r]);
+                        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+#pragma unroll
+                        for (int i = 0; i < VPL; ++i) {
+                            const int v = i * GT + gtid;
+                            if (!((FULL || v < nvec) && r < nr)) continue;
+                            const uint4 q = ABS ? rp[r * rv + v] : xr[r][i];
+                            if (i & 1) { add_centred_squares(q.x, nm2, a2, a3); add_centred_squares(q.y, nm2, a2, a3); add_centred_squares(q.z, nm2, a2, a3); add_centred_squares(q.w, nm2, a2, a3); }
+                            else { add_centred_squares(q.x, nm2, a0, a1); add_centred_squares(q.y, nm2, a0, a1); add_centred_squares(q.z, nm2, a0, a1); add_centred_squares(q.w, nm2, a0, a1); }
+                        }
+                        sq2[r] = (a0 + a1) + (a2 + a3);
+                    }
+                    if (WPR > 1) {
+                        const double part = rows_sum<R>(sq2, lane);
+                        if (lane % SUB == 0) s_ss2[j & 1][warp][lane / SUB] = part;
+                        named_sync(1 + group, GT);
+                        ss = 0.0;
+#pragma unroll
+                        for (int w = 0; w < WPR; ++w) ss += s_ss2[j & 1][group * WPR + w][lane / SUB];
+                    } else {
+                        ss = rows_sum<R>(sq2, lane);
+                    }
+                }
                 const float mine = inv_rms(__dmul_rn(ss, 0x1p822), K, p.inv_k, p.eps);
 #pragma unroll
                 for (int r = 0; r < R; ++r) ir[r] = __shfl_sync(kAll, mine, r * SUB);
@@ -392,15 +478,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                 for (int r = 0; r < R; ++r) ir[r] = 1.0f;
             }
 
-            if (MODE == MODE_ABSMAX) {
+            if (ABS) {
                 // ---- pass B: running column maxima
 #pragma unroll
                 for (int i = 0; i < VPL; ++i) {
                     const int v = i * GT + gtid;
+                    uint64_t g2[4], b2[4];                      // LayerNorm: gamma and beta pairs
+                    if (LN && (FULL || v < nvec)) ln_params(c_lo, c_hi, p.vec2, v, g2, b2);
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
                         if (!((FULL || v < nvec) && r < nr)) continue;
-                        if (NORM) {
+                        if (LN) {
+                            const uint64_t ir2 = pack2(ir[r], ir[r]), nm2 = pack2(-mu[r], -mu[r]);
+                            const uint4 q = rp[r * rv + v];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                uint32_t l, h;
+                                unpack2(ln_y2(word_of(q, k), nm2, ir2, g2[k], b2[k]), l, h);
+                                mx[i][2 * k] = fmaxf(mx[i][2 * k], fabsf(__uint_as_float(l)));
+                                mx[i][2 * k + 1] = fmaxf(mx[i][2 * k + 1], fabsf(__uint_as_float(h)));
+                            }
+                        } else if (NORM) {
                             const uint64_t ir2 = pack2(ir[r], ir[r]);
                             const uint4 q = rp[r * rv + v];
 #pragma unroll
@@ -469,14 +567,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                     const bool in = FULL || v < nvec;
                     float4 cl = make_float4(1.f, 1.f, 1.f, 1.f), ch = cl;
                     if (has_vec && in) { cl = c_lo[v]; ch = c_hi[v]; }
-                    const uint64_t c2[4] = {pack2(cl.x, cl.y), pack2(cl.z, cl.w), pack2(ch.x, ch.y), pack2(ch.z, ch.w)};
+                    uint64_t c2[4] = {pack2(cl.x, cl.y), pack2(cl.z, cl.w), pack2(ch.x, ch.y), pack2(ch.z, ch.w)};
+                    uint64_t b2[4];                             // LayerNorm: beta pairs
+                    if (LN && in) ln_params(c_lo, c_hi, p.vec2, v, c2, b2);
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
                         const uint64_t ir2 = pack2(ir[r], ir[r]);
+                        const uint64_t nm2 = LN ? pack2(-mu[r], -mu[r]) : 0ull;
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const uint64_t x2 = bf2_to_f2(word_of(xr[r][i], k));
-                            const uint64_t yy = NORM ? mul2_rn(mul2_rn(x2, ir2), c2[k]) : (has_vec ? mul2_rn(x2, c2[k]) : x2);
+                            // LayerNorm: an absent vector must not reach the row maximum (its y is not 0)
+                            const uint64_t yy = LN ? (in ? ln_y2(word_of(xr[r][i], k), nm2, ir2, c2[k], b2[k]) : 0ull)
+                                              : NORM ? mul2_rn(mul2_rn(x2, ir2), c2[k]) : (has_vec ? mul2_rn(x2, c2[k]) : x2);
                             y[r][i][k] = yy;
                             uint32_t yl, yh;
                             unpack2(yy, yl, yh);
@@ -538,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
     }
     __syncthreads();
 
-    if (MODE == MODE_ABSMAX) {
+    if (ABS) {
         __syncthreads();                                   // the ring is idle: reuse it
         float *red = reinterpret_cast<float *>(smem);      // [G][K]
         {
@@ -560,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
             float m = red[c];
 #pragma unroll
             for (int g = 1; g < G; ++g) m = fmaxf(m, red[static_cast<size_t>(g) * K + c]);
-            if (NORM) m = __fmul_rn(m, fabsf(__ldg(p.vec + c)));
+            if (NORM && !LN) m = __fmul_rn(m, fabsf(__ldg(p.vec + c)));
             red[c] = m;
         }
         cg::cluster_group cluster = cg::this_cluster();
@@ -639,7 +742,7 @@ size_t rows_smem(int K, int mode, const Geo &g, int stages) {
     const size_t slotbytes = static_cast<size_t>(K) * 2 * g.rpu;
     const size_t ctab = mode != MODE_ABSMAX ? static_cast<size_t>(K) * 4 : 0;
     const size_t ring = static_cast<size_t>(g.groups) * stages * slotbytes;
-    const size_t red = mode == MODE_ABSMAX ? static_cast<size_t>(g.groups) * K * 4 : 0;
+    const size_t red = mode == MODE_ABSMAX || mode == MODE_ALN ? static_cast<size_t>(g.groups) * K * 4 : 0;
     return (ring > red ? ring : red) + ctab;
 }
 
@@ -662,6 +765,7 @@ template <int WPR, int VPL, int R, int MODE, bool NORM, bool FULL>
 sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
     auto kern = k_rows<WPR, VPL, R, MODE, NORM, FULL>;
     constexpr int G = kWarps / WPR;
+    constexpr bool ABS = MODE == MODE_ABSMAX || MODE == MODE_ALN;   // column abs-max: cluster launch
     static size_t configured_smem[64];
     static int per_sm[64];
     static int cluster_size[64], cluster_ctas[64];
@@ -696,7 +800,7 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, smem);
         if (e != cudaSuccess) return sq::cuda_status(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor(rows)");
         per_sm[dev] = nb > 0 ? nb : 1;
-        if (MODE == MODE_ABSMAX) {
+        if (ABS) {
             // Whole clusters must fit on one GPU processing cluster; take the size that keeps the
             // most CTAs resident at once (ties: the larger cluster, fewer atomics).
             cluster_size[dev] = 1;
@@ -720,7 +824,7 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
     a.stream_once = static_cast<double>(a.rows) * static_cast<double>(a.ld_bytes) > 0.5 * sq::l2_bytes(dev) ? 1 : 0;
     if (a.status == nullptr) return sq::fail(SQ_ERR_CUDA, "device status word unavailable");
     const int64_t units = (a.rows + R - 1) / R;
-    if (MODE != MODE_ABSMAX) {
+    if (!ABS) {
         int64_t ctas = (units + G - 1) / G;
         if (ctas > full) ctas = full;
         kern<<<static_cast<unsigned>(ctas), kThreads, smem, st>>>(a);
@@ -794,6 +898,75 @@ sq_status sq_calibrate_absmax(const void *a, int64_t rows, int64_t cols, int64_t
     ra.eps = eps;
     ra.amax = amax;
     return norm_gamma ? dispatch_rows<MODE_ABSMAX, true>(ra, dev, st) : dispatch_rows<MODE_ABSMAX, false>(ra, dev, st);
+}
+
+// LayerNorm-fed layers ([WOVS] "SmoothQuant: Weight-Only vs W8A8", "Integration with
+// Transformers": S^-1 folded into the LayerNorm's gamma and beta). LayerNorm in the standard form,
+// each step rounded as listed: m = fl32(sum x / K) and ms = fl32(sum c^2 / K) with binary64 sums,
+// c = fl32(x - m), ir = fl32(1 / fl32(sqrt(fl32(ms + eps)))), y = fl32(fl32(fl32(c * ir) * g) + b).
+// The sum of x is exact unless a row's nonzero magnitudes span more than about 2^31; both binary64
+// sums are taken in a tree order, which can differ from another order only by binary64 roundings.
+sq_status sq_calibrate_absmax_layernorm(const void *a, int64_t rows, int64_t cols, int64_t ld, const float *gamma,
+                                        const float *beta, float eps, float *amax, int accumulate, void *stream)
+{
+    using sq::fail;
+    if (!amax || !gamma) return fail(SQ_ERR_INVALID_ARG, "sq_calibrate_absmax_layernorm: amax and gamma are required");
+    if (rows < 0 || cols < 8 || ld < cols)
+        return fail(SQ_ERR_INVALID_ARG, "sq_calibrate_absmax_layernorm: need rows >= 0, cols >= 8, ld >= cols (rows=%lld cols=%lld ld=%lld)",
+                    (long long)rows, (long long)cols, (long long)ld);
+    if (rows > 0 && !a) return fail(SQ_ERR_INVALID_ARG, "sq_calibrate_absmax_layernorm: a is NULL");
+    if (cols % 8 != 0 || ld % 8 != 0)
+        return fail(SQ_ERR_MISALIGNED, "sq_calibrate_absmax_layernorm: cols and ld must be multiples of 8");
+    if ((a && !sq::aligned(a, 16)) || !sq::aligned(gamma, 16) || (beta && !sq::aligned(beta, 16)) || !sq::aligned(amax, 4))
+        return fail(SQ_ERR_MISALIGNED, "sq_calibrate_absmax_layernorm: a, gamma and beta 16-byte, amax 4-byte alignment required");
+    if (cols > kMaxK) return fail(SQ_ERR_UNSUPPORTED, "sq_calibrate_absmax_layernorm: cols must be <= %d", kMaxK);
+    int dev = 0;
+    SQ_TRY_ARCH(dev);
+    cudaStream_t st = sq::as_stream(stream);
+    if (!accumulate) {
+        k_fill_zero<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(amax, cols);
+        sq_status s0 = sq::cuda_status(cudaGetLastError(), "launch(fill)");
+        if (s0 != SQ_OK) return s0;
+    }
+    if (rows == 0) return SQ_OK;
+    RowArgs ra = {};
+    ra.src = static_cast<const uint8_t *>(a);
+    ra.rows = rows;
+    ra.ld_bytes = ld * 2;
+    ra.K = static_cast<int>(cols);
+    ra.vec = gamma;
+    ra.vec2 = beta;
+    ra.eps = eps;
+    ra.amax = amax;
+    return dispatch_rows<MODE_ALN, true>(ra, dev, st);
+}
+
+sq_status sq_layernorm_smooth_quant(const void *x, int64_t T, int64_t K, const float *fold, const float *beta_fold,
+                                    float eps, int8_t *xq, float *x_scale, void *stream)
+{
+    using sq::fail;
+    if (T < 0 || K < 8) return fail(SQ_ERR_INVALID_ARG, "sq_layernorm_smooth_quant: need T >= 0 and K >= 8");
+    if (!fold) return fail(SQ_ERR_INVALID_ARG, "sq_layernorm_smooth_quant: fold is required");
+    if (T > 0 && (!x || !xq || !x_scale)) return fail(SQ_ERR_INVALID_ARG, "sq_layernorm_smooth_quant: x, xq and x_scale are required");
+    if (K % 8 != 0) return fail(SQ_ERR_MISALIGNED, "sq_layernorm_smooth_quant: K must be a multiple of 8");
+    if (K > kMaxK) return fail(SQ_ERR_UNSUPPORTED, "sq_layernorm_smooth_quant: K must be <= %d", kMaxK);
+    if ((x && !sq::aligned(x, 16)) || (xq && !sq::aligned(xq, 8)) || !sq::aligned(fold, 16) ||
+        (beta_fold && !sq::aligned(beta_fold, 16)) || (x_scale && !sq::aligned(x_scale, 4)))
+        return fail(SQ_ERR_MISALIGNED, "sq_layernorm_smooth_quant: x, fold and beta_fold 16-byte, xq 8-byte, x_scale 4-byte alignment required");
+    int dev = 0;
+    SQ_TRY_ARCH(dev);
+    if (T == 0) return SQ_OK;
+    RowArgs ra = {};
+    ra.src = static_cast<const uint8_t *>(x);
+    ra.rows = T;
+    ra.ld_bytes = K * 2;
+    ra.K = static_cast<int>(K);
+    ra.vec = fold;
+    ra.vec2 = beta_fold;
+    ra.eps = eps;
+    ra.q = xq;
+    ra.scale = x_scale;
+    return dispatch_rows<MODE_QLN, true>(ra, dev, sq::as_stream(stream));
 }
 
 sq_status sq_compute_scales(const float *amax_x, const float *amax_w, int64_t K, float alpha,
