@@ -250,9 +250,10 @@ def main_gpu(args, rank, local_rank, world):
     stream = torch.cuda.current_stream(dev)
     names = list(LAUNCHES)
 
-    def step(ev=None):
+    # ev: events recorded at the stage boundaries listed in `at` (None: all seven)
+    def step(ev=None, at=None):
         def mark(i):
-            if ev is not None:
+            if ev is not None and (at is None or i in at):
                 ev[i].record(stream)
         mark(0)
         sq.sq_calibrate_absmax(calib, norm_gamma=gamma, eps=w.eps, amax=amax, accumulate=False, stream=stream)
@@ -280,6 +281,21 @@ def main_gpu(args, rank, local_rank, world):
     if st != 0:
         raise RuntimeError(f"device status {sq.sq_status_string(st)} after warm-up")
 
+    # Stage breakdown: a separate, untimed pass with an event at every stage boundary. An event between
+    # two kernels stops the second from starting early (dependent launch) and cost ~20 us per step, so
+    # the timed steps below record events only around the dominant stage.
+    nb = max(3, min(args.steps, 200))
+    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(nb)]
+    for i in range(nb):
+        step(bevs[i])
+    torch.cuda.synchronize()
+    stage_ms = {n: 0.0 for n in names}
+    for e in bevs:
+        for j, n in enumerate(names):
+            stage_ms[n] += e[j].elapsed_time(e[j + 1])
+    stage_ms = {n: v / nb for n, v in stage_ms.items()}
+    dom_i = max(range(len(names)), key=lambda j: stage_ms[names[j]])
+
     clocks = ClockSampler(local_rank)
     clocks.start()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
@@ -289,7 +305,7 @@ def main_gpu(args, rank, local_rank, world):
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for i in range(args.steps):
-        step(evs[i])
+        step(evs[i], at=(dom_i, dom_i + 1))
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -298,12 +314,9 @@ def main_gpu(args, rank, local_rank, world):
     st = sq.sq_device_status()
     if st != 0:
         raise RuntimeError(f"device status {sq.sq_status_string(st)} after the timed steps")
-
-    stage_ms = {n: 0.0 for n in names}
-    for e in evs:
-        for j, n in enumerate(names):
-            stage_ms[n] += e[j].elapsed_time(e[j + 1])
-    stage_ms = {n: v / args.steps for n, v in stage_ms.items()}
+    # the dominant stage's own time, live in the timed region
+    stage_ms_breakdown = dict(stage_ms)
+    stage_ms[names[dom_i]] = sum(e[dom_i].elapsed_time(e[dom_i + 1]) for e in evs) / args.steps
 
     t_max = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -358,14 +371,14 @@ def main_gpu(args, rank, local_rank, world):
     for n in names:
         ms = stage_ms[n]
         wk = work[n]
-        ent = {"ms": ms, "launches": LAUNCHES[n]}
+        ent = {"ms": ms, "launches": LAUNCHES[n], "timed": "live" if n == names[dom_i] else "breakdown pass"}
         if wk["bound"] == "tensor":
             ent["tops"] = wk["ops"] / (ms * 1e-3) / 1e12
             ent["frac_of_int8_peak"] = ent["tops"] / int8_peak
         ent["gbs"] = wk["bytes"] / (ms * 1e-3) / 1e9
         ent["frac_of_hbm"] = ent["gbs"] / hbm
         stages[n] = ent
-    dom = max(names, key=lambda n: stage_ms[n])
+    dom = names[dom_i]
     kern, srcfile = KERNEL_OF[dom]
     if work[dom]["bound"] == "tensor":
         roof = {"bound": "tensor", "achieved": stages[dom]["tops"], "peak": int8_peak, "unit": "TOPS",
@@ -404,6 +417,9 @@ def main_gpu(args, rank, local_rank, world):
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"],
                    "samples": clk["samples"]},
         "stages": stages,
+        "stages_note": (f"the dominant stage is timed in the timed steps with events around it only; the others come "
+                        f"from a separate pass of {nb} steps with an event at every stage boundary (those events "
+                        f"add ~20 us per step, so they stay out of the timed steps)"),
         "gemm_tops": stages["gemm"]["tops"],
         "gemm_frac_of_int8_peak": stages["gemm"]["frac_of_int8_peak"],
         "quant_kernel_gbs": stages["act_quant"]["gbs"],

@@ -90,6 +90,17 @@ static __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     return pol;
 }
 
+// ---------------------------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: every libsq kernel is launched so that it may start while the
+// kernel before it in the stream is finishing. pdl_wait() returns once every earlier grid of the
+// stream has completed and its memory is visible; a kernel touches no global memory it shares with
+// earlier work before it (only shared memory, tensor memory and its parameters). pdl_trigger() lets
+// the next kernel of the stream start; every libsq grid fits in one wave (all its CTAs resident at
+// once), so the next kernel's CTAs never hold SMs this grid still needs. Both are no-ops when the
+// kernel was launched without the attribute.
+static __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+static __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------------------------- barriers
 static __device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

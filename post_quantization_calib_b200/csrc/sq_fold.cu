@@ -16,7 +16,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "sq_device.cuh"
 #include "sq_internal.h"
+
+using namespace sqdev;
 
 namespace {
 
@@ -31,6 +34,8 @@ __device__ __forceinline__ uint32_t scale_pair(uint32_t w, float f) {
 __global__ void __launch_bounds__(256) k_fold_rows(const uint4 *w, const uint16_t *b, int64_t K, int64_t vrow,
                                                    const float *__restrict__ fold, uint4 *w_out, uint16_t *b_out)
 {
+    pdl_wait();
+    pdl_trigger();
     for (int64_t j = blockIdx.x; j < K; j += gridDim.x) {
         const float f = __ldg(fold + j);
         const uint4 *src = w + j * vrow;
@@ -49,6 +54,8 @@ __global__ void __launch_bounds__(256) k_fold_rows(const uint4 *w, const uint16_
 
 __global__ void k_fold_w_scale(const float *ws, int64_t K, const float *__restrict__ fold, float *out)
 {
+    pdl_wait();
+    pdl_trigger();
     for (int64_t j = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; j < K;
          j += static_cast<int64_t>(gridDim.x) * blockDim.x)
         out[j] = __fmul_rn(ws[j], fold[j]);
@@ -58,6 +65,8 @@ __global__ void k_fold_w_scale(const float *ws, int64_t K, const float *__restri
 __global__ void k_fold_ln_bias(const float *__restrict__ beta, const float *__restrict__ s, int64_t K,
                                float *__restrict__ out)
 {
+    pdl_wait();
+    pdl_trigger();
     for (int64_t k = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; k < K;
          k += static_cast<int64_t>(gridDim.x) * blockDim.x)
         out[k] = __fdiv_rn(beta[k], s[k]);
@@ -82,10 +91,10 @@ sq_status sq_fold_into_prev_linear(const void *w, const void *b, int64_t K, int6
     SQ_TRY_ARCH(dev);
     if (K == 0) return SQ_OK;
     const int64_t grid = K < 8L * sq::sm_count(dev) ? K : 8L * sq::sm_count(dev);
-    k_fold_rows<<<static_cast<unsigned>(grid), 256, 0, sq::as_stream(stream)>>>(
-        static_cast<const uint4 *>(w), static_cast<const uint16_t *>(b), K, Kp / 8, fold, static_cast<uint4 *>(w_out),
-        static_cast<uint16_t *>(b_out));
-    return sq::cuda_status(cudaGetLastError(), "launch(fold_rows)");
+    return sq::cuda_status(sq::launch_pdl(k_fold_rows, dim3(static_cast<unsigned>(grid)), dim3(256), 0, sq::as_stream(stream),
+                                          nullptr, static_cast<const uint4 *>(w), static_cast<const uint16_t *>(b), K, Kp / 8,
+                                          fold, static_cast<uint4 *>(w_out), static_cast<uint16_t *>(b_out)),
+                           "launch(fold_rows)");
 }
 
 sq_status sq_fold_into_w_scale(const float *w_scale, int64_t K, const float *fold, float *w_scale_out, void *stream)
@@ -96,9 +105,9 @@ sq_status sq_fold_into_w_scale(const float *w_scale, int64_t K, const float *fol
         return fail(SQ_ERR_MISALIGNED, "sq_fold_into_w_scale: fp32 arrays must be 4-byte aligned");
     int dev = 0;
     SQ_TRY_ARCH(dev);
-    k_fold_w_scale<<<static_cast<unsigned>((K + 255) / 256 < 1024 ? (K + 255) / 256 : 1024), 256, 0, sq::as_stream(stream)>>>(
-        w_scale, K, fold, w_scale_out);
-    return sq::cuda_status(cudaGetLastError(), "launch(fold_w_scale)");
+    return sq::cuda_status(sq::launch_pdl(k_fold_w_scale, dim3(static_cast<unsigned>((K + 255) / 256 < 1024 ? (K + 255) / 256 : 1024)),
+                                          dim3(256), 0, sq::as_stream(stream), nullptr, w_scale, K, fold, w_scale_out),
+                           "launch(fold_w_scale)");
 }
 
 sq_status sq_fold_layernorm_bias(const float *beta, const float *s, int64_t K, float *beta_fold, void *stream)
@@ -109,9 +118,9 @@ sq_status sq_fold_layernorm_bias(const float *beta, const float *s, int64_t K, f
         return fail(SQ_ERR_MISALIGNED, "sq_fold_layernorm_bias: fp32 arrays must be 4-byte aligned");
     int dev = 0;
     SQ_TRY_ARCH(dev);
-    k_fold_ln_bias<<<static_cast<unsigned>((K + 255) / 256 < 1024 ? (K + 255) / 256 : 1024), 256, 0, sq::as_stream(stream)>>>(
-        beta, s, K, beta_fold);
-    return sq::cuda_status(cudaGetLastError(), "launch(fold_layernorm_bias)");
+    return sq::cuda_status(sq::launch_pdl(k_fold_ln_bias, dim3(static_cast<unsigned>((K + 255) / 256 < 1024 ? (K + 255) / 256 : 1024)),
+                                          dim3(256), 0, sq::as_stream(stream), nullptr, beta, s, K, beta_fold),
+                           "launch(fold_layernorm_bias)");
 }
 
 }  // extern "C"

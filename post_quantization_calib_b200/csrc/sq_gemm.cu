@@ -502,6 +502,9 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // dependent launch: the set-up above touched shared and tensor memory only
+    pdl_wait();
+    pdl_trigger();
 
     constexpr int KS = L::KS;
     const int k_blocks = (K + KS * BK - 1) / (KS * BK);   // slices beyond K are zero-filled by the TMA
@@ -713,6 +716,8 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     cluster_sync_all();                                 // both CTAs' barriers exist before any remote use
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();                                         // dependent launch (set-up above is on-chip only)
+    pdl_trigger();
 
     const int k_blocks = (K + BK - 1) / BK;
     const int num_tiles = m_tiles * n_tiles;
@@ -907,11 +912,12 @@ sq_status launch_single(const CUtensorMap &mA, const CUtensorMap &mB, const CUte
     const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
     if (tiles > 0x7FFFFFFF) return sq::fail(SQ_ERR_UNSUPPORTED, "sq_w8a8_linear: too many tiles");
     const int grid = static_cast<int>(tiles < sq::sm_count(dev) ? tiles : sq::sm_count(dev));
-    k_w8a8_linear<TN, SWAP, F8><<<grid, THREADS, L::SMEM_TOTAL, sq::as_stream(stream)>>>(
-        mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out,
-        static_cast<__nv_bfloat16 *>(y), static_cast<int>(T), static_cast<int>(N), static_cast<int>(K), m_tiles, n_tiles,
-        sq::wait_timeout_ns(dev));
-    return sq::cuda_status(cudaGetLastError(), "launch(w8a8_linear)");
+    return sq::cuda_status(
+        sq::launch_pdl(k_w8a8_linear<TN, SWAP, F8>, dim3(grid), dim3(THREADS), L::SMEM_TOTAL, sq::as_stream(stream), nullptr,
+                       mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out,
+                       static_cast<__nv_bfloat16 *>(y), static_cast<int>(T), static_cast<int>(N), static_cast<int>(K), m_tiles,
+                       n_tiles, sq::wait_timeout_ns(dev)),
+        "launch(w8a8_linear)");
 }
 
 template <bool F8>
@@ -990,11 +996,11 @@ sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const voi
         const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
         if (tiles > 0x7FFFFFFF) return fail(SQ_ERR_UNSUPPORTED, "%s: too many tiles", fn);
         const int clusters = static_cast<int>(tiles < pclusters[dev] ? tiles : pclusters[dev]);
-        cfg.gridDim = dim3(2 * clusters, 1, 1);
         return sq::cuda_status(
-            cudaLaunchKernelEx(&cfg, k_w8a8_linear_pair, mA, mB, mY, x_scale, w_scale,
-                               reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out, static_cast<int>(T), static_cast<int>(N),
-                               static_cast<int>(K), m_tiles, n_tiles, sq::wait_timeout_ns(dev)),
+            sq::launch_pdl(k_w8a8_linear_pair, dim3(2 * clusters), dim3(THREADS), P_SMEM_TOTAL, sq::as_stream(stream), &attr[0],
+                           mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out,
+                           static_cast<int>(T), static_cast<int>(N), static_cast<int>(K), m_tiles, n_tiles,
+                           sq::wait_timeout_ns(dev)),
             "launch(w8a8_linear_pair)");
     }
 

@@ -92,6 +92,8 @@ struct RowArgs {
     unsigned int *status;   // device status word
     uint64_t limit_ns;      // bound of every wait
     int stream_once;        // input larger than half the L2: its lines are evicted first
+    int early;              // ABSMAX modes launched right after this library's zero-fill of amax: the
+                            // rows may be read before pdl_wait(); amax is touched only after it
 };
 
 // 1 / sqrt(ss / K + eps) with each step rounded as the RMSNorm definition orders it. When K is a
@@ -313,6 +315,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
         for (int g = 0; g < G; ++g) s_abort[g] = 0;
         mbar_init_fence();
     }
+    // Dependent launch: everything above touched shared memory only. After the library's own
+    // zero-fill (early) every earlier grid is already complete, so the rows can stream at once and
+    // only amax waits for the fill (below).
+    if (!(ABS && p.early)) pdl_wait();
+    pdl_trigger();
     if (MODE != MODE_ABSMAX && has_vec) {
         const float4 *cv = reinterpret_cast<const float4 *>(p.vec);
         for (int v = tid; v < nvec; v += kThreads) { c_lo[v] = __ldg(cv + 2 * v); c_hi[v] = __ldg(cv + 2 * v + 1); }
@@ -668,6 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
         }
         cg::cluster_group cluster = cg::this_cluster();
         cluster.sync();
+        if (p.early) pdl_wait();                           // the zero-fill of amax is complete
         const int csize = static_cast<int>(cluster.num_blocks());
         const int share = (K + csize - 1) / csize;
         const int c0 = static_cast<int>(cluster.block_rank()) * share;
@@ -683,6 +691,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
 }
 
 __global__ void k_fill_zero(float *__restrict__ p, int64_t n) {
+    pdl_wait();          // earlier grids complete before the next kernel may start (it reads early)
+    pdl_trigger();
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x)
         p[i] = 0.0f;
@@ -696,6 +706,8 @@ __global__ void k_static_scale(const float *__restrict__ amax, const float *__re
                                float *__restrict__ scale2)
 {
     __shared__ float s_w[32];
+    pdl_wait();
+    pdl_trigger();
     float m = 0.0f;
     for (int64_t k = threadIdx.x; k < K; k += blockDim.x) {
         const float a = __ldg(amax + k);
@@ -720,6 +732,8 @@ __global__ void k_scales(const float *__restrict__ ax, const float *__restrict__
                          double ea, double eb, const float *__restrict__ gamma,
                          float *__restrict__ s, float *__restrict__ fold)
 {
+    pdl_wait();
+    pdl_trigger();
     const int64_t j = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
     if (j >= K) return;
     const double a = static_cast<double>(fmaxf(ax[j], kFloor));
@@ -827,8 +841,8 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
     if (!ABS) {
         int64_t ctas = (units + G - 1) / G;
         if (ctas > full) ctas = full;
-        kern<<<static_cast<unsigned>(ctas), kThreads, smem, st>>>(a);
-        return sq::cuda_status(cudaGetLastError(), "launch(rowquant)");
+        return sq::cuda_status(sq::launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), smem, st, nullptr, a),
+                               "launch(rowquant)");
     }
     // one wave of resident clusters at most, at least ~4 units per group
     const int csz = cluster_size[dev];
@@ -836,8 +850,8 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
     if (ctas > cluster_ctas[dev]) ctas = cluster_ctas[dev];
     ctas = ((ctas + csz - 1) / csz) * csz;
     attr[0].val.clusterDim.x = csz;
-    cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
-    return sq::cuda_status(cudaLaunchKernelEx(&cfg, kern, a), "launch(absmax)");
+    return sq::cuda_status(sq::launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), smem, st, &attr[0], a),
+                           "launch(absmax)");
 }
 
 template <int MODE, bool NORM, bool FULL>
@@ -884,8 +898,9 @@ sq_status sq_calibrate_absmax(const void *a, int64_t rows, int64_t cols, int64_t
     SQ_TRY_ARCH(dev);
     cudaStream_t st = sq::as_stream(stream);
     if (!accumulate) {
-        k_fill_zero<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(amax, cols);
-        sq_status s0 = sq::cuda_status(cudaGetLastError(), "launch(fill)");
+        sq_status s0 = sq::cuda_status(
+            sq::launch_pdl(k_fill_zero, dim3(static_cast<unsigned>((cols + 255) / 256)), dim3(256), 0, st, nullptr, amax, cols),
+            "launch(fill)");
         if (s0 != SQ_OK) return s0;
     }
     if (rows == 0) return SQ_OK;
@@ -897,6 +912,7 @@ sq_status sq_calibrate_absmax(const void *a, int64_t rows, int64_t cols, int64_t
     ra.vec = norm_gamma;
     ra.eps = eps;
     ra.amax = amax;
+    ra.early = accumulate ? 0 : 1;   // the zero-fill above was the stream's last kernel
     return norm_gamma ? dispatch_rows<MODE_ABSMAX, true>(ra, dev, st) : dispatch_rows<MODE_ABSMAX, false>(ra, dev, st);
 }
 
@@ -924,8 +940,9 @@ sq_status sq_calibrate_absmax_layernorm(const void *a, int64_t rows, int64_t col
     SQ_TRY_ARCH(dev);
     cudaStream_t st = sq::as_stream(stream);
     if (!accumulate) {
-        k_fill_zero<<<static_cast<unsigned>((cols + 255) / 256), 256, 0, st>>>(amax, cols);
-        sq_status s0 = sq::cuda_status(cudaGetLastError(), "launch(fill)");
+        sq_status s0 = sq::cuda_status(
+            sq::launch_pdl(k_fill_zero, dim3(static_cast<unsigned>((cols + 255) / 256)), dim3(256), 0, st, nullptr, amax, cols),
+            "launch(fill)");
         if (s0 != SQ_OK) return s0;
     }
     if (rows == 0) return SQ_OK;
@@ -938,6 +955,7 @@ sq_status sq_calibrate_absmax_layernorm(const void *a, int64_t rows, int64_t col
     ra.vec2 = beta;
     ra.eps = eps;
     ra.amax = amax;
+    ra.early = accumulate ? 0 : 1;   // the zero-fill above was the stream's last kernel
     return dispatch_rows<MODE_ALN, true>(ra, dev, st);
 }
 
@@ -983,8 +1001,9 @@ sq_status sq_compute_scales(const float *amax_x, const float *amax_w, int64_t K,
     SQ_TRY_ARCH(dev);
     const double ea = static_cast<double>(alpha);
     const double eb = 1.0 - static_cast<double>(alpha);
-    k_scales<<<static_cast<unsigned>((K + 255) / 256), 256, 0, sq::as_stream(stream)>>>(amax_x, amax_w, K, ea, eb, gamma, s, fold);
-    return sq::cuda_status(cudaGetLastError(), "launch(scales)");
+    return sq::cuda_status(sq::launch_pdl(k_scales, dim3(static_cast<unsigned>((K + 255) / 256)), dim3(256), 0,
+                                          sq::as_stream(stream), nullptr, amax_x, amax_w, K, ea, eb, gamma, s, fold),
+                           "launch(scales)");
 }
 
 sq_status sq_smooth_quantize_weight(const void *w, int64_t N, int64_t K, const float *s,
@@ -1102,8 +1121,9 @@ sq_status sq_static_scale(const float *amax, const float *factor, int64_t K, flo
         return fail(SQ_ERR_MISALIGNED, "sq_static_scale: fp32 arrays must be 4-byte aligned");
     int dev = 0;
     SQ_TRY_ARCH(dev);
-    k_static_scale<<<1, 1024, 0, sq::as_stream(stream)>>>(amax, factor, K, scale2);
-    return sq::cuda_status(cudaGetLastError(), "launch(static_scale)");
+    return sq::cuda_status(
+        sq::launch_pdl(k_static_scale, dim3(1), dim3(1024), 0, sq::as_stream(stream), nullptr, amax, factor, K, scale2),
+        "launch(static_scale)");
 }
 
 sq_status sq_rmsnorm_smooth_quant_static(const void *x, int64_t T, int64_t K, const float *fold, float eps,
