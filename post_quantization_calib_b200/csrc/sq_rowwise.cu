@@ -282,6 +282,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
     __shared__ double s_ss2[LN ? 2 : 1][kWarps][LN ? R : 1];   // LayerNorm: the centred sums of squares
     __shared__ float s_mx[2][kWarps][R];
     __shared__ int s_abort[G];
+    // Column abs-max over multi-warp groups: the last warp of a group to finish reading a slot refills it
+    // (s_done counts the group's warps per slot; s_issued counts the group's issued units).
+    constexpr bool LAST_REFILLS = ABS && WPR > 1;
+    __shared__ int s_done[LAST_REFILLS ? G * kMaxStages : 1];
+    __shared__ int s_issued[G];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int group = warp / WPR;
@@ -312,7 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
 
     if (tid == 0) {
         for (int i = 0; i < G * stages; ++i) mbar_init(smem_u32(&s_full[i]), 1);
-        for (int g = 0; g < G; ++g) s_abort[g] = 0;
+        for (int g = 0; g < G; ++g) { s_abort[g] = 0; s_issued[g] = 0; }
+        for (int i = 0; i < (LAST_REFILLS ? G * kMaxStages : 1); ++i) s_done[i] = 0;
         mbar_init_fence();
     }
     // Dependent launch: everything above touched shared memory only. After the library's own
@@ -362,6 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
     if (leader) {
         issued = nunits < stages ? nunits : stages;
         for (int64_t j = 0; j < issued; ++j) issue(j, static_cast<int>(j));
+        if (LAST_REFILLS) atomicMax(&s_issued[group], static_cast<int>(issued));
     }
     // Leader only, after the group's last read of slot st (unit j): refill it with unit j + stages.
     auto refill = [&](int64_t j, int st) {
@@ -369,6 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
             fence_proxy_async_smem();
             issue(j + stages, st);
             issued = j + stages + 1;
+            if (LAST_REFILLS) atomicMax(&s_issued[group], static_cast<int>(issued));
         }
     };
     {
@@ -412,8 +420,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
             }
             if (WPR > 1) {
                 // Group step, the one barrier of the unit for abs-max: partial sums become visible,
-                // failures propagate, and every warp of the group is past its reads of this slot
-                // (quantiser: the unit is in registers) and of the previous unit's slot (abs-max).
+                // failures propagate, and (quantiser) every warp holds the unit in registers, so its
+                // slot can be refilled. The abs-max re-reads the slot; its last warp refills it.
                 if (NORM) {
                     const double part = rows_sum<R>(ssr, lane);   // row lane / SUB, this warp's columns
                     if (lane % SUB == 0) s_ss[j & 1][warp][lane / SUB] = part;
@@ -422,10 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                     if (leader) { if (!*abort_flag) failed = true; *abort_flag = 1; }
                     break;
                 }
-                if (leader) {
-                    if (!ABS) refill(j, st);
-                    else if (j > 0) refill(j - 1, st == 0 ? stages - 1 : st - 1);
-                }
+                if (leader && !ABS) refill(j, st);      // the unit is in registers: its slot is free
             } else if (!ABS) {
                 __syncwarp();                                   // the unit is in registers now
                 if (leader) refill(j, st);
@@ -527,10 +532,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                         }
                     }
                 }
-                // a single warp is done with the slot; a wider group refills it at its next step
+                // this warp is done with the slot: a single warp refills it; in a wider group the last of
+                // its warps to get here does (the count orders every warp's reads before the copy)
+                __syncwarp();
                 if (WPR == 1) {
-                    __syncwarp();
                     if (leader) refill(j, st);
+                } else if (lane == 0) {
+                    if (atomicAdd(&s_done[group * kMaxStages + st], 1) == WPR - 1) {
+                        s_done[group * kMaxStages + st] = 0;
+                        refill(j, st);
+                    }
                 }
             } else if (MODE == MODE_QSTATIC) {
                 // ---- one pass: y = (x * inv_rms) * c (or x * c, or x), coded with the static scale
@@ -642,6 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
     if (failed) atomicCAS(p.status, 0u, static_cast<unsigned int>(SQ_ERR_TIMEOUT));
     // Copies issued but never consumed (only after a failed wait) must land before the CTA exits.
     if (leader) {
+        if (LAST_REFILLS) issued = s_issued[group];   // refills of the group's other warps included
         for (int64_t j = consumed; j < issued; ++j)
             if (!mbar_wait(full_bar(static_cast<int>(j % stages)), static_cast<uint32_t>((j / stages) & 1), p.limit_ns, nullptr))
                 atomicCAS(p.status, 0u, static_cast<unsigned int>(SQ_ERR_TIMEOUT));
