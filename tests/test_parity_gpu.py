@@ -445,6 +445,48 @@ def test_layernorm_fold_path(sq, orc, T, K, bias):
     ok_status(sq)
 
 
+# Dependent launch: every libsq kernel may start while the previous kernel of the stream finishes, and
+# the calibration abs-max reads its rows before its own wait (after the library's zero-fill). Inputs
+# written by a long torch kernel immediately before each call (same stream, no synchronisation) must
+# be seen complete: results equal those of the same calls on inputs written long before.
+def test_inputs_written_just_before_each_call(sq, orc):
+    dev = "cuda"
+    w = synth.WORKLOADS[1]
+    d = synth.group_inputs(w, 0, dev, T=2048)
+    gamma, W, X = d["gamma"], d["weight"], d["x"]
+    calib = torch.cat(list(synth.calibration_chunks(w, d["channels"], dev)))[:16384]
+    ref_amax = sq.sq_calibrate_absmax(calib, norm_gamma=gamma)
+    ref_aw = sq.sq_calibrate_absmax(W)
+    ref_s, ref_fold = sq.sq_compute_scales(ref_amax, ref_aw, 0.5, gamma=gamma)
+    ref_wq, ref_ws = sq.sq_smooth_quantize_weight(W, ref_s)
+    ref_xq, ref_xs = sq.sq_rmsnorm_smooth_quant(X, ref_fold)
+    ref_y = sq.sq_w8a8_linear(ref_xq, ref_xs, ref_wq, ref_ws)
+    torch.cuda.synchronize()
+    big = torch.empty(256 * 1024 * 1024 // 2, dtype=torch.bfloat16, device=dev)   # 256 MB: a kernel of ~100 us
+    for trial in range(3):
+        c2, W2, X2 = torch.empty_like(calib), torch.empty_like(W), torch.empty_like(X)
+        torch.cuda.synchronize()
+        big.fill_(trial)                      # keeps the stream busy, then the input is written last
+        c2.copy_(calib)
+        amax = sq.sq_calibrate_absmax(c2, norm_gamma=gamma)
+        big.fill_(trial + 1)
+        W2.copy_(W)
+        aw = sq.sq_calibrate_absmax(W2)
+        s, fold = sq.sq_compute_scales(amax, aw, 0.5, gamma=gamma)
+        wq, ws = sq.sq_smooth_quantize_weight(W2, s)
+        big.fill_(trial + 2)
+        X2.copy_(X)
+        xq, xs = sq.sq_rmsnorm_smooth_quant(X2, fold)
+        y = sq.sq_w8a8_linear(xq, xs, wq, ws)
+        ok_status(sq)
+        assert torch.equal(amax, ref_amax) and torch.equal(aw, ref_aw)
+        assert torch.equal(s, ref_s) and torch.equal(fold, ref_fold)
+        assert torch.equal(wq, ref_wq) and torch.equal(ws, ref_ws)
+        assert torch.equal(xq, ref_xq) and torch.equal(xs, ref_xs) and torch.equal(y, ref_y)
+    # and the reference chain itself against the oracle on its calibration maximum
+    assert np.array_equal(hnp(ref_amax), orc.calibrate_absmax(h16(calib), norm_gamma=hnp(gamma), eps=1e-6))
+
+
 def test_deterministic_bytes(sq):
     w = synth.WORKLOADS[1]
     d = synth.group_inputs(w, 0, "cuda", T=1000)
