@@ -5,9 +5,11 @@
  *   offline  per-input-channel abs-maxima of calibration activations and of the weight,
  *            smoothing factors s_j = max|X_j|^alpha / max|W_j|^(1-alpha), the smoothed weight
  *            diag(s) * W quantised to INT8 with one scale per output channel;
- *   online   1/s folded into the preceding RMSNorm weight, per-token dynamic symmetric INT8
- *            quantisation of the normalised activations, INT8 x INT8 -> INT32 GEMM, and a
- *            dequantisation epilogue (per-token scale x per-channel scale, plus bias) to bf16.
+ *   online   1/s folded into the preceding RMSNorm weight (or a LayerNorm's gamma and beta, or
+ *            the previous linear layer), per-token dynamic symmetric INT8 quantisation of the
+ *            normalised activations (or one static per-tensor scale), INT8 x INT8 -> INT32 GEMM, and
+ *            a dequantisation epilogue (per-token scale x per-channel scale, plus bias) to bf16;
+ *            the same path in FP8 E4M3.
  *
  * Pages cited (title, then section / equation / figure):
  *   [MIGRATE] "06 -- SmoothQuant: Migrating Difficulty from Activations to Weights"
@@ -22,14 +24,17 @@
  *     Sizes are element counts (int64_t).
  *   - `stream` is a cudaStream_t passed as `void *` (NULL = the legacy default stream). Each call
  *     enqueues its kernels on that stream and returns without synchronising; only
- *     sq_device_status() synchronises.
+ *     sq_device_status() synchronises. Kernels are launched as programmatic dependent launches:
+ *     one may be scheduled while the previous kernel of the stream is finishing, but it reads and
+ *     writes no global memory before that kernel has completed (griddepcontrol.wait), so stream
+ *     order holds for every input and output, whoever wrote them.
  *   - Outputs must not alias inputs.
  *   - Arguments are validated before anything is launched; a failed check returns its code and
  *     launches nothing. sq_last_error() then gives a one-line reason (per host thread).
  *   - Arithmetic: binary32 with every operation separately rounded (no contraction into fused
- *     multiply-adds), except the RMSNorm sum of squares (binary64) and the smoothing-factor power
- *     (binary64, rounded once to binary32). INT8 codes use round-half-away-from-zero and are
- *     clamped to [-127, 127].
+ *     multiply-adds), except the norm sums (binary64: the RMSNorm sum of squares, the LayerNorm sum
+ *     and centred sum of squares) and the smoothing-factor power (binary64, rounded once to
+ *     binary32). INT8 codes use round-half-away-from-zero and are clamped to [-127, 127].
  */
 #ifndef SQ_H
 #define SQ_H

@@ -19,8 +19,14 @@
 //     of one tile overlaps the main loop of the next;
 //   * warps 2..5 read the accumulator with tcgen05.ld (each warp its own 32-lane quarter), apply
 //     y = bf16(float(acc) * (x_scale * w_scale) + bias) in binary32 with explicit rounding, stage
-//     64-column boxes in swizzled shared memory and write them with TMA stores (the TMA clips rows
-//     beyond T and columns beyond N).
+//     32 x 32 boxes in 64-byte-swizzled shared memory and write them with TMA stores (the TMA clips
+//     rows beyond T and columns beyond N).
+// Other forms of the same kernel: 64-channel tiles when 256-wide tiles would leave SMs idle; for at
+// most 128 tokens the decode form, where the weight is the 128-row MMA operand and the tokens the
+// narrow one; an opt-in CTA-pair form (tcgen05 cta_group::2, 256 x 256 tiles); and FP8 E4M3 operands
+// (kind::f8f6f4, binary32 accumulators) with the same epilogue. Every launch is a programmatic
+// dependent launch: barrier and tensor-memory set-up overlap the previous kernel of the stream, and
+// griddepcontrol.wait precedes the first global-memory access.
 // Every mbarrier wait is bounded by a wall-clock limit (%globaltimer). When one runs out, the
 // kernel records SQ_ERR_TIMEOUT in a device status word, every role leaves its loop, in-flight
 // copies and MMAs are waited for (again with a limit), tensor memory is released and the kernel

@@ -1,7 +1,8 @@
 // sq_rowwise.cu -- the HBM-bound steps of the smoothed W8A8 linear on sm_100a:
-//   per-input-channel abs-max (calibration activations and weights), smoothing factors with the
-//   fold into the norm weight, and the row quantisers (weights per output channel, activations per
-//   token with the RMSNorm fused in).
+//   per-input-channel abs-max (calibration activations and weights, optionally of their RMSNorm or
+//   LayerNorm output), smoothing factors with the fold into the norm weight, the static per-tensor
+//   scale, and the row quantisers (weights per output channel, activations per token with the RMSNorm
+//   or LayerNorm fused in; INT8, INT8 with a static scale, or FP8 E4M3).
 //
 // Pages cited (title, then section / equation / figure):
 //   [MIGRATE] "06 -- SmoothQuant: Migrating Difficulty from Activations to Weights"
@@ -9,15 +10,22 @@
 //   [W8A8]    "SmoothQuant and W8A8: Quantizing Activations Too"
 //   [WOVS]    "SmoothQuant: Weight-Only vs W8A8"
 //
-// Design (B200). One kernel template serves the abs-max (MODE_ABSMAX) and the quantisers
-// (MODE_QUANT). A CTA (one per SM) has 16 warps, 4 per scheduler. Rows of up to 2048 elements are
+// Design (B200). One kernel template serves the abs-max and the quantisers (the MODE_* values below).
+// A CTA (one per SM) has 16 warps, 4 per scheduler. Rows of up to 2048 elements are
 // handled by a single warp each, wider rows by row groups of 2, 4 or 8 warps; narrower rows are
 // batched R at a time, so that a unit always gives a lane 8 vectors of 8 elements (64 element-rows)
 // against a fixed per-unit cost. Each row group streams its units through its own shared-memory ring
 // of 2-4 slots, filled with TMA bulk copies (one 1-D copy per row, completion on an mbarrier): as
-// soon as the group has read a slot for the last time, its leader lane issues the copies of the unit
-// that goes there next, so two or more units per group are in flight while the group computes on the
-// current one. There is no separate producer warp, so all 16 warps compute.
+// soon as the group has read a slot for the last time, a lane issues the copies of the unit that goes
+// there next (the leader once the quantiser holds the unit in registers; for the abs-max, which
+// re-reads the slot, the last warp of the group to finish with it), so two or more units per group
+// are in flight while the group computes on the current one. There is no separate producer warp, so
+// all 16 warps compute. A column abs-max over few rows uses four-warp groups instead of two.
+//
+// Every kernel is launched as a dependent launch: it sets up shared memory, then waits
+// (griddepcontrol.wait) for the previous kernel of the stream before it reads global memory. The
+// abs-max that follows this library's own zero-fill of amax streams its rows at once and waits only
+// before its atomics: the fill itself waited for all earlier work before it let the abs-max start.
 //
 // Per unit, sums and maxima of the R rows are reduced across the warp with one butterfly that
 // halves the number of values at each exchange, so a lane ends up with the total of one row; the
