@@ -487,6 +487,45 @@ def test_inputs_written_just_before_each_call(sq, orc):
     assert np.array_equal(hnp(ref_amax), orc.calibrate_absmax(h16(calib), norm_gamma=hnp(gamma), eps=1e-6))
 
 
+# The online path captured in a CUDA graph (its launches carry the dependent-launch attribute) replays
+# to the same bits as eager calls, for new input values copied into the captured buffers.
+def test_online_path_in_cuda_graph(sq):
+    dev = "cuda"
+    w = synth.WORKLOADS[1]
+    d = synth.group_inputs(w, 0, dev, T=1024)
+    gamma, W, X = d["gamma"], d["weight"], d["x"]
+    s, fold = sq.sq_compute_scales(sq.sq_calibrate_absmax(X, norm_gamma=gamma), sq.sq_calibrate_absmax(W), 0.5,
+                                   gamma=gamma)
+    wq, ws = sq.sq_smooth_quantize_weight(W, s)
+    xin = X.clone()
+    xq = torch.empty(X.shape, dtype=torch.int8, device=dev)
+    xs = torch.empty(X.shape[0], dtype=torch.float32, device=dev)
+    y = torch.empty(X.shape[0], W.shape[0], dtype=torch.bfloat16, device=dev)
+
+    def online():
+        sq.sq_rmsnorm_smooth_quant(xin, fold, xq=xq, x_scale=xs)
+        sq.sq_w8a8_linear(xq, xs, wq, ws, y=y)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        online()                                   # warm-up: one-time launch configuration
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        online()
+    for k in range(3):
+        xnew = (X.float() * (1.0 + 0.25 * k) + 0.01 * k).to(torch.bfloat16)
+        xin.copy_(xnew)
+        graph.replay()
+        torch.cuda.synchronize()
+        y_graph = y.clone()
+        xq_e, xs_e = sq.sq_rmsnorm_smooth_quant(xnew, fold)
+        y_e = sq.sq_w8a8_linear(xq_e, xs_e, wq, ws)
+        ok_status(sq)
+        assert torch.equal(xq, xq_e) and torch.equal(xs, xs_e) and torch.equal(y_graph, y_e)
+
+
 def test_deterministic_bytes(sq):
     w = synth.WORKLOADS[1]
     d = synth.group_inputs(w, 0, "cuda", T=1000)
