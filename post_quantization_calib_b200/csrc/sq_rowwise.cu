@@ -799,6 +799,12 @@ template <int WPR, int VPL, int R, int MODE, bool NORM, bool FULL>
 sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
     auto kern = k_rows<WPR, VPL, R, MODE, NORM, FULL>;
     constexpr int G = kWarps / WPR;
+    // The kernel's lanes cover exactly WPR * 32 * VPL vectors of a row (FULL: no per-vector bounds
+    // checks), R rows per unit: the geometry must be the one it was compiled for.
+    const int nvec = a.K / 8;
+    if (geo.wpr != WPR || geo.vpl != VPL || geo.rpu != R || geo.groups != G || nvec > WPR * 32 * VPL ||
+        (FULL && nvec != WPR * 32 * VPL))
+        return sq::fail(SQ_ERR_UNSUPPORTED, "row kernel geometry mismatch (K=%d)", a.K);
     constexpr bool ABS = MODE == MODE_ABSMAX || MODE == MODE_ALN;   // column abs-max: cluster launch
     static size_t configured_smem[64];
     static int per_sm[64];
