@@ -526,6 +526,83 @@ def test_online_path_in_cuda_graph(sq):
         assert torch.equal(xq, xq_e) and torch.equal(xs, xs_e) and torch.equal(y_graph, y_e)
 
 
+# The variant rows at the query-projection size (T 8192, K = N 4096, the calibration set of 65536 rows), in
+# the launch configuration the bench uses for the INT8 path: every code and scale compared with the
+# oracle; the GEMMs on sampled full rows and full columns (INT8: bit-exact; FP8: binary32 summation bound,
+# epilogue bit-exact).
+def test_variants_at_query_projection_size(sq, orc):
+    dev = "cuda"
+    w = synth.WORKLOADS[1]
+    d = synth.group_inputs(w, 0, dev)
+    gamma, W, X = d["gamma"], d["weight"], d["x"]
+    T, K, N = X.shape[0], X.shape[1], W.shape[0]
+    chunks = list(synth.calibration_chunks(w, d["channels"], dev))
+    rows = sample_indices(T, 24, 91)
+    cols = sample_indices(N, 24, 92)
+    amax = torch.empty(K, dtype=torch.float32, device=dev)
+    for i, c in enumerate(chunks):
+        sq.sq_calibrate_absmax(c, norm_gamma=gamma, eps=w.eps, amax=amax, accumulate=i > 0)
+    s, fold = sq.sq_compute_scales(amax, sq.sq_calibrate_absmax(W), 0.5, gamma=gamma)
+    s_h, fold_h = hnp(s), hnp(fold)
+    x16 = h16(X)
+    # f2: static per-tensor scale
+    amax_y = torch.empty(K, dtype=torch.float32, device=dev)
+    for i, c in enumerate(chunks):
+        sq.sq_calibrate_absmax(c, norm_gamma=fold, eps=w.eps, amax=amax_y, accumulate=i > 0)
+    s2 = sq.sq_static_scale(amax_y)
+    assert np.array_equal(hnp(s2), orc.static_scale(hnp(amax_y)))
+    xq, xs = sq.sq_rmsnorm_smooth_quant_static(X, fold, s2, eps=w.eps)
+    xq_o, xs_o = orc.rmsnorm_smooth_quant_static(x16, fold_h, hnp(s2), eps=w.eps)
+    assert np.array_equal(hnp(xq), xq_o) and np.array_equal(hnp(xs), xs_o)
+    wq, ws = sq.sq_smooth_quantize_weight(W, s)
+    acc = torch.empty(T, N, dtype=torch.int32, device=dev)
+    y = sq.sq_w8a8_linear(xq, xs, wq, ws, acc_out=acc)
+    check_linear(sq, orc, xq, xs, wq, ws, None, y, acc, rows=rows, cols=None)
+    check_linear(sq, orc, xq, xs, wq, ws, None, y, acc, rows=None, cols=cols)
+    # f3: FP8 E4M3
+    wq8, ws8 = sq.sq_smooth_quantize_weight_fp8(W, s)
+    wq8_o, ws8_o = orc.smooth_quantize_weight_f8(h16(W), s_h)
+    assert np.array_equal(hnp(wq8), wq8_o) and np.array_equal(hnp(ws8), ws8_o)
+    xq8, xs8 = sq.sq_rmsnorm_smooth_quant_fp8(X, fold, eps=w.eps)
+    xq8_o, xs8_o = orc.rmsnorm_smooth_quant_f8(x16, fold_h, eps=w.eps)
+    assert np.array_equal(hnp(xq8), xq8_o) and np.array_equal(hnp(xs8), xs8_o)
+    accf = torch.empty(T, N, dtype=torch.float32, device=dev)
+    y8 = sq.sq_w8a8_linear_fp8(xq8, xs8, wq8, ws8, acc_out=accf)
+    ok_status(sq)
+    table = orc.e4m3_decode(np.arange(256, dtype=np.uint8)).astype(np.float64)
+    for rr, cc in ((rows, None), (None, cols)):
+        exact = orc.gemm_f8(hnp(xq8), hnp(wq8), rr, cc)
+        xa = np.abs(table[hnp(xq8)[rr] if rr is not None else hnp(xq8)])
+        wa = np.abs(table[hnp(wq8)[cc] if cc is not None else hnp(wq8)])
+        mag = xa @ wa.T
+        a_g = hnp(accf)
+        a_g = a_g[rr] if rr is not None else a_g[:, cc]
+        assert np.all(np.abs(a_g.astype(np.float64) - exact) <= K * 2.0 ** -24 * mag + 1e-30)
+        y_g = h16(y8)
+        y_g = y_g[rr] if rr is not None else y_g[:, cc]
+        assert np.array_equal(y_g, orc.dequant_f32(np.ascontiguousarray(a_g), hnp(xs8), hnp(ws8), None, rr, cc))
+    # f4 (b): LayerNorm fold (gamma reused as the LayerNorm scale, a seeded beta)
+    beta = (0.05 * torch.randn(K, generator=torch.Generator(device="cpu").manual_seed(93))).to(dev)
+    amax_ln = torch.empty(K, dtype=torch.float32, device=dev)
+    amax_ln_o = np.zeros(K, np.float32)
+    for i, c in enumerate(chunks):
+        sq.sq_calibrate_absmax_layernorm(c, gamma, beta, amax=amax_ln, accumulate=i > 0)
+        orc.calibrate_absmax_layernorm(h16(c), hnp(gamma), hnp(beta), amax=amax_ln_o, accumulate=i > 0)
+    ok_status(sq)
+    assert np.array_equal(hnp(amax_ln), amax_ln_o)
+    s_ln, fold_ln = sq.sq_compute_scales(amax_ln, sq.sq_calibrate_absmax(W), 0.5, gamma=gamma)
+    bf = sq.sq_fold_layernorm_bias(beta, s_ln)
+    assert np.array_equal(hnp(bf), orc.fold_layernorm_bias(hnp(beta), hnp(s_ln)))
+    xq_ln, xs_ln = sq.sq_layernorm_smooth_quant(X, fold_ln, bf)
+    xq_ln_o, xs_ln_o = orc.layernorm_smooth_quant(x16, hnp(fold_ln), hnp(bf))
+    assert np.array_equal(hnp(xq_ln), xq_ln_o) and np.array_equal(hnp(xs_ln), xs_ln_o)
+    wq_ln, ws_ln = sq.sq_smooth_quantize_weight(W, s_ln)
+    y_ln = sq.sq_w8a8_linear(xq_ln, xs_ln, wq_ln, ws_ln, acc_out=acc)
+    check_linear(sq, orc, xq_ln, xs_ln, wq_ln, ws_ln, None, y_ln, acc, rows=rows, cols=None)
+    check_linear(sq, orc, xq_ln, xs_ln, wq_ln, ws_ln, None, y_ln, acc, rows=None, cols=cols)
+    ok_status(sq)
+
+
 def test_deterministic_bytes(sq):
     w = synth.WORKLOADS[1]
     d = synth.group_inputs(w, 0, "cuda", T=1000)
