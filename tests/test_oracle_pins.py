@@ -520,6 +520,36 @@ def test_chain_error_bound_with_norm(orc):
     _chain_bound_check(orc, x, w, gamma, None, 0.5, 1e-6, True)
 
 
+def test_taming_simulation_per_tensor(orc):
+    # "Taming the Outliers: A Deep Dive into SmoothQuant for LLM Quantization", "Implementation" (the
+    # SmoothQuantLinear simulation): 128 input features, 64 outputs, 5 % of the channels scaled by 50,
+    # 100 calibration and 10 test samples, alpha 0.5, per-tensor symmetric quantisation of both the
+    # activations and the weight; the page prints the smoothed and the unsmoothed MSE against the
+    # unquantised product and states that smoothing lowers it. Restated with the oracle's quantisers:
+    # one per-tensor scale for x / s (from the test tokens' own maximum) and one for diag(s) W.
+    K, N = 128, 64
+    ch = synth.outlier_channels(K, synth.OutlierSpec(int(K * 0.05), 50.0, 50.0), 61)
+    x_cal = bf16_bits(synth.outlier_tokens(100, K, ch, 62))
+    x = bf16_bits(synth.outlier_tokens(10, K, ch, 63))
+    w = bf16_bits(synth.normal_weight(N, K, 64, std=1.0))
+    exact = bits_to_f64(x) @ bits_to_f64(w).T
+
+    def mse(s):
+        f_x = (1.0 / s).astype(np.float32) if s is not None else np.ones(K, np.float32)
+        f_w = s.astype(np.float32) if s is not None else np.ones(K, np.float32)
+        sx = orc.static_scale((orc.calibrate_absmax(x) * np.abs(f_x)).astype(np.float32))
+        sw = orc.static_scale((orc.calibrate_absmax(w) * np.abs(f_w)).astype(np.float32))
+        xq, xs = orc.rmsnorm_smooth_quant_static(x, f_x, sx, apply_norm=False)
+        wq, ws = orc.rmsnorm_smooth_quant_static(w, f_w, sw, apply_norm=False)
+        acc = orc.gemm_s8(xq, wq).astype(np.float64)
+        y = acc * xs.astype(np.float64)[:, None] * ws.astype(np.float64)[None, :]
+        return float(np.mean((y - exact) ** 2))
+
+    s, _ = orc.compute_scales(orc.calibrate_absmax(x_cal), orc.calibrate_absmax(w), 0.5)
+    base, smooth = mse(None), mse(s)
+    assert smooth < 0.5 * base, (base, smooth)
+
+
 def test_smoothing_reduces_error_on_outlier_data(orc):
     # qualitative claim of the pages ("SmoothQuant and W8A8...", One layer, measured; the MSE
     # comparison of "Taming the Outliers..."): on outlier-shaped data the smoothed W8A8 output is
