@@ -873,16 +873,18 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 sq_status get_encoder(EncodeTiledFn *out) {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
+    static std::atomic<EncodeTiledFn> fn{nullptr};
+    EncodeTiledFn f = fn.load(std::memory_order_acquire);
+    if (!f) {
         void *p = nullptr;
         cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
         cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
         if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p)
             return sq::fail(SQ_ERR_CUDA, "cuTensorMapEncodeTiled entry point not available");
-        fn = reinterpret_cast<EncodeTiledFn>(p);
+        f = reinterpret_cast<EncodeTiledFn>(p);
+        fn.store(f, std::memory_order_release);
     }
-    *out = fn;
+    *out = f;
     return SQ_OK;
 }
 
@@ -906,11 +908,11 @@ sq_status launch_single(const CUtensorMap &mA, const CUtensorMap &mB, const CUte
                         const float *w_scale, const void *bias, int32_t *acc_out, void *y, int64_t T, int64_t N, int64_t K,
                         int dev, void *stream) {
     using L = Tile<TN, SWAP>;
-    static int configured[64];
-    if (!configured[dev]) {
+    static std::atomic<int> configured[64];
+    if (!configured[dev].load(std::memory_order_acquire)) {
         cudaError_t e = cudaFuncSetAttribute(k_w8a8_linear<TN, SWAP, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_TOTAL);
         if (e != cudaSuccess) return sq::cuda_status(e, "cudaFuncSetAttribute(w8a8_linear)");
-        configured[dev] = 1;
+        configured[dev].store(1, std::memory_order_release);
     }
     const int64_t rows = SWAP ? N : T, cols = SWAP ? T : N;
     const int m_tiles = static_cast<int>((rows + BM - 1) / BM);
@@ -974,7 +976,7 @@ sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const voi
     if (st == SQ_OK) st = encode_2d(enc, &mY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, T, N * 2, OUT_COLS, OUT_ROWS, CU_TENSOR_MAP_SWIZZLE_64B, "y");
     if (st != SQ_OK) return st;
     if (pair) {
-        static int pconfigured[64], pclusters[64];
+        static std::atomic<int> pclusters[64];   // 0: not configured yet on this device
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -986,7 +988,8 @@ sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const voi
         cfg.stream = sq::as_stream(stream);
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        if (!pconfigured[dev]) {
+        int npair = pclusters[dev].load(std::memory_order_acquire);
+        if (npair == 0) {
             cudaError_t e = cudaFuncSetAttribute(k_w8a8_linear_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, P_SMEM_TOTAL);
             if (e != cudaSuccess) return sq::cuda_status(e, "cudaFuncSetAttribute(w8a8_linear_pair)");
             cfg.gridDim = dim3(2, 1, 1);
@@ -994,14 +997,14 @@ sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const voi
             e = cudaOccupancyMaxActiveClusters(&nc, k_w8a8_linear_pair, &cfg);
             if (e != cudaSuccess) return sq::cuda_status(e, "cudaOccupancyMaxActiveClusters(w8a8_linear_pair)");
             if (nc < 1) return sq::fail(SQ_ERR_CUDA, "no CTA pair of the GEMM fits on this device");
-            pclusters[dev] = nc;
-            pconfigured[dev] = 1;
+            npair = nc;
+            pclusters[dev].store(nc, std::memory_order_release);
         }
         const int m_tiles = static_cast<int>((T + 2 * BM - 1) / (2 * BM));
         const int n_tiles = static_cast<int>((N + BN - 1) / BN);
         const int64_t tiles = static_cast<int64_t>(m_tiles) * n_tiles;
         if (tiles > 0x7FFFFFFF) return fail(SQ_ERR_UNSUPPORTED, "%s: too many tiles", fn);
-        const int clusters = static_cast<int>(tiles < pclusters[dev] ? tiles : pclusters[dev]);
+        const int clusters = static_cast<int>(tiles < npair ? tiles : npair);
         return sq::cuda_status(
             sq::launch_pdl(k_w8a8_linear_pair, dim3(2 * clusters), dim3(THREADS), P_SMEM_TOTAL, sq::as_stream(stream), &attr[0],
                            mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out,
@@ -1020,14 +1023,16 @@ sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const voi
 namespace sq {
 
 unsigned int *device_status_word(int device) {
-    static unsigned int *addr[64];
+    static std::atomic<unsigned int *> addr[64];
     if (device < 0 || device >= 64) return nullptr;
-    if (!addr[device]) {
+    unsigned int *a = addr[device].load(std::memory_order_acquire);
+    if (!a) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_sq_status) != cudaSuccess) return nullptr;
-        addr[device] = static_cast<unsigned int *>(p);
+        a = static_cast<unsigned int *>(p);
+        addr[device].store(a, std::memory_order_release);
     }
-    return addr[device];
+    return a;
 }
 
 }  // namespace sq

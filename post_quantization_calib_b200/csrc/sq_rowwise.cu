@@ -58,6 +58,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "sq_device.cuh"
 #include "sq_internal.h"
 
@@ -806,10 +808,14 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
         (FULL && nvec != WPR * 32 * VPL))
         return sq::fail(SQ_ERR_UNSUPPORTED, "row kernel geometry mismatch (K=%d)", a.K);
     constexpr bool ABS = MODE == MODE_ABSMAX || MODE == MODE_ALN;   // column abs-max: cluster launch
+    // Per-device launch configuration of this instantiation, set up on first use (guarded: calls may
+    // come from several host threads).
+    static std::mutex mu;
     static size_t configured_smem[64];
     static int per_sm[64];
     static int cluster_size[64], cluster_ctas[64];
     static size_t smem_cap[64];    // opt-in maximum minus this kernel's static shared memory
+    std::unique_lock<std::mutex> lk(mu);
     if (smem_cap[dev] == 0) {
         int optin = 0;
         cudaFuncAttributes fa;
@@ -856,7 +862,9 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
         }
         configured_smem[dev] = smem;
     }
-    const int64_t full = static_cast<int64_t>(sq::sm_count(dev)) * per_sm[dev];
+    const int per_sm_d = per_sm[dev], csz = cluster_size[dev], cctas = cluster_ctas[dev];
+    lk.unlock();
+    const int64_t full = static_cast<int64_t>(sq::sm_count(dev)) * per_sm_d;
     a.stages = stages;
     a.inv_k = (a.K & (a.K - 1)) == 0 ? 1.0 / static_cast<double>(a.K) : 0.0;
     a.status = sq::device_status_word(dev);
@@ -871,9 +879,8 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
                                "launch(rowquant)");
     }
     // one wave of resident clusters at most, at least ~4 units per group
-    const int csz = cluster_size[dev];
     int64_t ctas = (units + 4 * G - 1) / (4 * G);
-    if (ctas > cluster_ctas[dev]) ctas = cluster_ctas[dev];
+    if (ctas > cctas) ctas = cctas;
     ctas = ((ctas + csz - 1) / csz) * csz;
     attr[0].val.clusterDim.x = csz;
     return sq::cuda_status(sq::launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), smem, st, &attr[0], a),

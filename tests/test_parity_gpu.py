@@ -603,6 +603,53 @@ def test_variants_at_query_projection_size(sq, orc):
     ok_status(sq)
 
 
+# Calls from several host threads at once, each on its own stream (the launch configuration caches
+# are shared between threads): every thread gets the bits the same calls give one after another.
+def test_concurrent_host_threads(sq):
+    import threading
+    dev = "cuda"
+    shapes = [(300, 1032, 2064), (129, 2056, 1040), (1000, 520, 4096), (64, 3000, 272)]
+    inputs = []
+    for i, (T, N, K) in enumerate(shapes):
+        g = torch.Generator(device="cpu").manual_seed(500 + i)
+        X = torch.randn(T, K, generator=g).to(torch.bfloat16).to(dev)
+        W = (torch.randn(N, K, generator=g) * 0.02).to(torch.bfloat16).to(dev)
+        gamma = (1 + 0.1 * torch.randn(K, generator=g)).to(dev)
+        inputs.append((X, W, gamma))
+
+    def chain(X, W, gamma, stream):
+        with torch.cuda.stream(stream):
+            s, fold = sq.sq_compute_scales(sq.sq_calibrate_absmax(X, norm_gamma=gamma), sq.sq_calibrate_absmax(W), 0.5,
+                                           gamma=gamma)
+            wq, ws = sq.sq_smooth_quantize_weight(W, s)
+            xq, xs = sq.sq_rmsnorm_smooth_quant(X, fold)
+            return sq.sq_w8a8_linear(xq, xs, wq, ws)
+
+    ref = [chain(*inp, torch.cuda.current_stream()) for inp in inputs]
+    torch.cuda.synchronize()
+    for _ in range(3):
+        out = [None] * len(inputs)
+        streams = [torch.cuda.Stream() for _ in inputs]
+        errors = []
+
+        def work(i):
+            try:
+                out[i] = chain(*inputs[i], streams[i])
+            except Exception as e:           # reported below, in the main thread
+                errors.append(e)
+
+        threads = [threading.Thread(target=work, args=(i,)) for i in range(len(inputs))]
+        for t in threads:
+            t.start()
+        for t in threads:
+            t.join()
+        torch.cuda.synchronize()
+        assert not errors, errors
+        ok_status(sq)
+        for a, b in zip(out, ref):
+            assert torch.equal(a, b)
+
+
 def test_deterministic_bytes(sq):
     w = synth.WORKLOADS[1]
     d = synth.group_inputs(w, 0, "cuda", T=1000)
