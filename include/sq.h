@@ -49,7 +49,7 @@ extern "C" {
 typedef enum {
     SQ_OK = 0,
     SQ_ERR_INVALID_ARG = 1,   /* null pointer, negative or inconsistent size, alpha outside [0,1] */
-    SQ_ERR_UNSUPPORTED = 2,   /* a size this build does not handle (limits stated per call) */
+    SQ_ERR_UNSUPPORTED = 2,   /* a size the library does not handle (limits stated per call) */
     SQ_ERR_MISALIGNED = 3,    /* pointer or leading dimension not aligned as required */
     SQ_ERR_ARCH = 4,          /* current device is not compute capability 10.0 (B200 class) */
     SQ_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
@@ -261,7 +261,7 @@ sq_status sq_w8a8_linear_fp8(const uint8_t *xq, const float *x_scale, int64_t T,
                              const float *w_scale, int64_t N, int64_t K, const void *bias, void *y,
                              float *acc_out, void *workspace, size_t workspace_bytes, void *stream);
 
-/* Bytes of workspace sq_w8a8_linear needs for these sizes (0 in this build). */
+/* Bytes of workspace sq_w8a8_linear needs for these sizes: always 0 (no form of the GEMM uses one). */
 size_t sq_w8a8_linear_workspace_size(int64_t T, int64_t N, int64_t K);
 
 /*

@@ -1,6 +1,6 @@
 """GPU parity: every libsq stage against the CPU oracle on the same seeded inputs (through the C ABI).
 
-Bars (fixed by the benchmark spec of the method, written here in the tests):
+Bars (the tolerances stated for the method, written here in the tests):
   * abs-maxima, INT8 codes, per-row scales and INT32 accumulators: bit-exact;
   * smoothing factors and fold: within 1e-6 relative (the device pow is not correctly rounded);
   * bf16 outputs: within 1e-2 relative of the exact dequantised value, and in practice bit-exact
