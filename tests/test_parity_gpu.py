@@ -650,6 +650,39 @@ def test_concurrent_host_threads(sq):
             assert torch.equal(a, b)
 
 
+# The decode form in a chain of calls on distinct weights, each call's tokens and scales written by a
+# torch kernel right before it on the same stream: bits equal to the same calls on inputs written
+# long before, and to the oracle.
+@pytest.mark.parametrize("T", [1, 17, 64, 128])
+def test_decode_chain_inputs_written_just_before(sq, orc, T):
+    dev = "cuda"
+    N, K, L = 2056, 4096, 4
+    g = torch.Generator(device="cpu").manual_seed(900 + T)
+    ws_ = [(torch.randint(-127, 128, (N, K), generator=g, dtype=torch.int8).to(dev), (torch.rand(N, generator=g) * 1e-2).to(dev))
+           for _ in range(L)]
+    xq_src = torch.randint(-127, 128, (T, K), generator=g, dtype=torch.int8).to(dev)
+    xs_src = (torch.rand(T, generator=g) * 1e-2).to(dev)
+    b = (torch.randn(N, generator=g) * 0.1).to(torch.bfloat16).to(dev)
+    ref = []
+    for wq, wsc in ws_:
+        acc = torch.empty(T, N, dtype=torch.int32, device=dev)
+        ref.append((sq.sq_w8a8_linear(xq_src, xs_src, wq, wsc, bias=b, acc_out=acc), acc))
+    torch.cuda.synchronize()
+    for _ in range(3):
+        got = []
+        for wq, wsc in ws_:
+            xq, xs = torch.empty_like(xq_src), torch.empty_like(xs_src)
+            xq.copy_(xq_src)
+            xs.copy_(xs_src)
+            acc = torch.empty(T, N, dtype=torch.int32, device=dev)
+            got.append((sq.sq_w8a8_linear(xq, xs, wq, wsc, bias=b, acc_out=acc), acc))
+        torch.cuda.synchronize()
+        ok_status(sq)
+        for (y, acc), (y0, acc0) in zip(got, ref):
+            assert torch.equal(acc, acc0) and torch.equal(y, y0)
+    check_linear(sq, orc, xq_src, xs_src, ws_[0][0], ws_[0][1], b, ref[0][0], ref[0][1])
+
+
 def test_deterministic_bytes(sq):
     w = synth.WORKLOADS[1]
     d = synth.group_inputs(w, 0, "cuda", T=1000)
