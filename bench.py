@@ -422,6 +422,9 @@ def main_gpu(args, rank, local_rank, world):
                         f"add ~20 us per step, so they stay out of the timed steps)"),
         "gemm_tops": stages["gemm"]["tops"],
         "gemm_frac_of_int8_peak": stages["gemm"]["frac_of_int8_peak"],
+        # the GEMM runs inside a long step: its fraction of the sustained (power-capped) reference too
+        "gemm_frac_of_int8_sustained": (stages["gemm"]["tops"] / (float(peaks["bf16_tflops_sustained"]) * INT8_PER_BF16)
+                                        if "bf16_tflops_sustained" in peaks else None),
         "quant_kernel_gbs": stages["act_quant"]["gbs"],
         "online_ms_per_step": stage_ms["act_quant"] + stage_ms["gemm"],
     }
