@@ -22,6 +22,12 @@
  *   - RMSNorm is the standard x / sqrt(mean(x^2) + eps) * gamma (the pages name RMSNorm but do not
  *     print it).
  *   - Scale floors: both abs-maxima and s itself are floored at 1e-5 (binary32 constant).
+ *   - Static per-tensor scale: the maximum of the smoothed activation over the calibration tokens,
+ *     delta = m / 127, codes clamped at +-127 (see the static-scale section below).
+ *   - FP8: the OCP E4M3 "FN" format, scale m / 448, round to nearest even with saturation at
+ *     +-448, the sign kept on zero (see the FP8 section below).
+ *   - LayerNorm (not printed on the pages): the standard per-token form, mean and centred sum of
+ *     squares in binary64, every other step rounded to binary32 (see the LayerNorm section below).
  *
  * bf16 tensors are passed as uint16_t bit patterns.
  */
