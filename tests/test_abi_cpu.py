@@ -190,3 +190,20 @@ def test_binding_rejects_host_tensors(sqmod):
         sqmod.sq_rmsnorm_smooth_quant(x, torch.ones(64))
     with pytest.raises(ValueError):
         sqmod.sq_calibrate_absmax(x)
+
+
+def test_layer_object_rejects_unsupported_combinations(sqmod):
+    from post_quantization_calib_b200.layer import SmoothedW8A8Linear
+    w = [torch.zeros(16, 64, dtype=torch.bfloat16)]
+    g = torch.ones(64)
+    with pytest.raises(ValueError):
+        SmoothedW8A8Linear(w, 0.5, gamma=g, scheme="int4")
+    with pytest.raises(ValueError):
+        SmoothedW8A8Linear(w, 0.5, gamma=g, norm="layer", scheme="fp8")        # LayerNorm: INT8 only
+    with pytest.raises(ValueError):
+        SmoothedW8A8Linear(w, 0.5, gamma=None, norm="rms")                     # a norm needs gamma
+    with pytest.raises(ValueError):
+        SmoothedW8A8Linear(w, 0.5, gamma=g, beta=g, norm="rms")                # beta is a LayerNorm's
+    layer = SmoothedW8A8Linear(w, 0.5, gamma=g, norm="layer", beta=g)
+    assert layer.eps == 1e-5 and layer.norm == "layer" and layer.wq.dtype == torch.int8
+    assert SmoothedW8A8Linear(w, 0.5, scheme="fp8").wq.dtype == torch.uint8

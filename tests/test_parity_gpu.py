@@ -683,6 +683,76 @@ def test_decode_chain_inputs_written_just_before(sq, orc, T):
     check_linear(sq, orc, xq_src, xs_src, ws_[0][0], ws_[0][1], b, ref[0][0], ref[0][1])
 
 
+# The user-facing layer object (SmoothedW8A8Linear): calibrate on batches, then forward, for every norm
+# / scheme it offers, against the oracle chain fed the layer's own s and fold (codes, scales and bf16
+# outputs bit-exact; FP8 accumulators within the binary32 summation bound).
+LAYER_CASES = [("rms", "int8"), ("rms", "int8_static"), ("rms", "fp8"), ("none", "int8"), ("none", "int8_static"),
+               ("none", "fp8"), ("layer", "int8")]
+
+
+@pytest.mark.parametrize("norm,scheme", LAYER_CASES)
+def test_layer_object(sq, orc, norm, scheme):
+    from post_quantization_calib_b200.layer import SmoothedW8A8Linear
+    dev = "cuda"
+    T, K, Ns = 300, 1040, (264, 256)
+    seed = 70 + LAYER_CASES.index((norm, scheme))
+    ch = synth.outlier_channels(K, synth.OutlierSpec(12, 10.0, 40.0), seed)
+    batches = [synth.outlier_tokens(200, K, ch, seed + 1 + i, dev) for i in range(3)]
+    x = synth.outlier_tokens(T, K, ch, seed + 9, dev)
+    ws = [synth.normal_weight(n, K, seed + 10 + i, dev) for i, n in enumerate(Ns)]
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    gamma = (1 + 0.1 * torch.randn(K, generator=g)).to(dev) if norm != "none" else None
+    beta = (0.05 * torch.randn(K, generator=g)).to(dev) if norm == "layer" else None
+    bias = synth.bias_vector(sum(Ns), seed + 20, dev)
+    layer = SmoothedW8A8Linear(ws, 0.5, gamma=gamma, beta=beta, bias=bias, norm=None if norm == "none" else norm,
+                               scheme=scheme)
+    layer.calibrate(batches)
+    N = layer.N
+    acc = torch.empty(T, N, dtype=torch.float32 if scheme == "fp8" else torch.int32, device=dev)
+    y = layer(x, acc_out=acc)
+    ok_status(sq)
+    cal = np.concatenate([h16(b) for b in batches])
+    g_h = hnp(gamma) if gamma is not None else None
+    if norm == "layer":
+        amax_o = orc.calibrate_absmax_layernorm(cal, g_h, hnp(beta), eps=layer.eps)
+    else:
+        amax_o = orc.calibrate_absmax(cal, norm_gamma=g_h, eps=layer.eps)
+    assert np.array_equal(hnp(layer.amax_x), amax_o)
+    s_o, _ = orc.compute_scales(amax_o, orc.calibrate_absmax(h16(layer.weight)), 0.5, g_h)
+    assert np.all(np.abs(hnp(layer.s).astype(np.float64) / s_o - 1) <= 1e-6)
+    s_h, f_h, x16 = hnp(layer.s), hnp(layer.fold), h16(x)
+    if scheme == "fp8":
+        wq_o, ws_o = orc.smooth_quantize_weight_f8(h16(layer.weight), s_h)
+        xq_o, xs_o = orc.rmsnorm_smooth_quant_f8(x16, f_h, eps=layer.eps, apply_norm=norm == "rms")
+    else:
+        wq_o, ws_o = orc.smooth_quantize_weight(h16(layer.weight), s_h)
+        if norm == "layer":
+            bf_o = orc.fold_layernorm_bias(hnp(beta), s_h)
+            assert np.array_equal(hnp(layer.beta_fold), bf_o)
+            xq_o, xs_o = orc.layernorm_smooth_quant(x16, f_h, bf_o, eps=layer.eps)
+        elif scheme == "int8_static":
+            if norm == "rms":
+                amax_y = orc.calibrate_absmax(cal, norm_gamma=f_h, eps=layer.eps)
+            else:
+                amax_y = (orc.calibrate_absmax(cal) * np.abs(f_h)).astype(np.float32)
+            s2_o = orc.static_scale(amax_y)
+            assert np.array_equal(hnp(layer.scale2), s2_o)
+            xq_o, xs_o = orc.rmsnorm_smooth_quant_static(x16, f_h, s2_o, eps=layer.eps, apply_norm=norm == "rms")
+        else:
+            xq_o, xs_o = orc.rmsnorm_smooth_quant(x16, f_h, eps=layer.eps, apply_norm=norm == "rms")
+    assert np.array_equal(hnp(layer.wq), wq_o) and np.array_equal(hnp(layer.w_scale), ws_o)
+    if scheme == "fp8":
+        exact = orc.gemm_f8(xq_o, wq_o)
+        table = orc.e4m3_decode(np.arange(256, dtype=np.uint8)).astype(np.float64)
+        mag = np.abs(table[xq_o]) @ np.abs(table[wq_o]).T
+        assert np.all(np.abs(hnp(acc).astype(np.float64) - exact) <= K * 2.0 ** -24 * mag + 1e-30)
+        assert np.array_equal(h16(y), orc.dequant_f32(hnp(acc), xs_o, ws_o, h16(bias)))
+    else:
+        y_o, acc_o = orc.w8a8_linear(xq_o, xs_o, wq_o, ws_o, h16(bias))
+        assert np.array_equal(hnp(acc), acc_o) and np.array_equal(h16(y), y_o)
+    assert [t.shape[1] for t in layer.split_output(y)] == list(Ns)
+
+
 def test_deterministic_bytes(sq):
     w = synth.WORKLOADS[1]
     d = synth.group_inputs(w, 0, "cuda", T=1000)
