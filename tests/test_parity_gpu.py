@@ -753,6 +753,36 @@ def test_layer_object(sq, orc, norm, scheme):
     assert [t.shape[1] for t in layer.split_output(y)] == list(Ns)
 
 
+# Layer object, input used directly: 1/s folded into the previous linear layer (bf16 weight and bias,
+# in place, bit-exact against the oracle fold); the layer then quantises with factor 1, and its output
+# on the folded previous layer's output stays within quantisation error of the unfolded path.
+def test_layer_fold_into_previous(sq, orc):
+    from post_quantization_calib_b200.layer import SmoothedW8A8Linear
+    dev = "cuda"
+    T, Kp, K, N = 256, 512, 1024, 264
+    g = torch.Generator(device="cpu").manual_seed(81)
+    w_prev = (torch.randn(K, Kp, generator=g) * 0.05).to(torch.bfloat16).to(dev)
+    b_prev = (torch.randn(K, generator=g) * 0.05).to(torch.bfloat16).to(dev)
+    x_in = torch.randn(T, Kp, generator=g).to(torch.bfloat16).to(dev)
+    W = synth.normal_weight(N, K, 82, dev)
+    h = torch.nn.functional.linear(x_in, w_prev, b_prev)          # the previous layer, run by the caller
+    layer = SmoothedW8A8Linear([W], 0.5, scheme="int8")
+    layer.calibrate([h])
+    y_unfolded = layer(h)
+    fold = layer.fold.clone()
+    w_o, b_o = orc.fold_into_prev_linear(h16(w_prev), h16(b_prev), hnp(fold))
+    layer.fold_into_previous(w_prev, b_prev)
+    assert np.array_equal(h16(w_prev), w_o) and np.array_equal(h16(b_prev), b_o)
+    assert torch.equal(layer.fold, torch.ones_like(layer.fold))
+    h2 = torch.nn.functional.linear(x_in, w_prev, b_prev)          # arrives already divided by s
+    y_folded = layer(h2)
+    ok_status(sq)
+    ref = h.double() @ W.double().t()
+    err_u = torch.linalg.vector_norm(y_unfolded.double() - ref) / torch.linalg.vector_norm(ref)
+    err_f = torch.linalg.vector_norm(y_folded.double() - ref) / torch.linalg.vector_norm(ref)
+    assert err_f < 1.5 * err_u + 1e-3, (float(err_u), float(err_f))
+
+
 def test_deterministic_bytes(sq):
     w = synth.WORKLOADS[1]
     d = synth.group_inputs(w, 0, "cuda", T=1000)
