@@ -53,7 +53,9 @@ typedef enum {
     SQ_ERR_MISALIGNED = 3,    /* pointer or leading dimension not aligned as required */
     SQ_ERR_ARCH = 4,          /* current device is not compute capability 10.0 (B200 class) */
     SQ_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
-    SQ_ERR_TIMEOUT = 6        /* a bounded device-side wait ran out (reported by sq_device_status) */
+    SQ_ERR_TIMEOUT = 6,       /* a bounded device-side wait ran out (reported by sq_device_status) */
+    SQ_ERR_BOUNDS = 7         /* checked build only: a device-side bounds check failed and its access
+                                 was skipped (reported by sq_device_status) */
 } sq_status;
 
 /* Name of a status code ("SQ_OK", ...). Never NULL. */
@@ -267,8 +269,10 @@ size_t sq_w8a8_linear_workspace_size(int64_t T, int64_t N, int64_t K);
 /*
  * Synchronises `stream`, then reports the device-side status word of the current device:
  * SQ_OK, SQ_ERR_TIMEOUT (a bounded wait in a kernel ran out; the kernel stopped its work and
- * returned, the context stays usable) or SQ_ERR_CUDA (an asynchronous CUDA error). Reading the
- * word clears it. The word is shared by every stream on the device.
+ * returned, the context stays usable), SQ_ERR_BOUNDS (libsq_checked.so only: a device-side bounds
+ * check failed and the access it guards was skipped) or SQ_ERR_CUDA (an asynchronous CUDA error).
+ * The first error recorded is kept. Reading the word clears it. The word is shared by every stream
+ * on the device.
  */
 sq_status sq_device_status(void *stream);
 
@@ -285,6 +289,15 @@ sq_status sq_set_wait_timeout_ns(uint64_t ns);
  * Used by the test suite to show that an expired wait ends in a status, not a hang.
  */
 sq_status sq_selftest_wait_timeout(void *stream);
+
+/*
+ * Self-test of the device-side bounds checks of libsq_checked.so (the library built with
+ * SQ_DEVICE_CHECKS): launches one small kernel whose store fails its check, so the kernel records
+ * SQ_ERR_BOUNDS in the status word and skips the store (the store's target lies inside the kernel's
+ * own array either way). Returns SQ_ERR_UNSUPPORTED, launching nothing, in the product libsq.so.
+ * Neither the checks nor this call has a counterpart in SmoothQuant: they are a debugging aid.
+ */
+sq_status sq_selftest_bounds_check(void *stream);
 
 #ifdef __cplusplus
 }

@@ -4,6 +4,23 @@
 
 #include <stdint.h>
 
+#include "sq.h"
+
+// Device-side bounds checks. A build with SQ_DEVICE_CHECKS defined (libsq_checked.so) evaluates
+// each SQ_CHECK(ok, status): a false `ok` records SQ_ERR_BOUNDS in the device status word (the first
+// error recorded is kept) and the caller skips the access the check guards, so a wrong index shows
+// up as a status from sq_device_status instead of a fault. In the product build SQ_CHECK is the
+// constant true and its arguments are not compiled at all.
+#ifdef SQ_DEVICE_CHECKS
+static __device__ __forceinline__ bool sq_check_record(bool ok, unsigned int *status) {
+    if (!ok) atomicCAS(status, 0u, static_cast<unsigned int>(SQ_ERR_BOUNDS));
+    return ok;
+}
+#define SQ_CHECK(ok, status) sq_check_record((ok), (status))
+#else
+#define SQ_CHECK(ok, status) true
+#endif
+
 // Every helper is `static` (internal linkage): each translation unit keeps its own copy.
 namespace sqdev {
 

@@ -129,13 +129,17 @@ __device__ __forceinline__ void give_up(volatile int *abort_flag) {
     *abort_flag = 1;
 }
 
+// The tensor maps loaded here hold 8-bit operands: the innermost coordinate c0 must be a multiple of
+// 16 elements (16 bytes). Stores write bf16: c0 a multiple of 8, and no coordinate negative.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar, int c0, int c1) {
+    if (!SQ_CHECK(c0 >= 0 && (c0 & 15) == 0, &g_sq_status)) return;
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
         : "memory");
 }
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t src, int c0, int c1) {
+    if (!SQ_CHECK(c0 >= 0 && c1 >= 0 && (c0 & 7) == 0, &g_sq_status)) return;
     asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
                      reinterpret_cast<uint64_t>(map)),
                  "r"(src), "r"(c0), "r"(c1)
@@ -217,6 +221,7 @@ __device__ __forceinline__ void cluster_sync_all() {
 // TMA load into this CTA's shared memory whose completion is counted on `bar_cluster`, a barrier of
 // either CTA of the pair (shared::cluster address).
 __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, uint32_t bar_cluster, int c0, int c1) {
+    if (!SQ_CHECK(c0 >= 0 && (c0 & 15) == 0, &g_sq_status)) return;   // 8-bit operands, as above
     asm volatile(
         "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1)
@@ -365,7 +370,7 @@ __device__ __forceinline__ void epilogue_rows(uint32_t tmem_base, int quad, int 
             int4 *dst = reinterpret_cast<int4 *>(acc_out + static_cast<int64_t>(row) * N + col0);
 #pragma unroll
             for (int g = 0; g < OUT_COLS / 4; ++g) {
-                if (col0 + 4 * g < N)
+                if (col0 + 4 * g < N && SQ_CHECK(row >= 0 && col0 + 4 * g + 4 <= N, &g_sq_status))
                     dst[g] = make_int4(static_cast<int>(cur[4 * g]), static_cast<int>(cur[4 * g + 1]),
                                        static_cast<int>(cur[4 * g + 2]), static_cast<int>(cur[4 * g + 3]));
             }
@@ -455,6 +460,7 @@ __device__ __forceinline__ void epilogue_swap(uint32_t tmem_base, int quad, int 
             if (t < T && okn) {
                 const int acc = static_cast<int>(r[j]);
                 const int64_t o = static_cast<int64_t>(t) * N + n;
+                if (!SQ_CHECK(t >= 0 && n >= 0 && o < static_cast<int64_t>(T) * N, &g_sq_status)) continue;
                 if (acc_out != nullptr) acc_out[o] = acc;
                 float v = __fmul_rn(acc_value<F8>(r[j]), __fmul_rn(__ldg(x_scale + t), ws));
                 if (bias != nullptr) v = __fadd_rn(v, b);
@@ -865,6 +871,16 @@ __global__ void k_selftest_wait(uint64_t limit_ns) {
     }
 }
 
+#ifdef SQ_DEVICE_CHECKS
+// Self-test of the bounds checks: one thread stores to index `i` of an 8-word array under a check
+// whose limit is 4. Called with i in [4, 8), the check fails, records SQ_ERR_BOUNDS and skips the
+// store; were the check missing, the store would still land inside the array.
+__device__ unsigned int g_selftest_words[8];
+__global__ void k_selftest_bounds(int i) {
+    if (threadIdx.x == 0 && i >= 0 && i < 8 && SQ_CHECK(i < 4, &g_sq_status)) g_selftest_words[i] = 1u;
+}
+#endif
+
 // ------------------------------------------------------------------------------------------------
 // Host side.
 
@@ -1092,6 +1108,18 @@ sq_status sq_selftest_wait_timeout(void *stream) {
     SQ_TRY_ARCH(dev);
     k_selftest_wait<<<1, 32, 0, sq::as_stream(stream)>>>(sq::wait_timeout_ns(dev));
     return sq::cuda_status(cudaGetLastError(), "launch(selftest_wait)");
+}
+
+sq_status sq_selftest_bounds_check(void *stream) {
+    int dev = 0;
+    SQ_TRY_ARCH(dev);
+#ifdef SQ_DEVICE_CHECKS
+    k_selftest_bounds<<<1, 32, 0, sq::as_stream(stream)>>>(5);
+    return sq::cuda_status(cudaGetLastError(), "launch(selftest_bounds)");
+#else
+    (void)stream;
+    return sq::fail(SQ_ERR_UNSUPPORTED, "sq_selftest_bounds_check: the library was built without device checks");
+#endif
 }
 
 }  // extern "C"

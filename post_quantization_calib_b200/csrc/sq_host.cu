@@ -95,6 +95,7 @@ const char *sq_status_string(int status) {
         case SQ_ERR_ARCH: return "SQ_ERR_ARCH";
         case SQ_ERR_CUDA: return "SQ_ERR_CUDA";
         case SQ_ERR_TIMEOUT: return "SQ_ERR_TIMEOUT";
+        case SQ_ERR_BOUNDS: return "SQ_ERR_BOUNDS";
         default: return "SQ_ERR_UNKNOWN";
     }
 }

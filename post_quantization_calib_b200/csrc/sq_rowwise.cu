@@ -273,6 +273,14 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
     return d;
 }
 
+// Column vector v of a row lies inside it. A FULL geometry covers the row exactly, so the bound holds
+// by construction there; the checked build verifies it.
+#ifdef SQ_DEVICE_CHECKS
+#define SQ_COL_IN(v) (FULL ? SQ_CHECK((v) < nvec, p.status) : (v) < nvec)
+#else
+#define SQ_COL_IN(v) (FULL || (v) < nvec)
+#endif
+
 // One CTA = 16 warps in row groups of WPR warps. A group processes units of R consecutive rows; lane l
 // of warp w of the group covers the 8-element vectors v = i * 32 * WPR + 32 * w + l (i < VPL) of
 // every row of the unit. R > 1 only with WPR == 1.
@@ -356,6 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
         const int ncopies = packed ? 1 : nr;
         const uint32_t bytes = packed ? rowbytes * static_cast<uint32_t>(nr) : rowbytes;
         for (int r = 0; r < ncopies; ++r) {
+            // the copy lands inside the slot and reads rows of the input only
+            if (!SQ_CHECK(st >= 0 && st < stages && r0 >= 0 && nr >= 1 && r0 + nr <= p.rows &&
+                              static_cast<uint64_t>(r) * rowbytes + bytes <= slotbytes, p.status))
+                continue;
             const uint32_t dst = smem_u32(slot(st) + r * rowbytes);
             const uint8_t *src = p.src + (r0 + r) * p.ld_bytes;
             if (p.stream_once) bulk_g2s_hint(dst, src, bytes, full_bar(st), policy);
@@ -414,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
 #pragma unroll
                 for (int i = 0; i < VPL; ++i) {
                     const int v = i * GT + gtid;
-                    const bool in = (FULL || v < nvec) && r < nr;
+                    const bool in = SQ_COL_IN(v) && r < nr;
                     if (MODE == MODE_ABSMAX && !NORM) continue;
                     const uint4 q = in ? rp[r * rv + v] : make_uint4(0u, 0u, 0u, 0u);
                     if (!ABS) xr[r][i] = q;
@@ -474,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
 #pragma unroll
                         for (int i = 0; i < VPL; ++i) {
                             const int v = i * GT + gtid;
-                            if (!((FULL || v < nvec) && r < nr)) continue;
+                            if (!(SQ_COL_IN(v) && r < nr)) continue;
                             const uint4 q = ABS ? rp[r * rv + v] : xr[r][i];
                             if (i & 1) { add_centred_squares(q.x, nm2, a2, a3); add_centred_squares(q.y, nm2, a2, a3); add_centred_squares(q.z, nm2, a2, a3); add_centred_squares(q.w, nm2, a2, a3); }
                             else { add_centred_squares(q.x, nm2, a0, a1); add_centred_squares(q.y, nm2, a0, a1); add_centred_squares(q.z, nm2, a0, a1); add_centred_squares(q.w, nm2, a0, a1); }
@@ -506,10 +518,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                 for (int i = 0; i < VPL; ++i) {
                     const int v = i * GT + gtid;
                     uint64_t g2[4], b2[4];                      // LayerNorm: gamma and beta pairs
-                    if (LN && (FULL || v < nvec)) ln_params(c_lo, c_hi, p.vec2, v, g2, b2);
+                    if (LN && SQ_COL_IN(v)) ln_params(c_lo, c_hi, p.vec2, v, g2, b2);
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
-                        if (!((FULL || v < nvec) && r < nr)) continue;
+                        if (!(SQ_COL_IN(v) && r < nr)) continue;
                         if (LN) {
                             const uint64_t ir2 = pack2(ir[r], ir[r]), nm2 = pack2(-mu[r], -mu[r]);
                             const uint4 q = rp[r * rv + v];
@@ -563,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
 #pragma unroll
                         for (int i = 0; i < VPL; ++i) {
                             const int v = i * GT + gtid;
-                            if (!(FULL || v < nvec)) continue;
+                            if (!SQ_COL_IN(v)) continue;
                             float4 cl = make_float4(1.f, 1.f, 1.f, 1.f), ch = cl;
                             if (has_vec) { cl = c_lo[v]; ch = c_hi[v]; }
                             const uint64_t c2[4] = {pack2(cl.x, cl.y), pack2(cl.z, cl.w), pack2(ch.x, ch.y), pack2(ch.z, ch.w)};
@@ -574,14 +586,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                                 const uint64_t yy = NORM ? mul2_rn(mul2_rn(x2, ir2), c2[k]) : (has_vec ? mul2_rn(x2, c2[k]) : x2);
                                 cc[k] = codes2_clamped(mul2_rn(yy, sinv2));
                             }
-                            qrow[v] = make_uint2(__byte_perm(cc[0], cc[1], 0x5410), __byte_perm(cc[2], cc[3], 0x5410));
+                            if (SQ_CHECK(r0 + r < p.rows, p.status))
+                                qrow[v] = make_uint2(__byte_perm(cc[0], cc[1], 0x5410), __byte_perm(cc[2], cc[3], 0x5410));
                         }
                     }
                 }
                 if (gtid == 0) {
 #pragma unroll
                     for (int r = 0; r < R; ++r)
-                        if (r < nr) p.scale[r0 + r] = sdelta;
+                        if (r < nr && SQ_CHECK(r0 + r < p.rows, p.status)) p.scale[r0 + r] = sdelta;
                 }
             } else {
                 // ---- pass B: y = (x * inv_rms) * c  (or x * c, or x) as element pairs, row maxima
@@ -592,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
 #pragma unroll
                 for (int i = 0; i < VPL; ++i) {
                     const int v = i * GT + gtid;
-                    const bool in = FULL || v < nvec;
+                    const bool in = SQ_COL_IN(v);
                     float4 cl = make_float4(1.f, 1.f, 1.f, 1.f), ch = cl;
                     if (has_vec && in) { cl = c_lo[v]; ch = c_hi[v]; }
                     uint64_t c2[4] = {pack2(cl.x, cl.y), pack2(cl.z, cl.w), pack2(ch.x, ch.y), pack2(ch.z, ch.w)};
@@ -627,7 +640,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                 constexpr float qmax = MODE == MODE_QF8 ? kF8Max : kQmax;
                 const float delta = mrow > 0.0f ? __fdiv_rn(mrow, qmax) : 0.0f;
                 const float inv_m = mrow > 0.0f ? __fdiv_rn(qmax, mrow) : 0.0f;
-                if (wig == 0 && (lane % SUB) == 0 && lane / SUB < nr) p.scale[r0 + lane / SUB] = delta;
+                if (wig == 0 && (lane % SUB) == 0 && lane / SUB < nr && SQ_CHECK(r0 + lane / SUB < p.rows, p.status))
+                    p.scale[r0 + lane / SUB] = delta;
                 // ---- pass C: codes
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
@@ -638,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
 #pragma unroll
                         for (int i = 0; i < VPL; ++i) {
                             const int v = i * GT + gtid;
-                            if (FULL || v < nvec) {
+                            if (SQ_COL_IN(v)) {
                                 uint32_t c01, c23, c45, c67;
                                 if (MODE == MODE_QF8) {
                                     c01 = f8codes2(mul2_rn(y[r][i][0], inv2)); c23 = f8codes2(mul2_rn(y[r][i][1], inv2));
@@ -649,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
                                 }
                                 uint2 out = make_uint2(__byte_perm(c01, c23, 0x5410), __byte_perm(c45, c67, 0x5410));
                                 if (MODE == MODE_QF8 && iv == 0.0f) out = make_uint2(0u, 0u);   // a zero row: codes +0
-                                qrow[v] = out;
+                                if (SQ_CHECK(r0 + r < p.rows, p.status)) qrow[v] = out;
                             }
                         }
                     }
@@ -677,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
 #pragma unroll
             for (int i = 0; i < VPL; ++i) {
                 const int v = i * GT + gtid;
-                if (FULL || v < nvec) {
+                if (SQ_COL_IN(v)) {
                     float *dst = red + static_cast<size_t>(group) * K + v * 8;
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
@@ -706,7 +720,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
             float m = 0.0f;
             for (int q = 0; q < csize; ++q) m = fmaxf(m, cluster.map_shared_rank(red, q)[c]);
             // abs-maxima are non-negative, where IEEE order equals unsigned integer order
-            if (m > 0.0f) atomicMax(reinterpret_cast<unsigned int *>(p.amax + c), __float_as_uint(m));
+            if (m > 0.0f && SQ_CHECK(c >= 0 && c < K, p.status))
+                atomicMax(reinterpret_cast<unsigned int *>(p.amax + c), __float_as_uint(m));
         }
         cluster.sync();
     }

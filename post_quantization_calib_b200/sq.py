@@ -4,6 +4,10 @@ Every step of the smoothed W8A8 linear runs in libsq's CUDA kernels. This module
 tensor placement / dtype, allocates outputs with PyTorch when the caller does not pass them, and
 forwards raw device pointers, sizes and the current CUDA stream. Importing it fails (ImportError)
 when ``libsq.so`` has not been built: there is no fallback path.
+
+With the environment variable ``SQ_CHECKED=1`` set at import, the binding loads
+``libsq_checked.so`` instead: the same kernels built with device-side bounds checks, which record
+SQ_ERR_BOUNDS in the status word (read by ``sq_device_status``) and skip the access, never fault.
 """
 from __future__ import annotations
 
@@ -16,18 +20,20 @@ import torch
 __all__ = [
     "SQError", "lib", "sq_calibrate_absmax", "sq_compute_scales", "sq_smooth_quantize_weight",
     "sq_rmsnorm_smooth_quant", "sq_w8a8_linear", "sq_w8a8_linear_workspace_size", "sq_device_status",
-    "sq_set_wait_timeout_ns", "sq_selftest_wait_timeout", "sq_set_gemm_cta_pair",
+    "sq_set_wait_timeout_ns", "sq_selftest_wait_timeout", "sq_selftest_bounds_check", "sq_set_gemm_cta_pair",
     "sq_static_scale", "sq_rmsnorm_smooth_quant_static", "sq_fold_into_prev_linear", "sq_fold_into_w_scale",
     "sq_smooth_quantize_weight_fp8", "sq_rmsnorm_smooth_quant_fp8", "sq_w8a8_linear_fp8", "sq_calibrate_absmax_layernorm", "sq_fold_layernorm_bias",
     "sq_layernorm_smooth_quant", "sq_status_string", "sq_last_error",
-    "sq_version", "LIB_PATH", "EXPORTS",
+    "sq_version", "LIB_PATH", "EXPORTS", "CHECKED",
 ]
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsq.so")
+CHECKED = os.environ.get("SQ_CHECKED", "0") not in ("", "0")
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libsq_checked.so" if CHECKED else "libsq.so")
 
 SQ_OK = 0
 STATUS_NAMES = {0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_UNSUPPORTED", 3: "SQ_ERR_MISALIGNED",
-                4: "SQ_ERR_ARCH", 5: "SQ_ERR_CUDA", 6: "SQ_ERR_TIMEOUT"}
+                4: "SQ_ERR_ARCH", 5: "SQ_ERR_CUDA", 6: "SQ_ERR_TIMEOUT", 7: "SQ_ERR_BOUNDS"}
 
 _p, _i64, _f, _i, _sz, _u64 = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_float, ctypes.c_int,
                                ctypes.c_size_t, ctypes.c_uint64)
@@ -46,6 +52,7 @@ EXPORTS = {
     "sq_device_status": (_i, [_p]),
     "sq_set_wait_timeout_ns": (_i, [_u64]),
     "sq_selftest_wait_timeout": (_i, [_p]),
+    "sq_selftest_bounds_check": (_i, [_p]),
     "sq_set_gemm_cta_pair": (_i, [_i]),
     "sq_static_scale": (_i, [_p, _p, _i64, _p, _p]),
     "sq_rmsnorm_smooth_quant_static": (_i, [_p, _i64, _i64, _p, _f, _i, _p, _p, _p, _p]),
@@ -62,8 +69,9 @@ EXPORTS = {
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libsq.so not found at {LIB_PATH}; build it with "
-                          "`python -m post_quantization_calib_b200.build` (nvcc, sm_100a)")
+        raise ImportError(f"{os.path.basename(LIB_PATH)} not found at {LIB_PATH}; build it with "
+                          "`python -m post_quantization_calib_b200.build"
+                          f"{' --checked' if CHECKED else ''}` (nvcc, sm_100a)")
     L = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in EXPORTS.items():
         fn = getattr(L, name)
@@ -392,3 +400,8 @@ def sq_set_gemm_cta_pair(enable: bool) -> None:
 
 def sq_selftest_wait_timeout(stream=None) -> None:
     _check(_lib.sq_selftest_wait_timeout(_stream(stream)), "sq_selftest_wait_timeout")
+
+
+def sq_selftest_bounds_check(stream=None) -> None:
+    """Launch the failing bounds check of libsq_checked.so (SQ_ERR_UNSUPPORTED in libsq.so)."""
+    _check(_lib.sq_selftest_bounds_check(_stream(stream)), "sq_selftest_bounds_check")

@@ -11,7 +11,7 @@ import torch
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "sq.h")
 
-SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_UNSUPPORTED, SQ_ERR_MISALIGNED, SQ_ERR_ARCH, SQ_ERR_CUDA, SQ_ERR_TIMEOUT = range(7)
+SQ_OK, SQ_ERR_INVALID_ARG, SQ_ERR_UNSUPPORTED, SQ_ERR_MISALIGNED, SQ_ERR_ARCH, SQ_ERR_CUDA, SQ_ERR_TIMEOUT, SQ_ERR_BOUNDS = range(8)
 
 
 @pytest.fixture(scope="module")
@@ -47,10 +47,21 @@ def test_library_exports_every_declared_symbol(sqmod):
     assert set(sqmod.EXPORTS) == set(names)
 
 
+def test_checked_library_exports_the_same_symbols(sqmod):
+    """libsq_checked.so (device bounds checks compiled in) exports the same C ABI as libsq.so."""
+    from post_quantization_calib_b200 import build
+    path = build.build(checked=True)
+    assert path.endswith("libsq_checked.so") and path != sqmod.LIB_PATH
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (sq_[a-z0-9_]+)", out))
+    assert set(declared_functions()) <= exported
+
+
 def test_status_strings(sqmod):
-    names = [sqmod.sq_status_string(i) for i in range(7)]
+    names = [sqmod.sq_status_string(i) for i in range(8)]
     assert names == ["SQ_OK", "SQ_ERR_INVALID_ARG", "SQ_ERR_UNSUPPORTED", "SQ_ERR_MISALIGNED",
-                     "SQ_ERR_ARCH", "SQ_ERR_CUDA", "SQ_ERR_TIMEOUT"]
+                     "SQ_ERR_ARCH", "SQ_ERR_CUDA", "SQ_ERR_TIMEOUT", "SQ_ERR_BOUNDS"]
+    assert all(sqmod.STATUS_NAMES[i] == names[i] for i in range(8))
     assert sqmod.sq_status_string(99) == "SQ_ERR_UNKNOWN"
     assert "sm_100a" in sqmod.sq_version()
 

@@ -11,6 +11,8 @@ All five workloads run at their full sizes in the launch configuration the bench
 is checked on sampled full output rows and full output columns (the oracle computes those one by
 one), the other stages on every element.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -19,14 +21,29 @@ pytestmark = pytest.mark.gpu
 
 from post_quantization_calib_b200 import synth  # noqa: E402
 
+# SQ_CHECKED=1: run against libsq_checked.so, the kernels with device-side bounds checks compiled in
+CHECKED = os.environ.get("SQ_CHECKED", "0") not in ("", "0")
+SQ_ERR_BOUNDS = 7
+
 
 @pytest.fixture(scope="module")
 def sq():
     from post_quantization_calib_b200 import build
-    build.build()
+    build.build(checked=CHECKED)
     from post_quantization_calib_b200 import sq as m
+    assert m.CHECKED == CHECKED
     assert torch.cuda.is_available(), "GPU tests need a CUDA device"
     return m
+
+
+@pytest.fixture(autouse=True)
+def no_failed_bounds_check():
+    """Under the checked library, no test may leave a failed device-side bounds check behind."""
+    yield
+    if CHECKED:
+        from post_quantization_calib_b200 import sq as m
+        st = m.sq_device_status()
+        assert st != SQ_ERR_BOUNDS, "a device-side bounds check failed (SQ_ERR_BOUNDS)"
 
 
 def h16(t):
