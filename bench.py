@@ -250,25 +250,28 @@ def main_gpu(args, rank, local_rank, world):
     stream = torch.cuda.current_stream(dev)
     names = list(LAUNCHES)
 
-    # ev: events recorded at the stage boundaries listed in `at` (None: all seven)
-    def step(ev=None, at=None):
+    # ev: events recorded at the stage boundaries listed in `at` (None: all seven). bufs: the step's
+    # (calibration set, weight, tokens, output) buffers (default: the resident ones).
+    def step(ev=None, at=None, bufs=None):
+        c_in, w_in, x_in, y_out = bufs if bufs is not None else (calib, W, X, y)
+
         def mark(i):
             if ev is not None and (at is None or i in at):
                 ev[i].record(stream)
         mark(0)
-        sq.sq_calibrate_absmax(calib, norm_gamma=gamma, eps=w.eps, amax=amax, accumulate=False, stream=stream)
+        sq.sq_calibrate_absmax(c_in, norm_gamma=gamma, eps=w.eps, amax=amax, accumulate=False, stream=stream)
         mark(1)
         if world > 1:
             sqdist.allreduce_max_(amax)
-        sq.sq_calibrate_absmax(W, amax=aw, accumulate=False, stream=stream)
+        sq.sq_calibrate_absmax(w_in, amax=aw, accumulate=False, stream=stream)
         mark(2)
         sq.sq_compute_scales(amax, aw, w.alpha, gamma=gamma, s=s, fold=fold, stream=stream)
         mark(3)
-        sq.sq_smooth_quantize_weight(W, s, wq=wq, w_scale=ws, stream=stream)
+        sq.sq_smooth_quantize_weight(w_in, s, wq=wq, w_scale=ws, stream=stream)
         mark(4)
-        sq.sq_rmsnorm_smooth_quant(X, fold, eps=w.eps, apply_norm=w.norm, xq=xq, x_scale=xs, stream=stream)
+        sq.sq_rmsnorm_smooth_quant(x_in, fold, eps=w.eps, apply_norm=w.norm, xq=xq, x_scale=xs, stream=stream)
         mark(5)
-        sq.sq_w8a8_linear(xq, xs, wq, ws, y=y, stream=stream)
+        sq.sq_w8a8_linear(xq, xs, wq, ws, y=y_out, stream=stream)
         mark(6)
 
     def barrier():
@@ -325,31 +328,69 @@ def main_gpu(args, rank, local_rank, world):
     ms_per_step = elapsed_ms / args.steps
     value = world * w.linear_ops() * args.steps / (elapsed_ms * 1e-3) / 1e12
 
-    # ---- end to end through the C ABI with host buffers: pinned H2D of this step's inputs, D2H of y
+    # ---- end to end through the C ABI with host buffers: every step copies its inputs from pinned
+    # host memory and its output y back. Consecutive steps are pipelined as a user streaming batches
+    # would: two sets of device buffers, host-to-device copies on one stream, device-to-host copies on
+    # another (the two directions use separate copy engines), the library calls on the compute stream.
+    # A step's copy into a buffer set waits until the step two earlier has finished reading it; a
+    # step's output waits until its buffer's previous copy to the host is done.
     e2e_steps = 0 if args.no_e2e else max(2, min(args.steps, 20))
     pin = (lambda t: t.cpu().pin_memory()) if e2e_steps else (lambda t: t.cpu()[:0])
     calib_h, W_h, X_h = pin(calib), pin(W), pin(X)
-    y_h = torch.empty(T, N, dtype=torch.bfloat16).pin_memory() if e2e_steps else torch.empty(0)
+    if e2e_steps:
+        sets = [(calib, W, X, y), (torch.empty_like(calib), torch.empty_like(W), torch.empty_like(X), torch.empty_like(y))]
+        y_hs = [torch.empty(T, N, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    h2d_stream = torch.cuda.Stream(dev)
+    d2h_stream = torch.cuda.Stream(dev)
+    done_reading = [None, None]    # per buffer set: the compute of its last step has finished
+    done_writing = [None, None]    # per buffer set: the copy of its last output to the host has finished
 
-    def e2e_step():
-        calib.copy_(calib_h, non_blocking=True)
-        W.copy_(W_h, non_blocking=True)
-        X.copy_(X_h, non_blocking=True)
-        step()
-        y_h.copy_(y, non_blocking=True)
+    def e2e_step(i):
+        k = i % 2
+        c_in, w_in, x_in, y_out = sets[k]
+        with torch.cuda.stream(h2d_stream):
+            if done_reading[k] is not None:
+                h2d_stream.wait_event(done_reading[k])
+            c_in.copy_(calib_h, non_blocking=True)
+            w_in.copy_(W_h, non_blocking=True)
+            x_in.copy_(X_h, non_blocking=True)
+            loaded = torch.cuda.Event()
+            loaded.record(h2d_stream)
+        stream.wait_event(loaded)
+        if done_writing[k] is not None:
+            stream.wait_event(done_writing[k])
+        step(bufs=sets[k])
+        computed = torch.cuda.Event()
+        computed.record(stream)
+        done_reading[k] = computed
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(computed)
+            y_hs[k].copy_(y_out, non_blocking=True)
+            written = torch.cuda.Event()
+            written.record(d2h_stream)
+        done_writing[k] = written
 
     if e2e_steps:
-        e2e_step()
+        for i in range(2):
+            e2e_step(i)
     barrier()
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    h2d_stream.wait_stream(stream)
+    d2h_stream.wait_stream(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    stream.wait_stream(d2h_stream)
+    stream.wait_stream(h2d_stream)
     b.record(stream)
     torch.cuda.synchronize()
     e2e_ms = a.elapsed_time(b) / e2e_steps if e2e_steps else float("nan")
+    if e2e_steps:
+        # the last step's output arrived on the host intact
+        if not torch.equal(y_hs[(e2e_steps - 1) % 2], y.cpu()):
+            raise RuntimeError("end-to-end output differs from the device-resident step's output")
     te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(te, op=dist.ReduceOp.MAX)
