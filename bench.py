@@ -2,14 +2,14 @@
 
 One step is one pass of the whole path over one batch of synthetic, outlier-shaped input resident in
 HBM, for the Qwen3-8B-shaped query projection (T = 8192 tokens, K = N = 4096, RMSNorm-fed, alpha 0.5):
-  1. abs-max of the RMSNorm output over 128 x 512 calibration tokens (537 MB read),
-  2. abs-max of the weight per input channel,
+  1. abs-max of the RMSNorm output over 128 x 512 calibration tokens (537 MB read) and
+  2. abs-max of the weight per input channel, both in one launch,
   3. smoothing factors s and the folded norm weight gamma / s,
   4. diag(s) W quantised to INT8 per output channel,
   5. fused RMSNorm(gamma / s) + per-token INT8 quantisation of the 8192 tokens,
   6. INT8 x INT8 -> INT32 GEMM with the per-token x per-channel dequant epilogue to bf16.
 With N > 1 GPUs every rank runs the same step on its own tokens (weak scaling) and the calibration
-abs-maxima are combined with an NCCL all-reduce(MAX) between steps 1 and 3 -- the path's only exchange.
+abs-maxima are combined with an NCCL all-reduce(MAX) between steps 1-2 and 3 -- the path's only exchange.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
        (N > 1: launch with torchrun, one process per GPU)
@@ -121,8 +121,8 @@ class ClockSampler:
 
 def stage_work(w, T, N, K, calib_rows):
     return {
-        "calib_absmax": {"bytes": 2 * calib_rows * K + 4 * K + 4 * K, "bound": "hbm"},
-        "weight_absmax": {"bytes": 2 * N * K + 4 * K, "bound": "hbm"},
+        # the calibration rows and the weight rows read, gamma read, both maxima written
+        "calib_absmax": {"bytes": 2 * calib_rows * K + 2 * N * K + 4 * K + 4 * K + 4 * K, "bound": "hbm"},
         "scales": {"bytes": 4 * K * 5, "bound": "hbm"},
         "weight_quant": {"bytes": 2 * N * K + N * K + 4 * K + 4 * N, "bound": "hbm"},
         "act_quant": {"bytes": 2 * T * K + T * K + 4 * K + 4 * T, "bound": "hbm"},
@@ -130,10 +130,10 @@ def stage_work(w, T, N, K, calib_rows):
     }
 
 
-KERNEL_OF = {"calib_absmax": ("k_rows<2,8,1,ABSMAX,NORM>", "sq_rowwise.cu"), "weight_absmax": ("k_rows<2,8,1,ABSMAX>", "sq_rowwise.cu"),
+KERNEL_OF = {"calib_absmax": ("k_absmax_pair<2,8,1,NORM>", "sq_rowwise.cu"),
              "scales": ("k_scales", "sq_rowwise.cu"), "weight_quant": ("k_rows<2,8,1,QUANT>", "sq_rowwise.cu"),
              "act_quant": ("k_rows<2,8,1,QUANT,NORM>", "sq_rowwise.cu"), "gemm": ("k_w8a8_linear<256>", "sq_gemm.cu")}
-LAUNCHES = {"calib_absmax": 2, "weight_absmax": 2, "scales": 1, "weight_quant": 1, "act_quant": 1, "gemm": 1}
+LAUNCHES = {"calib_absmax": 2, "scales": 1, "weight_quant": 1, "act_quant": 1, "gemm": 1}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -250,7 +250,7 @@ def main_gpu(args, rank, local_rank, world):
     stream = torch.cuda.current_stream(dev)
     names = list(LAUNCHES)
 
-    # ev: events recorded at the stage boundaries listed in `at` (None: all seven). bufs: the step's
+    # ev: events recorded at the stage boundaries listed in `at` (None: all). bufs: the step's
     # (calibration set, weight, tokens, output) buffers (default: the resident ones).
     def step(ev=None, at=None, bufs=None):
         c_in, w_in, x_in, y_out = bufs if bufs is not None else (calib, W, X, y)
@@ -259,20 +259,20 @@ def main_gpu(args, rank, local_rank, world):
             if ev is not None and (at is None or i in at):
                 ev[i].record(stream)
         mark(0)
-        sq.sq_calibrate_absmax(c_in, norm_gamma=gamma, eps=w.eps, amax=amax, accumulate=False, stream=stream)
-        mark(1)
+        # S1 + S2: the calibration maxima (of the RMSNorm output) and the weight maxima, one launch
+        sq.sq_calibrate_absmax_pair(c_in, w_in, norm_gamma=gamma, eps=w.eps, amax=amax, amax_w=aw,
+                                    accumulate=False, stream=stream)
         if world > 1:
-            sqdist.allreduce_max_(amax)
-        sq.sq_calibrate_absmax(w_in, amax=aw, accumulate=False, stream=stream)
-        mark(2)
+            sqdist.allreduce_max_(amax)         # every rank's calibration rows: the global maxima
+        mark(1)
         sq.sq_compute_scales(amax, aw, w.alpha, gamma=gamma, s=s, fold=fold, stream=stream)
-        mark(3)
+        mark(2)
         sq.sq_smooth_quantize_weight(w_in, s, wq=wq, w_scale=ws, stream=stream)
-        mark(4)
+        mark(3)
         sq.sq_rmsnorm_smooth_quant(x_in, fold, eps=w.eps, apply_norm=w.norm, xq=xq, x_scale=xs, stream=stream)
-        mark(5)
+        mark(4)
         sq.sq_w8a8_linear(xq, xs, wq, ws, y=y_out, stream=stream)
-        mark(6)
+        mark(5)
 
     def barrier():
         if world > 1:
@@ -288,7 +288,7 @@ def main_gpu(args, rank, local_rank, world):
     # two kernels stops the second from starting early (dependent launch) and cost ~20 us per step, so
     # the timed steps below record events only around the dominant stage.
     nb = max(3, min(args.steps, 200))
-    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(nb)]
+    bevs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(nb)]
     for i in range(nb):
         step(bevs[i])
     torch.cuda.synchronize()
@@ -301,7 +301,7 @@ def main_gpu(args, rank, local_rank, world):
 
     clocks = ClockSampler(local_rank)
     clocks.start()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)

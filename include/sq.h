@@ -90,6 +90,26 @@ sq_status sq_calibrate_absmax(const void *a, int64_t rows, int64_t cols, int64_t
                               void *stream);
 
 /*
+ * Both maxima of one smoothing group in one launch: the same result as
+ *   sq_calibrate_absmax(a, rows, cols, ld, norm_gamma, eps, amax, accumulate, stream) and then
+ *   sq_calibrate_absmax(w, w_rows, cols, w_ld, NULL, 0, amax_w, accumulate, stream),
+ * the activation maxima max|X_j| and the weight maxima max|W_j| that the smoothing factor of
+ * [MIGRATE] section 3 combines. The two reductions are independent. When cols > 2048 and both inputs
+ * have rows, one kernel reduces both: part of its CTAs streams the weight rows while the rest stream
+ * the activation rows (the split follows the inputs' sizes). Otherwise the two reductions are
+ * launched one after the other.
+ * a, rows, ld, norm_gamma, eps, amax: as in sq_calibrate_absmax.
+ * w          bf16 [w_rows, cols], row stride w_ld elements (a weight stored [N, K]); never normalised.
+ * amax_w     fp32 [cols], in/out; a different array from amax.
+ * accumulate applies to both outputs (0 overwrites both, 1 keeps both running maxima).
+ * Requirements: those of sq_calibrate_absmax for each input; amax != amax_w (else
+ * SQ_ERR_INVALID_ARG).
+ */
+sq_status sq_calibrate_absmax_pair(const void *a, int64_t rows, int64_t cols, int64_t ld, const float *norm_gamma,
+                                   float eps, float *amax, const void *w, int64_t w_rows, int64_t w_ld, float *amax_w,
+                                   int accumulate, void *stream);
+
+/*
  * Smoothing factors and the folded norm weight.
  *   [MIGRATE] section 3; [W8A8] "The trick: move the range into the weights" (formula and the
  *   fold into the norm's weights); clamp of s from [TAMING] "Implementation in PyTorch".

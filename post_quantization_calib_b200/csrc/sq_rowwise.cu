@@ -284,8 +284,9 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
 // One CTA = 16 warps in row groups of WPR warps. A group processes units of R consecutive rows; lane l
 // of warp w of the group covers the 8-element vectors v = i * 32 * WPR + 32 * w + l (i < VPL) of
 // every row of the unit. R > 1 only with WPR == 1.
+// The body of a row kernel: this CTA is number `cta` of the `nctas` CTAs that share problem p.
 template <int WPR, int VPL, int R, int MODE, bool NORM, bool FULL>
-__global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
+__device__ __forceinline__ void rows_body(const RowArgs p, unsigned cta, unsigned nctas)
 {
     constexpr int G = kWarps / WPR;   // row groups per CTA
     constexpr int GT = 32 * WPR;      // consumer threads per row group
@@ -329,8 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
     }
 
     const int64_t units = (p.rows + R - 1) / R;
-    const int64_t g0 = static_cast<int64_t>(blockIdx.x) * G + group;
-    const int64_t gstride = static_cast<int64_t>(gridDim.x) * G;
+    const int64_t g0 = static_cast<int64_t>(cta) * G + group;
+    const int64_t gstride = static_cast<int64_t>(nctas) * G;
     const int64_t nunits = g0 < units ? (units - 1 - g0) / gstride + 1 : 0;
 
     if (tid == 0) {
@@ -727,6 +728,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
     }
 }
 
+template <int WPR, int VPL, int R, int MODE, bool NORM, bool FULL>
+__global__ void __launch_bounds__(kThreads, 1) k_rows(const RowArgs p)
+{
+    rows_body<WPR, VPL, R, MODE, NORM, FULL>(p, blockIdx.x, gridDim.x);
+}
+
+// Column abs-maxima of two inputs with the same row length in one launch: CTAs [0, ctas_a) reduce the
+// rows of pa (their RMSNorm output when NORM_A), the others the plain rows of pw (a weight). The split
+// lies on a cluster boundary, so the cross-CTA reduction of every cluster stays within one input.
+template <int WPR, int VPL, int R, bool NORM_A, bool FULL>
+__global__ void __launch_bounds__(kThreads, 1) k_absmax_pair(const RowArgs pa, const RowArgs pw, unsigned ctas_a)
+{
+    if (blockIdx.x < ctas_a) rows_body<WPR, VPL, R, MODE_ABSMAX, NORM_A, FULL>(pa, blockIdx.x, ctas_a);
+    else rows_body<WPR, VPL, R, MODE_ABSMAX, false, FULL>(pw, blockIdx.x - ctas_a, gridDim.x - ctas_a);
+}
+
+// Zero-fill of two arrays in one launch (the running maxima of k_absmax_pair); waits for the
+// previous work of the stream, then lets the next kernel start.
+__global__ void k_fill_zero2(float *__restrict__ p, int64_t n, float *__restrict__ q, int64_t m) {
+    pdl_wait();
+    pdl_trigger();
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n + m;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        if (i < n) p[i] = 0.0f;
+        else q[i - n] = 0.0f;
+    }
+}
+
 __global__ void k_fill_zero(float *__restrict__ p, int64_t n) {
     pdl_wait();          // earlier grids complete before the next kernel may start (it reads early)
     pdl_trigger();
@@ -934,6 +963,111 @@ sq_status dispatch_rows(const RowArgs &a, int dev, cudaStream_t st) {
     return full ? dispatch_rows_f<MODE, NORM, true>(a, g, dev, st) : dispatch_rows_f<MODE, NORM, false>(a, g, dev, st);
 }
 
+// Relative cost of a row of the plain abs-max against a row of the RMSNorm-fed one (same length): the
+// plain rows only stream through the ring, the norm-fed ones are bound by their per-element work.
+constexpr double kPlainRowCost = 0.5;
+
+template <int WPR, int VPL, int R, bool NORM_A, bool FULL>
+sq_status launch_pair_t(RowArgs a, RowArgs w, const Geo &geo, int dev, cudaStream_t st) {
+    auto kern = k_absmax_pair<WPR, VPL, R, NORM_A, FULL>;
+    constexpr int G = kWarps / WPR;
+    const int nvec = a.K / 8;
+    if (geo.wpr != WPR || geo.vpl != VPL || geo.rpu != R || geo.groups != G || nvec > WPR * 32 * VPL ||
+        (FULL && nvec != WPR * 32 * VPL))
+        return sq::fail(SQ_ERR_UNSUPPORTED, "row kernel geometry mismatch (K=%d)", a.K);
+    static std::mutex mu;
+    static size_t configured_smem[64];
+    static int cluster_size[64], cluster_ctas[64];
+    static size_t smem_cap[64];
+    std::unique_lock<std::mutex> lk(mu);
+    if (smem_cap[dev] == 0) {
+        int optin = 0;
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e == cudaSuccess) e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return sq::cuda_status(e, "shared memory limits (absmax pair)");
+        smem_cap[dev] = static_cast<size_t>(optin) - fa.sharedSizeBytes;
+    }
+    int stages = kMaxStages;
+    while (stages > 2 && rows_smem(a.K, MODE_ABSMAX, geo, stages) > smem_cap[dev]) --stages;
+    const size_t smem = rows_smem(a.K, MODE_ABSMAX, geo, stages);
+    if (smem > smem_cap[dev]) return sq::fail(SQ_ERR_UNSUPPORTED, "row kernel needs %zu bytes of shared memory", smem);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    if (configured_smem[dev] < smem) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return sq::cuda_status(e, "cudaFuncSetAttribute(absmax pair)");
+        cudaLaunchConfig_t cfg = {};
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        // the cluster size that keeps the most CTAs resident at once (ties: the larger cluster)
+        cluster_size[dev] = 1;
+        cluster_ctas[dev] = 0;
+        for (int c = kMaxCluster; c >= 2; c /= 2) {
+            attr[0].val.clusterDim.x = c;
+            cfg.gridDim = dim3(c, 1, 1);
+            int nc = 0;
+            if (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) != cudaSuccess) { (void)cudaGetLastError(); continue; }
+            if (nc * c > cluster_ctas[dev]) { cluster_ctas[dev] = nc * c; cluster_size[dev] = c; }
+        }
+        if (cluster_ctas[dev] == 0) return sq::fail(SQ_ERR_CUDA, "no cluster configuration fits the abs-max kernel");
+        configured_smem[dev] = smem;
+    }
+    const int csz = cluster_size[dev], cctas = cluster_ctas[dev];
+    lk.unlock();
+    if (cctas < 2 * csz) return sq::fail(SQ_ERR_UNSUPPORTED, "fewer than two clusters fit for the abs-max pair");
+    for (RowArgs *r : {&a, &w}) {
+        r->stages = stages;
+        r->inv_k = (r->K & (r->K - 1)) == 0 ? 1.0 / static_cast<double>(r->K) : 0.0;
+        r->status = sq::device_status_word(dev);
+        r->limit_ns = sq::wait_timeout_ns(dev);
+        r->stream_once = static_cast<double>(r->rows) * static_cast<double>(r->ld_bytes) > 0.5 * sq::l2_bytes(dev) ? 1 : 0;
+    }
+    if (a.status == nullptr) return sq::fail(SQ_ERR_CUDA, "device status word unavailable");
+    // CTAs per input: at most one per ~4 units per group, whole clusters, one wave in total; when both
+    // do not fit, the wave is divided by the inputs' costs.
+    auto want = [&](int64_t rows) {
+        const int64_t units = (rows + R - 1) / R;
+        const int64_t c = (units + 4 * G - 1) / (4 * G);
+        return ((c + csz - 1) / csz) * csz;
+    };
+    const int64_t wa = want(a.rows), ww = want(w.rows);
+    const int64_t wave = (cctas / csz) * csz;
+    int64_t ca = wa, cw = ww;
+    if (ca + cw > wave) {
+        const double cost_a = static_cast<double>(a.rows), cost_w = kPlainRowCost * static_cast<double>(w.rows);
+        int64_t share_w = static_cast<int64_t>(static_cast<double>(wave) * cost_w / (cost_a + cost_w) / csz + 0.5) * csz;
+        share_w = share_w < csz ? csz : share_w > wave - csz ? wave - csz : share_w;
+        cw = ww < share_w ? ww : share_w;
+        ca = wa < wave - cw ? wa : wave - cw;
+        cw = ww < wave - ca ? ww : wave - ca;      // CTAs the other input leaves unused
+    }
+    attr[0].val.clusterDim.x = csz;
+    return sq::cuda_status(sq::launch_pdl(kern, dim3(static_cast<unsigned>(ca + cw)), dim3(kThreads), smem, st, &attr[0], a, w,
+                                          static_cast<unsigned>(ca)),
+                           "launch(absmax pair)");
+}
+
+// The one-launch form covers rows of more than 2048 elements (one row per unit); false when the
+// geometry has none, and the caller then launches the two reductions one after the other.
+template <bool NORM_A>
+bool dispatch_pair(const RowArgs &a, const RowArgs &w, int dev, cudaStream_t st, sq_status *out) {
+    const Geo g = row_geo(a.K);
+    if (g.wpr < 2) return false;
+    const bool full = (a.K / 8) == g.vpl * 32 * g.wpr;
+    switch (g.wpr) {
+        case 2: *out = full ? launch_pair_t<2, 8, 1, NORM_A, true>(a, w, g, dev, st) : launch_pair_t<2, 8, 1, NORM_A, false>(a, w, g, dev, st); break;
+        case 4: *out = full ? launch_pair_t<4, 8, 1, NORM_A, true>(a, w, g, dev, st) : launch_pair_t<4, 8, 1, NORM_A, false>(a, w, g, dev, st); break;
+        default: *out = full ? launch_pair_t<8, 8, 1, NORM_A, true>(a, w, g, dev, st) : launch_pair_t<8, 8, 1, NORM_A, false>(a, w, g, dev, st); break;
+    }
+    return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -973,6 +1107,76 @@ sq_status sq_calibrate_absmax(const void *a, int64_t rows, int64_t cols, int64_t
     ra.amax = amax;
     ra.early = accumulate ? 0 : 1;   // the zero-fill above was the stream's last kernel
     return norm_gamma ? dispatch_rows<MODE_ABSMAX, true>(ra, dev, st) : dispatch_rows<MODE_ABSMAX, false>(ra, dev, st);
+}
+
+// Arguments of one input of sq_calibrate_absmax_pair, checked as sq_calibrate_absmax checks them.
+static sq_status check_absmax_input(const char *fn, const char *name, const void *a, int64_t rows, int64_t cols,
+                                    int64_t ld, const float *amax) {
+    using sq::fail;
+    if (!amax) return fail(SQ_ERR_INVALID_ARG, "%s: the maxima of %s are NULL", fn, name);
+    if (rows < 0 || cols < 8 || ld < cols)
+        return fail(SQ_ERR_INVALID_ARG, "%s: need rows >= 0, cols >= 8, ld >= cols for %s (rows=%lld cols=%lld ld=%lld)",
+                    fn, name, (long long)rows, (long long)cols, (long long)ld);
+    if (rows > 0 && !a) return fail(SQ_ERR_INVALID_ARG, "%s: %s is NULL", fn, name);
+    if (cols % 8 != 0 || ld % 8 != 0) return fail(SQ_ERR_MISALIGNED, "%s: cols and the ld of %s must be multiples of 8", fn, name);
+    if ((a && !sq::aligned(a, 16)) || !sq::aligned(amax, 4))
+        return fail(SQ_ERR_MISALIGNED, "%s: %s must be 16-byte aligned and its maxima 4-byte aligned", fn, name);
+    if (cols > kMaxK) return fail(SQ_ERR_UNSUPPORTED, "%s: cols must be <= %d", fn, kMaxK);
+    return SQ_OK;
+}
+
+// The activation and weight maxima of one smoothing group (the two per-channel maxima that the
+// smoothing factor of [MIGRATE] section 3 combines) in one launch. The two reductions are
+// independent; sharing the launch saves the second one's start-up and end phase.
+sq_status sq_calibrate_absmax_pair(const void *a, int64_t rows, int64_t cols, int64_t ld, const float *norm_gamma,
+                                   float eps, float *amax, const void *w, int64_t w_rows, int64_t w_ld, float *amax_w,
+                                   int accumulate, void *stream)
+{
+    using sq::fail;
+    const char *fn = "sq_calibrate_absmax_pair";
+    sq_status c = check_absmax_input(fn, "a", a, rows, cols, ld, amax);
+    if (c == SQ_OK) c = check_absmax_input(fn, "w", w, w_rows, cols, w_ld, amax_w);
+    if (c != SQ_OK) return c;
+    if (norm_gamma && !sq::aligned(norm_gamma, 16)) return fail(SQ_ERR_MISALIGNED, "%s: norm_gamma must be 16-byte aligned", fn);
+    if (amax == amax_w) return fail(SQ_ERR_INVALID_ARG, "%s: amax and amax_w must be different arrays", fn);
+    int dev = 0;
+    SQ_TRY_ARCH(dev);
+    cudaStream_t st = sq::as_stream(stream);
+    if (!accumulate) {
+        const int64_t n = 2 * cols;
+        sq_status s0 = sq::cuda_status(sq::launch_pdl(k_fill_zero2, dim3(static_cast<unsigned>((n + 255) / 256)), dim3(256), 0,
+                                                      st, nullptr, amax, cols, amax_w, cols),
+                                       "launch(fill)");
+        if (s0 != SQ_OK) return s0;
+    }
+    RowArgs ra = {};
+    ra.src = static_cast<const uint8_t *>(a);
+    ra.rows = rows;
+    ra.ld_bytes = ld * 2;
+    ra.K = static_cast<int>(cols);
+    ra.vec = norm_gamma;
+    ra.eps = eps;
+    ra.amax = amax;
+    ra.early = accumulate ? 0 : 1;   // the zero-fill above was the stream's last kernel
+    RowArgs rw = ra;
+    rw.src = static_cast<const uint8_t *>(w);
+    rw.rows = w_rows;
+    rw.ld_bytes = w_ld * 2;
+    rw.vec = nullptr;
+    rw.amax = amax_w;
+    if (rows > 0 && w_rows > 0) {
+        sq_status out = SQ_OK;
+        if (norm_gamma ? dispatch_pair<true>(ra, rw, dev, st, &out) : dispatch_pair<false>(ra, rw, dev, st, &out)) return out;
+    }
+    // one input empty, or rows of at most 2048 elements: the two reductions one after the other (the
+    // second reads its rows only after the first has finished)
+    if (rows > 0) {
+        const sq_status s1 = norm_gamma ? dispatch_rows<MODE_ABSMAX, true>(ra, dev, st) : dispatch_rows<MODE_ABSMAX, false>(ra, dev, st);
+        if (s1 != SQ_OK) return s1;
+        rw.early = 0;
+    }
+    if (w_rows > 0) return dispatch_rows<MODE_ABSMAX, false>(rw, dev, st);
+    return SQ_OK;
 }
 
 // LayerNorm-fed layers ([WOVS] "SmoothQuant: Weight-Only vs W8A8", "Integration with

@@ -18,7 +18,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = [
-    "SQError", "lib", "sq_calibrate_absmax", "sq_compute_scales", "sq_smooth_quantize_weight",
+    "SQError", "lib", "sq_calibrate_absmax", "sq_calibrate_absmax_pair", "sq_compute_scales", "sq_smooth_quantize_weight",
     "sq_rmsnorm_smooth_quant", "sq_w8a8_linear", "sq_w8a8_linear_workspace_size", "sq_device_status",
     "sq_set_wait_timeout_ns", "sq_selftest_wait_timeout", "sq_selftest_bounds_check", "sq_set_gemm_cta_pair",
     "sq_static_scale", "sq_rmsnorm_smooth_quant_static", "sq_fold_into_prev_linear", "sq_fold_into_w_scale",
@@ -44,6 +44,7 @@ EXPORTS = {
     "sq_last_error": (ctypes.c_char_p, []),
     "sq_version": (ctypes.c_char_p, []),
     "sq_calibrate_absmax": (_i, [_p, _i64, _i64, _i64, _p, _f, _p, _i, _p]),
+    "sq_calibrate_absmax_pair": (_i, [_p, _i64, _i64, _i64, _p, _f, _p, _p, _i64, _i64, _p, _i, _p]),
     "sq_compute_scales": (_i, [_p, _p, _i64, _f, _p, _p, _p, _p]),
     "sq_smooth_quantize_weight": (_i, [_p, _i64, _i64, _p, _p, _p, _p]),
     "sq_rmsnorm_smooth_quant": (_i, [_p, _i64, _i64, _p, _f, _i, _p, _p, _p]),
@@ -156,6 +157,39 @@ def sq_calibrate_absmax(a: torch.Tensor, norm_gamma: Optional[torch.Tensor] = No
                                     float(eps), _ptr(amax), int(bool(accumulate)), _stream(stream)),
            "sq_calibrate_absmax")
     return amax
+
+
+def sq_calibrate_absmax_pair(a: torch.Tensor, w: torch.Tensor, norm_gamma: Optional[torch.Tensor] = None,
+                             eps: float = 1e-6, amax: Optional[torch.Tensor] = None,
+                             amax_w: Optional[torch.Tensor] = None, accumulate: bool = False,
+                             stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-column abs-max of bf16 ``a`` (its RMSNorm output with ``norm_gamma``) and of bf16 ``w`` in
+    one call; see sq.h. Returns (amax, amax_w)."""
+    for t, name in ((a, "a"), (w, "w")):
+        _dev(t, name, torch.bfloat16, contiguous=False)
+        if t.dim() != 2 or t.stride(1) != 1:
+            raise ValueError(f"{name} must be 2-D with unit column stride")
+    rows, cols = a.shape
+    w_rows, w_cols = w.shape
+    if w_cols != cols:
+        raise ValueError("a and w must have the same number of columns")
+    if amax is None or amax_w is None:
+        accumulate = False
+    if amax is None:
+        amax = torch.empty(cols, dtype=torch.float32, device=a.device)
+    if amax_w is None:
+        amax_w = torch.empty(cols, dtype=torch.float32, device=a.device)
+    _dev(amax, "amax", torch.float32)
+    _dev(amax_w, "amax_w", torch.float32)
+    if norm_gamma is not None:
+        _dev(norm_gamma, "norm_gamma", torch.float32)
+    ld = a.stride(0) if a.stride(0) >= cols else cols
+    w_ld = w.stride(0) if w.stride(0) >= cols else cols
+    _check(_lib.sq_calibrate_absmax_pair(_ptr(a), rows, cols, ld, _ptr(norm_gamma), float(eps), _ptr(amax),
+                                         _ptr(w), w_rows, w_ld, _ptr(amax_w), int(bool(accumulate)),
+                                         _stream(stream)),
+           "sq_calibrate_absmax_pair")
+    return amax, amax_w
 
 
 def sq_compute_scales(amax_x: torch.Tensor, amax_w: torch.Tensor, alpha: float,

@@ -145,6 +145,22 @@ def test_layernorm_argument_checks(sqmod):
     assert q(FAKE, -1, 64, FAKE, None, 1e-5, FAKE, FAKE, None) == SQ_ERR_INVALID_ARG
 
 
+def test_absmax_pair_argument_checks(sqmod):
+    c = sqmod.lib().sq_calibrate_absmax_pair
+    G = FAKE + 4096
+    #        a     rows cols ld   gamma eps   amax  w     wrows wld  amax_w acc stream
+    assert c(FAKE, 4, 64, 64, None, 1e-6, None, FAKE, 4, 64, G, 0, None) == SQ_ERR_INVALID_ARG     # amax NULL
+    assert c(FAKE, 4, 64, 64, None, 1e-6, G, FAKE, 4, 64, None, 0, None) == SQ_ERR_INVALID_ARG     # amax_w NULL
+    assert c(FAKE, 4, 64, 64, None, 1e-6, G, FAKE, 4, 64, G, 0, None) == SQ_ERR_INVALID_ARG        # same array
+    assert c(FAKE, 4, 64, 64, None, 1e-6, G, FAKE, 4, 32, G + 256, 0, None) == SQ_ERR_INVALID_ARG  # w_ld < cols
+    assert c(FAKE, 4, 64, 64, None, 1e-6, G, None, 4, 64, G + 256, 0, None) == SQ_ERR_INVALID_ARG  # w NULL with rows
+    assert c(FAKE, 4, 64, 64, None, 1e-6, G, FAKE, -1, 64, G + 256, 0, None) == SQ_ERR_INVALID_ARG # w_rows < 0
+    assert c(FAKE, 4, 64, 64, None, 1e-6, G, FAKE + 2, 4, 64, G + 256, 0, None) == SQ_ERR_MISALIGNED
+    assert c(FAKE, 4, 64, 64, FAKE + 4, 1e-6, G, FAKE, 4, 64, G + 256, 0, None) == SQ_ERR_MISALIGNED  # gamma
+    assert c(FAKE, 4, 64, 64, None, 1e-6, G, FAKE, 4, 68, G + 256, 0, None) == SQ_ERR_MISALIGNED   # w_ld % 8
+    assert c(FAKE, 4, 32768, 32768, None, 1e-6, G, FAKE, 4, 32768, G + 256, 0, None) == SQ_ERR_UNSUPPORTED
+
+
 def test_fp8_argument_checks(sqmod):
     L = sqmod.lib()
     assert L.sq_smooth_quantize_weight_fp8(FAKE, 4, 12, None, FAKE, FAKE, None) == SQ_ERR_MISALIGNED

@@ -255,6 +255,65 @@ def test_absmax_strided_rows_and_empty(sq, orc):
     ok_status(sq)
 
 
+# Both maxima of a smoothing group in one call, against the oracle's two reductions: the one-launch
+# form (rows of more than 2048 elements, both inputs non-empty; norm-fed or plain activations; whole
+# and ragged rows; strided inputs) and the two-launch form (narrow rows, one input empty), each with
+# overwrite and running-maximum semantics.
+PAIR_ABSMAX = [  # rows, w_rows, cols, norm, extra columns of a's row stride, of w's row stride
+    (65536, 4096, 4096, True, 0, 0),      # the query projection's calibration set and weight
+    (3000, 5000, 4096, True, 0, 0),       # more weight rows than activation rows
+    (777, 130, 2568, True, 8, 16),        # a row that is not a whole number of lane vectors; strided
+    (500, 7000, 8192, False, 0, 8),       # plain activations, wider rows
+    (64, 64, 16384, True, 0, 0),          # the widest rows
+    (1000, 300, 1024, True, 0, 0),        # narrow rows: two launches
+    (0, 300, 4096, True, 0, 0),           # no activation rows
+    (300, 0, 4096, False, 0, 0),          # no weight rows
+]
+
+
+@pytest.mark.parametrize("rows,w_rows,cols,norm,xa,xw", PAIR_ABSMAX)
+def test_absmax_pair(sq, orc, rows, w_rows, cols, norm, xa, xw):
+    dev = "cuda"
+    ch = synth.outlier_channels(cols + xa, synth.OutlierSpec(max(1, cols // 64), 10, 40), 5)
+    a = synth.outlier_tokens(rows, cols + xa, ch, 6, dev)[:, :cols]
+    w = synth.normal_weight(w_rows, cols + xw, 7, dev)[:, :cols]
+    g = synth.norm_gamma(cols, 8, dev) if norm else None
+    g_h = None if g is None else hnp(g)
+    ax, aw = sq.sq_calibrate_absmax_pair(a, w, norm_gamma=g, eps=1e-6)
+    ok_status(sq)
+    a_h, w_h = h16(a), h16(w)
+    ref_a = orc.calibrate_absmax(a_h, norm_gamma=g_h, eps=1e-6)
+    ref_w = orc.calibrate_absmax(w_h)
+    assert np.array_equal(hnp(ax), ref_a)
+    assert np.array_equal(hnp(aw), ref_w)
+    # running maxima: a second batch (half the rows, scaled up) raises some columns of each output
+    a2, w2 = (a[: rows // 2] * 3).contiguous(), (w[: w_rows // 2] * 3).contiguous()
+    sq.sq_calibrate_absmax_pair(a2, w2, norm_gamma=g, eps=1e-6, amax=ax, amax_w=aw, accumulate=True)
+    ok_status(sq)
+    orc.calibrate_absmax(h16(a2), norm_gamma=g_h, eps=1e-6, amax=ref_a, accumulate=True)
+    orc.calibrate_absmax(h16(w2), amax=ref_w, accumulate=True)
+    assert np.array_equal(hnp(ax), ref_a)
+    assert np.array_equal(hnp(aw), ref_w)
+
+
+def test_absmax_pair_matches_two_calls_at_every_split(sq):
+    """The one-launch form against two sq_calibrate_absmax calls over a range of input sizes, so that
+    the CTA split between the inputs takes many values (including the smallest share)."""
+    dev = "cuda"
+    K = 4096
+    ch = synth.outlier_channels(K, synth.OutlierSpec(64, 10, 40), 9)
+    a_all = synth.outlier_tokens(40000, K, ch, 10, dev)
+    w_all = synth.normal_weight(40000, K, 11, dev)
+    g = synth.norm_gamma(K, 12, dev)
+    for rows, w_rows in [(40000, 1), (40000, 40), (20000, 2000), (9000, 9000), (2000, 20000), (1, 40000), (37, 333)]:
+        a, w = a_all[:rows], w_all[:w_rows]
+        ax, aw = sq.sq_calibrate_absmax_pair(a, w, norm_gamma=g, eps=1e-6)
+        rx = sq.sq_calibrate_absmax(a, norm_gamma=g, eps=1e-6)
+        rw = sq.sq_calibrate_absmax(w)
+        assert torch.equal(ax, rx) and torch.equal(aw, rw), (rows, w_rows)
+    ok_status(sq)
+
+
 # The CTA-pair GEMM (cta_group::2, 256 x 256 tiles) against the single-SM form and the oracle:
 # ragged T and N, K not a multiple of the 128-byte stage, bias on and off, and T below 256 (which
 # keeps the single-SM form even when pairs are enabled).
