@@ -19,7 +19,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 # parity tests that reach every row-kernel mode and geometry, every GEMM form and the folds
 SUBSET = " or ".join([
-    "single_linear_full", "block_prefill_groups", "edge_shapes", "extreme_codes", "absmax_strided",
+    "single_linear_full", "block_prefill_groups", "edge_shapes", "extreme_codes", "absmax_strided", "absmax_pair",
     "cta_pair_gemm", "decode_form_buckets", "static_scale_path", "fold_into_prev_linear", "fp8_path",
     "layernorm_fold_path", "layer_object", "layer_fold_into_previous",
 ])
