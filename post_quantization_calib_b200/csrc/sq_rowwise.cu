@@ -58,6 +58,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <cmath>
 #include <mutex>
 
 #include "sq_device.cuh"
@@ -966,7 +967,8 @@ sq_status dispatch_rows(const RowArgs &a, int dev, cudaStream_t st) {
 // Relative cost of a row of the plain abs-max against a row of the RMSNorm-fed one (same length): the
 // plain rows only stream through the ring, the norm-fed ones are bound by their per-element work. On a
 // B200, 4096-element rows: a CTA streams plain rows at ~82 GB/s and RMSNorm-fed rows at ~32 GB/s; a
-// 65536 + 4096 row pair ran in 205.7 / 117.9 / 121.9 / 128.3 us with 2 / 4 / 8 / 16 weight CTAs.
+// 65536 + 4096 row pair ran in 205.7 / 117.9 / 121.9 / 128.3 us with 2 / 4 / 8 / 16 weight CTAs, and
+// 262144 + 28672 rows of 8192 elements took 910 us with 6 weight CTAs (the weight side the slower).
 constexpr double kPlainRowCost = 0.4;
 
 template <int WPR, int VPL, int R, bool NORM_A, bool FULL>
@@ -1044,7 +1046,9 @@ sq_status launch_pair_t(RowArgs a, RowArgs w, const Geo &geo, int dev, cudaStrea
     if (ca + cw > wave) {
         const double cost_a = static_cast<double>(a.rows);
         const double cost_w = (NORM_A ? kPlainRowCost : 1.0) * static_cast<double>(w.rows);
-        int64_t share_w = static_cast<int64_t>(static_cast<double>(wave) * cost_w / (cost_a + cost_w) / csz + 0.5) * csz;
+        // rounded up to whole clusters: a weight CTA too few slows the whole launch by the weight's
+        // share of its rows, a CTA too many takes one of the many calibration CTAs
+        int64_t share_w = static_cast<int64_t>(std::ceil(static_cast<double>(wave) * cost_w / (cost_a + cost_w) / csz)) * csz;
         share_w = share_w < csz ? csz : share_w > wave - csz ? wave - csz : share_w;
         cw = ww < share_w ? ww : share_w;
         ca = wa < wave - cw ? wa : wave - cw;

@@ -94,7 +94,7 @@ class SmoothedW8A8Linear:
         self._seen += 1
 
     def finalize(self, reduce_max: Optional[Callable[[torch.Tensor], None]] = None, alpha: Optional[float] = None,
-                 smooth: bool = True, stream=None) -> None:
+                 smooth: bool = True, stream=None, *, _weight_absmax_done: bool = False) -> None:
         """Weight abs-max, smoothing factors, fold and the quantised weight.
 
         reduce_max: in-place max-reduction of the activation abs-max across data-parallel ranks
@@ -103,7 +103,8 @@ class SmoothedW8A8Linear:
         """
         if reduce_max is not None:
             reduce_max(self.amax_x)
-        sq.sq_calibrate_absmax(self.weight, amax=self.amax_w, accumulate=False, stream=stream)
+        if not _weight_absmax_done:
+            sq.sq_calibrate_absmax(self.weight, amax=self.amax_w, accumulate=False, stream=stream)
         a = self.alpha if alpha is None else float(alpha)
         sq.sq_compute_scales(self.amax_x, self.amax_w, a, gamma=self.gamma, s=self.s, fold=self.fold, stream=stream)
         if not smooth:
@@ -125,9 +126,18 @@ class SmoothedW8A8Linear:
         calibration batches a second time, for the maximum of the activation as it is quantised."""
         batches = list(batches)
         self._seen = 0
-        for b in batches:
-            self.observe(b, stream=stream)
-        self.finalize(reduce_max=reduce_max, stream=stream)
+        # the first batch and the weight share one launch (both maxima overwritten); LayerNorm-fed
+        # inputs take their own calibration kernel
+        paired = bool(batches) and self.norm != "layer"
+        for i, b in enumerate(batches):
+            if i == 0 and paired:
+                sq.sq_calibrate_absmax_pair(b, self.weight, norm_gamma=self.gamma if self.norm == "rms" else None,
+                                            eps=self.eps, amax=self.amax_x, amax_w=self.amax_w, accumulate=False,
+                                            stream=stream)
+                self._seen += 1
+            else:
+                self.observe(b, stream=stream)
+        self.finalize(reduce_max=reduce_max, stream=stream, _weight_absmax_done=paired)
         if self.scheme == "int8_static":
             if self.norm == "rms":
                 amax_y = torch.empty(self.K, dtype=torch.float32, device=self.weight.device)
