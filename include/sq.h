@@ -100,9 +100,9 @@ sq_status sq_calibrate_absmax(const void *a, int64_t rows, int64_t cols, int64_t
  * launched one after the other.
  * a, rows, ld, norm_gamma, eps, amax: as in sq_calibrate_absmax.
  * w          bf16 [w_rows, cols], row stride w_ld elements (a weight stored [N, K]); never normalised.
- * amax_w     fp32 [cols], in/out; a different array from amax.
+ * amax_w     fp32 [cols], in/out; must not overlap amax.
  * accumulate applies to both outputs (0 overwrites both, 1 keeps both running maxima).
- * Requirements: those of sq_calibrate_absmax for each input; amax != amax_w (else
+ * Requirements: those of sq_calibrate_absmax for each input; amax and amax_w disjoint (else
  * SQ_ERR_INVALID_ARG).
  */
 sq_status sq_calibrate_absmax_pair(const void *a, int64_t rows, int64_t cols, int64_t ld, const float *norm_gamma,

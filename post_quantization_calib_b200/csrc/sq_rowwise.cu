@@ -1145,7 +1145,8 @@ sq_status sq_calibrate_absmax_pair(const void *a, int64_t rows, int64_t cols, in
     if (c == SQ_OK) c = check_absmax_input(fn, "w", w, w_rows, cols, w_ld, amax_w);
     if (c != SQ_OK) return c;
     if (norm_gamma && !sq::aligned(norm_gamma, 16)) return fail(SQ_ERR_MISALIGNED, "%s: norm_gamma must be 16-byte aligned", fn);
-    if (amax == amax_w) return fail(SQ_ERR_INVALID_ARG, "%s: amax and amax_w must be different arrays", fn);
+    if (amax < amax_w + cols && amax_w < amax + cols)
+        return fail(SQ_ERR_INVALID_ARG, "%s: amax and amax_w must not overlap", fn);
     int dev = 0;
     SQ_TRY_ARCH(dev);
     cudaStream_t st = sq::as_stream(stream);

@@ -152,6 +152,8 @@ def test_absmax_pair_argument_checks(sqmod):
     assert c(FAKE, 4, 64, 64, None, 1e-6, None, FAKE, 4, 64, G, 0, None) == SQ_ERR_INVALID_ARG     # amax NULL
     assert c(FAKE, 4, 64, 64, None, 1e-6, G, FAKE, 4, 64, None, 0, None) == SQ_ERR_INVALID_ARG     # amax_w NULL
     assert c(FAKE, 4, 64, 64, None, 1e-6, G, FAKE, 4, 64, G, 0, None) == SQ_ERR_INVALID_ARG        # same array
+    assert c(FAKE, 4, 64, 64, None, 1e-6, G, FAKE, 4, 64, G + 4 * 63, 0, None) == SQ_ERR_INVALID_ARG  # overlap
+    assert c(FAKE, 4, 64, 64, None, 1e-6, G + 4 * 63, FAKE, 4, 64, G, 0, None) == SQ_ERR_INVALID_ARG  # overlap
     assert c(FAKE, 4, 64, 64, None, 1e-6, G, FAKE, 4, 32, G + 256, 0, None) == SQ_ERR_INVALID_ARG  # w_ld < cols
     assert c(FAKE, 4, 64, 64, None, 1e-6, G, None, 4, 64, G + 256, 0, None) == SQ_ERR_INVALID_ARG  # w NULL with rows
     assert c(FAKE, 4, 64, 64, None, 1e-6, G, FAKE, -1, 64, G + 256, 0, None) == SQ_ERR_INVALID_ARG # w_rows < 0
