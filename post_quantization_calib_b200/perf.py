@@ -1,0 +1,169 @@
+"""Per-workload timing of every stage of the smoothed W8A8 path: one JSON line per workload, group and stage.
+
+    python -m post_quantization_calib_b200.perf [--workload NAME ...] [--reps 20]
+
+Each stage runs through the C ABI on the workload's seeded synthetic inputs (``synth``), resident in HBM:
+  calib_absmax_pair  S1 + S2: column abs-max of the calibration set (of its RMSNorm output when norm-fed)
+                     and of the group's weight, one launch
+  scales             S3: smoothing factors and the folded norm weight
+  weight_quant       S4: diag(s) W quantised to INT8 per output channel
+  act_quant          S5: fused RMSNorm(gamma / s) + per-token INT8 of the workload's T tokens
+  gemm               S6 + S7: INT8 GEMM with the dequant epilogue to bf16
+Decode workloads add act_quant and gemm at each decode token count, once as a single call and once per
+call in a chain of 8 back-to-back calls captured in a CUDA graph (the way a decoder runs one layer after
+another, without the host's per-call cost).
+
+Times are medians of CUDA-event intervals on the launching stream, with the L2 flushed (a 256 MB write)
+before every repetition of a single call. Rates are algorithmic bytes (or 2 x multiply-adds) over that
+time, also given as fractions of the HBM copy bandwidth and of the dense INT8 reference (2 x the bf16
+GEMM burst) measured on the machine (``MEASURED_PEAKS.json`` at the repository root; else a fallback
+pair, marked as such).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import sys
+from typing import Callable, Dict, List, Optional
+
+import torch
+
+from . import sq, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+INT8_PER_BF16 = 2.0          # nominal dense INT8 / bf16 tensor throughput of the B200
+
+
+def load_peaks() -> Dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]), "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+class Timer:
+    """CUDA-event medians on the current stream, L2 flushed before each repetition."""
+
+    def __init__(self, device, reps: int):
+        self.reps = reps
+        self.flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+
+    def single(self, fn: Callable[[], None]) -> float:
+        fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(self.reps)]
+        for a, b in ev:
+            self.flush.fill_(1.0)
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        t = sorted(a.elapsed_time(b) * 1e3 for a, b in ev)
+        return t[len(t) // 2]
+
+    def chained(self, fn: Callable[[], None], calls: int = 8) -> float:
+        """Microseconds per call of `calls` back-to-back calls captured in one CUDA graph (so that the
+        host's per-call cost does not enter), median over the repetitions."""
+        fn()                                   # first call: the library's per-device set-up
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(graph, stream=side):
+            for _ in range(calls):
+                fn()
+        graph.replay()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(self.reps)]
+        for a, b in ev:
+            self.flush.fill_(1.0)
+            a.record()
+            graph.replay()
+            b.record()
+        torch.cuda.synchronize()
+        t = sorted(a.elapsed_time(b) * 1e3 / calls for a, b in ev)
+        return t[len(t) // 2]
+
+
+def line(peaks: Dict, workload: str, group: int, stage: str, us: float, nbytes: int,
+         ops: Optional[int] = None, **extra) -> Dict:
+    out = {"workload": workload, "group": group, "stage": stage, **extra, "us": round(us, 2),
+           "gbs": round(nbytes / us / 1e3, 1), "frac_hbm": round(nbytes / us / 1e3 / peaks["hbm_gbs"], 3)}
+    if ops is not None:
+        int8 = peaks["bf16_tflops"] * INT8_PER_BF16
+        out["tops"] = round(ops / us / 1e6, 1)
+        out["frac_int8"] = round(ops / us / 1e6 / int8, 3)
+    out["peaks"] = peaks["source"]
+    return out
+
+
+def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device) -> List[Dict]:
+    rows: List[Dict] = []
+    K = w.K
+    for g in range(w.groups):
+        N = w.group_N(g)
+        d = synth.group_inputs(w, g, device)
+        gamma, W, X, bias = d["gamma"], d["weight"], d["x"], d["bias"]
+        calib = torch.cat(list(synth.calibration_chunks(w, d["channels"], device, group=g)))
+        R = calib.shape[0]
+        amax = torch.empty(K, dtype=torch.float32, device=device)
+        aw = torch.empty(K, dtype=torch.float32, device=device)
+        us = timer.single(lambda: sq.sq_calibrate_absmax_pair(calib, W, norm_gamma=gamma, eps=w.eps, amax=amax,
+                                                              amax_w=aw))
+        rows.append(line(peaks, w.name, g, "calib_absmax_pair", us, 2 * R * K + 2 * N * K + 12 * K, rows=R, N=N, K=K))
+        s = torch.empty(K, dtype=torch.float32, device=device)
+        fold = torch.empty(K, dtype=torch.float32, device=device)
+        us = timer.single(lambda: sq.sq_compute_scales(amax, aw, w.alpha, gamma=gamma, s=s, fold=fold))
+        rows.append(line(peaks, w.name, g, "scales", us, 20 * K, K=K))
+        wq = torch.empty(N, K, dtype=torch.int8, device=device)
+        ws = torch.empty(N, dtype=torch.float32, device=device)
+        us = timer.single(lambda: sq.sq_smooth_quantize_weight(W, s, wq=wq, w_scale=ws))
+        rows.append(line(peaks, w.name, g, "weight_quant", us, 3 * N * K + 4 * K + 4 * N, N=N, K=K))
+        token_counts = [w.T] + [t for t in w.decode_T if t != w.T]
+        for T in token_counts:
+            x = X[:T] if T <= X.shape[0] else synth.outlier_tokens(T, K, d["channels"], synth.seed_for(w.index, "x", g), device)
+            xq = torch.empty(T, K, dtype=torch.int8, device=device)
+            xs = torch.empty(T, dtype=torch.float32, device=device)
+            y = torch.empty(T, N, dtype=torch.bfloat16, device=device)
+            quant = lambda: sq.sq_rmsnorm_smooth_quant(x, fold, eps=w.eps, apply_norm=w.norm, xq=xq, x_scale=xs)
+            gemm = lambda: sq.sq_w8a8_linear(xq, xs, wq, ws, bias=bias, y=y)
+            qbytes = 3 * T * K + 4 * K + 4 * T
+            gbytes = T * K + N * K + 2 * T * N + 4 * T + 4 * N + (2 * N if bias is not None else 0)
+            ops = 2 * T * N * K
+            rows.append(line(peaks, w.name, g, "act_quant", timer.single(quant), qbytes, T=T, K=K))
+            rows.append(line(peaks, w.name, g, "gemm", timer.single(gemm), gbytes, ops, T=T, N=N, K=K))
+            if T in w.decode_T:
+                rows.append(line(peaks, w.name, g, "act_quant", timer.chained(quant), qbytes, T=T, K=K, chain=8))
+                rows.append(line(peaks, w.name, g, "gemm", timer.chained(gemm), gbytes, ops, T=T, N=N, K=K, chain=8))
+        del calib
+        torch.cuda.empty_cache()
+    st = sq.sq_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {sq.sq_status_string(st)} after workload {w.name}")
+    return rows
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--workload", action="append", help="workload name (repeatable; default: all five)")
+    ap.add_argument("--reps", type=int, default=20)
+    args = ap.parse_args(argv)
+    if not torch.cuda.is_available():
+        print("perf: needs a CUDA device", file=sys.stderr)
+        return 2
+    device = torch.device("cuda", torch.cuda.current_device())
+    peaks = load_peaks()
+    timer = Timer(device, args.reps)
+    names = args.workload or [w.name for w in synth.WORKLOADS]
+    for n in names:
+        for r in run_workload(synth.workload(n), timer, peaks, device):
+            print(json.dumps(r), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -21,7 +21,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SUBSET = " or ".join([
     "single_linear_full", "block_prefill_groups", "edge_shapes", "extreme_codes", "absmax_strided", "absmax_pair",
     "cta_pair_gemm", "decode_form_buckets", "static_scale_path", "fold_into_prev_linear", "fp8_path",
-    "layernorm_fold_path", "layer_object", "layer_fold_into_previous",
+    "layernorm_fold_path", "layer_object", "layer_fold_into_previous", "quantisers_over_few_rows",
 ])
 
 SELFTEST = """

@@ -314,6 +314,45 @@ def test_absmax_pair_matches_two_calls_at_every_split(sq):
     ok_status(sq)
 
 
+# Quantisers over few rows (decode-sized token counts) take one row per group of eight warps, up to 4
+# rows per SM; every quantiser mode against the oracle at token counts on both sides of that bound
+# (592 rows on 148 SMs), at widths whose rows fill the eight-warp group exactly (4096, 8192) or not
+# (2568, 6144).
+FEW_ROWS = [(1, 4096), (7, 2568), (64, 8192), (300, 6144), (592, 4096), (593, 4096)]
+
+
+@pytest.mark.parametrize("T,K", FEW_ROWS)
+def test_quantisers_over_few_rows(sq, orc, T, K):
+    dev = "cuda"
+    ch = synth.outlier_channels(K, synth.OutlierSpec(max(1, K // 256), 10, 40), 21)
+    x = synth.outlier_tokens(T, K, ch, 22, dev)
+    fold = synth.norm_gamma(K, 23, dev)
+    x_h, f_h = h16(x), hnp(fold)
+    for norm in (True, False):
+        q, sc = sq.sq_rmsnorm_smooth_quant(x, fold, apply_norm=norm)
+        rq, rs = orc.rmsnorm_smooth_quant(x_h, f_h, apply_norm=norm)
+        assert np.array_equal(hnp(q), rq) and np.array_equal(hnp(sc), rs)
+        q, sc = sq.sq_rmsnorm_smooth_quant_fp8(x, fold, apply_norm=norm)
+        rq, rs = orc.rmsnorm_smooth_quant_f8(x_h, f_h, apply_norm=norm)
+        assert np.array_equal(hnp(q), rq) and np.array_equal(hnp(sc), rs)
+    amax_y = np.full(K, 2.0, np.float32)
+    amax_y[K // 3] = 6.0                                # values past the calibrated maximum are clipped
+    s2 = orc.static_scale(amax_y)
+    for norm in (True, False):
+        q, sc = sq.sq_rmsnorm_smooth_quant_static(x, fold, torch.from_numpy(s2).to(dev), apply_norm=norm)
+        rq, rs = orc.rmsnorm_smooth_quant_static(x_h, f_h, s2, apply_norm=norm)
+        assert np.array_equal(hnp(q), rq) and np.array_equal(hnp(sc), rs)
+    beta = synth.norm_gamma(K, 24, dev) - 1.0
+    q, sc = sq.sq_layernorm_smooth_quant(x + 3, fold, beta)
+    rq, rs = orc.layernorm_smooth_quant(h16(x + 3), f_h, hnp(beta))
+    assert np.array_equal(hnp(q), rq) and np.array_equal(hnp(sc), rs)
+    w = synth.normal_weight(T, K, 25, dev)              # a weight with as few output channels
+    q, sc = sq.sq_smooth_quantize_weight(w, fold)
+    rq, rs = orc.smooth_quantize_weight(h16(w), f_h)
+    assert np.array_equal(hnp(q), rq) and np.array_equal(hnp(sc), rs)
+    ok_status(sq)
+
+
 # The CTA-pair GEMM (cta_group::2, 256 x 256 tiles) against the single-SM form and the oracle:
 # ragged T and N, K not a multiple of the 128-byte stage, bias on and off, and T below 256 (which
 # keeps the single-SM form even when pairs are enabled).

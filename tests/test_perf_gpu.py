@@ -1,0 +1,40 @@
+"""The per-workload timing tool: one JSON line per stage with positive times and rates (GPU), and a clean
+exit without a device (CPU)."""
+import io
+import json
+from contextlib import redirect_stdout
+
+import pytest
+import torch
+
+
+def test_perf_needs_a_device():
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    from post_quantization_calib_b200 import perf
+    assert perf.main(["--workload", "single_linear_t256_k1024_n1024", "--reps", "2"]) == 2
+
+
+@pytest.mark.gpu
+def test_perf_lines_for_the_smallest_and_the_decode_workload():
+    from post_quantization_calib_b200 import build
+    build.build()
+    from post_quantization_calib_b200 import perf
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        rc = perf.main(["--workload", "single_linear_t256_k1024_n1024", "--workload", "decode_k4096_n14336",
+                        "--reps", "3"])
+    assert rc == 0
+    rows = [json.loads(l) for l in buf.getvalue().splitlines() if l.strip()]
+    stages = {(r["workload"], r["stage"], r.get("T"), r.get("chain")) for r in rows}
+    for st in ("calib_absmax_pair", "scales", "weight_quant"):
+        assert ("single_linear_t256_k1024_n1024", st, None, None) in stages
+    assert ("single_linear_t256_k1024_n1024", "gemm", 256, None) in stages
+    for T in (1, 8, 32, 64):
+        assert ("decode_k4096_n14336", "gemm", T, None) in stages
+        assert ("decode_k4096_n14336", "gemm", T, 8) in stages
+        assert ("decode_k4096_n14336", "act_quant", T, 8) in stages
+    for r in rows:
+        assert r["us"] > 0 and r["gbs"] > 0 and r["peaks"] in ("measured", "fallback")
+        if r["stage"] == "gemm":
+            assert r["tops"] > 0
