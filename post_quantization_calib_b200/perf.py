@@ -11,10 +11,12 @@ Each stage runs through the C ABI on the workload's seeded synthetic inputs (``s
   gemm               S6 + S7: INT8 GEMM with the dequant epilogue to bf16
 Decode workloads add act_quant and gemm at each decode token count, once as a single call and once per
 call in a chain of 8 back-to-back calls captured in a CUDA graph (the way a decoder runs one layer after
-another, without the host's per-call cost).
+another, without the host's per-call cost; the 8 GEMMs read 8 distinct copies of the weight, which
+together exceed the L2). The GEMM chain is also timed issued call by call on the stream ("chain_form":
+"stream"), where each call's dependent launch overlaps the previous call's end.
 
-Times are medians of CUDA-event intervals on the launching stream, with the L2 flushed (a 256 MB write)
-before every repetition of a single call. Rates are algorithmic bytes (or 2 x multiply-adds) over that
+Times are medians of CUDA-event intervals on the launching stream, with the L2 flushed (a 256 MB read)
+before every repetition. Rates are algorithmic bytes (or 2 x multiply-adds) over that
 time, also given as fractions of the HBM copy bandwidth and of the dense INT8 reference (2 x the bf16
 GEMM burst) measured on the machine (``MEASURED_PEAKS.json`` at the repository root; else a fallback
 pair, marked as such).
@@ -46,18 +48,23 @@ def load_peaks() -> Dict:
 
 
 class Timer:
-    """CUDA-event medians on the current stream, L2 flushed before each repetition."""
+    """CUDA-event medians on the current stream, L2 flushed before each repetition by reading a 256 MB
+    buffer (a read leaves clean lines, so no write-back of the flush lands inside the timed call)."""
 
     def __init__(self, device, reps: int):
         self.reps = reps
-        self.flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+        self.flush = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+        self.sink = torch.empty((), dtype=torch.float32, device=device)
+
+    def clear_l2(self) -> None:
+        torch.sum(self.flush, dim=0, out=self.sink)
 
     def single(self, fn: Callable[[], None]) -> float:
         fn()
         torch.cuda.synchronize()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(self.reps)]
         for a, b in ev:
-            self.flush.fill_(1.0)
+            self.clear_l2()
             a.record()
             fn()
             b.record()
@@ -65,22 +72,41 @@ class Timer:
         t = sorted(a.elapsed_time(b) * 1e3 for a, b in ev)
         return t[len(t) // 2]
 
-    def chained(self, fn: Callable[[], None], calls: int = 8) -> float:
-        """Microseconds per call of `calls` back-to-back calls captured in one CUDA graph (so that the
-        host's per-call cost does not enter), median over the repetitions."""
-        fn()                                   # first call: the library's per-device set-up
+    def stream_chained(self, fns: List[Callable[[], None]]) -> float:
+        """Microseconds per call of the calls `fns` issued back to back on the stream (each call may
+        start while the previous one finishes), median over the repetitions. Only meaningful where a
+        call takes longer on the device than on the host."""
+        for fn in fns:
+            fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(self.reps)]
+        for a, b in ev:
+            self.clear_l2()
+            a.record()
+            for fn in fns:
+                fn()
+            b.record()
+        torch.cuda.synchronize()
+        t = sorted(a.elapsed_time(b) * 1e3 / len(fns) for a, b in ev)
+        return t[len(t) // 2]
+
+    def chained(self, fns: List[Callable[[], None]]) -> float:
+        """Microseconds per call of the calls `fns`, back to back, captured in one CUDA graph (so that
+        the host's per-call cost does not enter), median over the repetitions."""
+        calls = len(fns)
+        fns[0]()                               # first call: the library's per-device set-up
         torch.cuda.synchronize()
         graph = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
         with torch.cuda.graph(graph, stream=side):
-            for _ in range(calls):
+            for fn in fns:
                 fn()
         graph.replay()
         torch.cuda.synchronize()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(self.reps)]
         for a, b in ev:
-            self.flush.fill_(1.0)
+            self.clear_l2()
             a.record()
             graph.replay()
             b.record()
@@ -137,8 +163,15 @@ def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device) -> List[D
             rows.append(line(peaks, w.name, g, "act_quant", timer.single(quant), qbytes, T=T, K=K))
             rows.append(line(peaks, w.name, g, "gemm", timer.single(gemm), gbytes, ops, T=T, N=N, K=K))
             if T in w.decode_T:
-                rows.append(line(peaks, w.name, g, "act_quant", timer.chained(quant), qbytes, T=T, K=K, chain=8))
-                rows.append(line(peaks, w.name, g, "gemm", timer.chained(gemm), gbytes, ops, T=T, N=N, K=K, chain=8))
+                # a decoder's consecutive layers: each GEMM streams its own weight (8 together exceed
+                # the L2); the activations are small and stay in L2 either way
+                wqs = [wq] + [wq.clone() for _ in range(7)]
+                gemms = [lambda m=m: sq.sq_w8a8_linear(xq, xs, m, ws, bias=bias, y=y) for m in wqs]
+                rows.append(line(peaks, w.name, g, "act_quant", timer.chained([quant] * 8), qbytes, T=T, K=K, chain=8))
+                rows.append(line(peaks, w.name, g, "gemm", timer.chained(gemms), gbytes, ops, T=T, N=N, K=K, chain=8))
+                rows.append(line(peaks, w.name, g, "gemm", timer.stream_chained(gemms), gbytes, ops, T=T, N=N, K=K,
+                                 chain=8, chain_form="stream"))
+                del wqs, gemms
         del calib
         torch.cuda.empty_cache()
     st = sq.sq_device_status()

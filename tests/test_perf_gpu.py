@@ -27,6 +27,7 @@ def test_perf_lines_for_the_smallest_and_the_decode_workload():
     assert rc == 0
     rows = [json.loads(l) for l in buf.getvalue().splitlines() if l.strip()]
     stages = {(r["workload"], r["stage"], r.get("T"), r.get("chain")) for r in rows}
+    forms = {(r["stage"], r.get("T"), r.get("chain_form")) for r in rows if r.get("chain")}
     for st in ("calib_absmax_pair", "scales", "weight_quant"):
         assert ("single_linear_t256_k1024_n1024", st, None, None) in stages
     assert ("single_linear_t256_k1024_n1024", "gemm", 256, None) in stages
@@ -34,6 +35,7 @@ def test_perf_lines_for_the_smallest_and_the_decode_workload():
         assert ("decode_k4096_n14336", "gemm", T, None) in stages
         assert ("decode_k4096_n14336", "gemm", T, 8) in stages
         assert ("decode_k4096_n14336", "act_quant", T, 8) in stages
+        assert ("gemm", T, "stream") in forms and ("gemm", T, None) in forms
     for r in rows:
         assert r["us"] > 0 and r["gbs"] > 0 and r["peaks"] in ("measured", "fallback")
         if r["stage"] == "gemm":
