@@ -569,3 +569,37 @@ def test_smoothing_reduces_error_on_outlier_data(orc):
 
     s, _ = orc.compute_scales(orc.calibrate_absmax(x), orc.calibrate_absmax(w), 0.5)
     assert err(s) < 0.7 * err(None)
+
+
+def test_alpha_sweet_spot_and_traps(orc):
+    # The alpha sweep of "SmoothQuant and W8A8: Quantizing Activations Too", One layer, measured
+    # (weights per output channel, activations on one static per-tensor scale from the calibration
+    # maximum): alpha has a best middle range and two traps. Too small an alpha rescales channels by
+    # their weights' range rather than flattening the activations, which is worse than no smoothing
+    # when the outlier channels also carry the larger weights (built here: 2x weights there); too
+    # large an alpha moves the range into the weights, whose quantisation error then dominates.
+    K, N, T = 512, 128, 256
+    ch = synth.outlier_channels(K, synth.OutlierSpec(16, 10.0, 25.0, pinned=25.0), 41)
+    x = bf16_bits(synth.outlier_tokens(T, K, ch, 42))
+    wt = synth.normal_weight(N, K, 43).float()
+    wt[:, ch[0]] *= 2.0
+    w = bf16_bits(wt.to(torch.bfloat16))
+    exact = bits_to_f64(x) @ bits_to_f64(w).T
+    ax, aw = orc.calibrate_absmax(x), orc.calibrate_absmax(w)
+
+    def err(alpha):
+        if alpha is None:
+            s, fold = None, np.ones(K, np.float32)
+        else:
+            s, _ = orc.compute_scales(ax, aw, alpha)
+            fold = (np.float32(1.0) / s).astype(np.float32)
+        wq, ws = orc.smooth_quantize_weight(w, s)
+        amax_y = (ax * fold).astype(np.float32)     # max |x * f| = fl(max |x| * f), rounding being monotone
+        xq, xs = orc.rmsnorm_smooth_quant_static(x, fold, orc.static_scale(amax_y), apply_norm=False)
+        y, _ = orc.w8a8_linear(xq, xs, wq, ws)
+        return np.linalg.norm(bits_to_f64(y) - exact) / np.linalg.norm(exact)
+
+    none, low, mid, high = err(None), err(0.1), err(0.7), err(1.0)
+    assert mid < 0.5 * none            # the sweet spot
+    assert low > none                  # too little: worse than no smoothing
+    assert high > 2.0 * mid            # too much: the weights' error takes over
