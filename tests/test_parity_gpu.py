@@ -641,6 +641,52 @@ def test_online_path_in_cuda_graph(sq):
         assert torch.equal(xq, xq_e) and torch.equal(xs, xs_e) and torch.equal(y_graph, y_e)
 
 
+def test_offline_path_in_cuda_graph(sq):
+    """The offline steps (the abs-max pair after its zero-fill, the scales, the weight quantiser)
+    captured once in a CUDA graph and replayed on new calibration rows and weights: every output equals
+    the one of direct calls."""
+    dev = "cuda"
+    w = synth.WORKLOADS[1]
+    d = synth.group_inputs(w, 0, dev, T=2048)
+    gamma, W0, X0 = d["gamma"], d["weight"], d["x"]
+    cal, wt = X0.clone(), W0.clone()
+    K, N = W0.shape[1], W0.shape[0]
+    amax = torch.empty(K, device=dev)
+    aw = torch.empty(K, device=dev)
+    s = torch.empty(K, device=dev)
+    fold = torch.empty(K, device=dev)
+    wq = torch.empty(N, K, dtype=torch.int8, device=dev)
+    ws = torch.empty(N, device=dev)
+
+    def offline():
+        sq.sq_calibrate_absmax_pair(cal, wt, norm_gamma=gamma, amax=amax, amax_w=aw)
+        sq.sq_compute_scales(amax, aw, 0.5, gamma=gamma, s=s, fold=fold)
+        sq.sq_smooth_quantize_weight(wt, s, wq=wq, w_scale=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        offline()                                  # warm-up: one-time launch configuration
+    torch.cuda.current_stream().wait_stream(side)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        offline()
+    for k in range(3):
+        cnew = (X0.float() * (1.0 + 0.5 * k) + 0.02 * k).to(torch.bfloat16)
+        wnew = (W0.float() * (1.0 - 0.2 * k)).to(torch.bfloat16)
+        cal.copy_(cnew)
+        wt.copy_(wnew)
+        graph.replay()
+        torch.cuda.synchronize()
+        ax_e, aw_e = sq.sq_calibrate_absmax_pair(cnew, wnew, norm_gamma=gamma)
+        s_e, f_e = sq.sq_compute_scales(ax_e, aw_e, 0.5, gamma=gamma)
+        wq_e, ws_e = sq.sq_smooth_quantize_weight(wnew, s_e)
+        ok_status(sq)
+        assert torch.equal(amax, ax_e) and torch.equal(aw, aw_e)
+        assert torch.equal(s, s_e) and torch.equal(fold, f_e)
+        assert torch.equal(wq, wq_e) and torch.equal(ws, ws_e)
+
+
 # The variant rows at the query-projection size (T 8192, K = N 4096, the calibration set of 65536 rows), in
 # the launch configuration the bench uses for the INT8 path: every code and scale compared with the
 # oracle; the GEMMs on sampled full rows and full columns (INT8: bit-exact; FP8: binary32 summation bound,
