@@ -1,6 +1,7 @@
 """Per-workload timing of every stage of the smoothed W8A8 path: one JSON line per workload, group and stage.
 
-    python -m post_quantization_calib_b200.perf [--workload NAME ...] [--reps 20]
+    python -m post_quantization_calib_b200.perf [--workload NAME ...] [--stage NAME ...] [--tokens T ...]
+                                                [--reps 20]
 
 Each stage runs through the C ABI on the workload's seeded synthetic inputs (``synth``), resident in HBM:
   calib_absmax_pair  S1 + S2: column abs-max of the calibration set (of its RMSNorm output when norm-fed)
@@ -127,7 +128,14 @@ def line(peaks: Dict, workload: str, group: int, stage: str, us: float, nbytes: 
     return out
 
 
-def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device) -> List[Dict]:
+STAGES = ("calib_absmax_pair", "scales", "weight_quant", "act_quant", "gemm")
+
+
+def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device, stages=STAGES,
+                 tokens: Optional[List[int]] = None) -> List[Dict]:
+    """The workload's stages (those in `stages`; the others still run once, untimed, where a later
+    stage needs their output), at the workload's token count and its decode token counts (or at
+    `tokens`)."""
     rows: List[Dict] = []
     K = w.K
     for g in range(w.groups):
@@ -138,18 +146,28 @@ def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device) -> List[D
         R = calib.shape[0]
         amax = torch.empty(K, dtype=torch.float32, device=device)
         aw = torch.empty(K, dtype=torch.float32, device=device)
-        us = timer.single(lambda: sq.sq_calibrate_absmax_pair(calib, W, norm_gamma=gamma, eps=w.eps, amax=amax,
-                                                              amax_w=aw))
-        rows.append(line(peaks, w.name, g, "calib_absmax_pair", us, 2 * R * K + 2 * N * K + 12 * K, rows=R, N=N, K=K))
+        pair = lambda: sq.sq_calibrate_absmax_pair(calib, W, norm_gamma=gamma, eps=w.eps, amax=amax, amax_w=aw)
+        if "calib_absmax_pair" in stages:
+            rows.append(line(peaks, w.name, g, "calib_absmax_pair", timer.single(pair),
+                             2 * R * K + 2 * N * K + 12 * K, rows=R, N=N, K=K))
+        else:
+            pair()
         s = torch.empty(K, dtype=torch.float32, device=device)
         fold = torch.empty(K, dtype=torch.float32, device=device)
-        us = timer.single(lambda: sq.sq_compute_scales(amax, aw, w.alpha, gamma=gamma, s=s, fold=fold))
-        rows.append(line(peaks, w.name, g, "scales", us, 20 * K, K=K))
+        scales = lambda: sq.sq_compute_scales(amax, aw, w.alpha, gamma=gamma, s=s, fold=fold)
+        if "scales" in stages:
+            rows.append(line(peaks, w.name, g, "scales", timer.single(scales), 20 * K, K=K))
+        else:
+            scales()
         wq = torch.empty(N, K, dtype=torch.int8, device=device)
         ws = torch.empty(N, dtype=torch.float32, device=device)
-        us = timer.single(lambda: sq.sq_smooth_quantize_weight(W, s, wq=wq, w_scale=ws))
-        rows.append(line(peaks, w.name, g, "weight_quant", us, 3 * N * K + 4 * K + 4 * N, N=N, K=K))
-        token_counts = [w.T] + [t for t in w.decode_T if t != w.T]
+        wquant = lambda: sq.sq_smooth_quantize_weight(W, s, wq=wq, w_scale=ws)
+        if "weight_quant" in stages:
+            rows.append(line(peaks, w.name, g, "weight_quant", timer.single(wquant), 3 * N * K + 4 * K + 4 * N,
+                             N=N, K=K))
+        else:
+            wquant()
+        token_counts = tokens if tokens else [w.T] + [t for t in w.decode_T if t != w.T]
         for T in token_counts:
             x = X[:T] if T <= X.shape[0] else synth.outlier_tokens(T, K, d["channels"], synth.seed_for(w.index, "x", g), device)
             xq = torch.empty(T, K, dtype=torch.int8, device=device)
@@ -160,9 +178,13 @@ def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device) -> List[D
             qbytes = 3 * T * K + 4 * K + 4 * T
             gbytes = T * K + N * K + 2 * T * N + 4 * T + 4 * N + (2 * N if bias is not None else 0)
             ops = 2 * T * N * K
-            rows.append(line(peaks, w.name, g, "act_quant", timer.single(quant), qbytes, T=T, K=K))
-            rows.append(line(peaks, w.name, g, "gemm", timer.single(gemm), gbytes, ops, T=T, N=N, K=K))
-            if T in w.decode_T:
+            if "act_quant" in stages:
+                rows.append(line(peaks, w.name, g, "act_quant", timer.single(quant), qbytes, T=T, K=K))
+            else:
+                quant()
+            if "gemm" in stages:
+                rows.append(line(peaks, w.name, g, "gemm", timer.single(gemm), gbytes, ops, T=T, N=N, K=K))
+            if T in w.decode_T and "gemm" in stages and "act_quant" in stages:
                 # a decoder's consecutive layers: each GEMM streams its own weight (8 together exceed
                 # the L2); the activations are small and stay in L2 either way
                 wqs = [wq] + [wq.clone() for _ in range(7)]
@@ -183,6 +205,8 @@ def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device) -> List[D
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--workload", action="append", help="workload name (repeatable; default: all five)")
+    ap.add_argument("--stage", action="append", choices=STAGES, help="stage to time (repeatable; default: all)")
+    ap.add_argument("--tokens", action="append", type=int, help="token count (repeatable; default: the workload's)")
     ap.add_argument("--reps", type=int, default=20)
     args = ap.parse_args(argv)
     if not torch.cuda.is_available():
@@ -193,7 +217,8 @@ def main(argv=None) -> int:
     timer = Timer(device, args.reps)
     names = args.workload or [w.name for w in synth.WORKLOADS]
     for n in names:
-        for r in run_workload(synth.workload(n), timer, peaks, device):
+        for r in run_workload(synth.workload(n), timer, peaks, device, stages=tuple(args.stage or STAGES),
+                              tokens=args.tokens):
             print(json.dumps(r), flush=True)
     return 0
 
