@@ -13,6 +13,9 @@ def test_perf_needs_a_device():
         pytest.skip("a device is present")
     from post_quantization_calib_b200 import perf
     assert perf.main(["--workload", "single_linear_t256_k1024_n1024", "--reps", "2"]) == 2
+    assert perf.main(["--stage", "gemm", "--tokens", "1", "--tokens", "64"]) == 2
+    with pytest.raises(SystemExit):
+        perf.main(["--stage", "not_a_stage"])
 
 
 @pytest.mark.gpu
