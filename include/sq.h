@@ -35,6 +35,10 @@
  *     multiply-adds), except the norm sums (binary64: the RMSNorm sum of squares, the LayerNorm sum
  *     and centred sum of squares) and the smoothing-factor power (binary64, rounded once to
  *     binary32). INT8 codes use round-half-away-from-zero and are clamped to [-127, 127].
+ *   - Rows of very small values: every per-row quantiser (weights, tokens, INT8 and FP8) codes a row
+ *     with m = max|v| as round(v * fl(qmax / m)), qmax = 127 (448 for FP8). When qmax / m overflows
+ *     binary32 (m below about 3.7e-37 for INT8, 1.3e-36 for FP8), the row is first multiplied by 2^64
+ *     (exact) and coded as round(fl(v * 2^64) * fl(qmax / fl(m * 2^64))); its scale is still m / qmax.
  */
 #ifndef SQ_H
 #define SQ_H
@@ -161,7 +165,8 @@ sq_status sq_rmsnorm_smooth_quant(const void *x, int64_t T, int64_t K, const flo
  *   layer fed directly: sq_calibrate_absmax(calibration tokens) and factor = fold (= 1/s).
  * Rounding is monotone, so either way m equals the largest |y| the quantiser would form on the
  * calibration tokens. amax fp32 [K]; factor nullable fp32 [K]; scale2 fp32 [2] out (device memory).
- * K >= 1.
+ * K >= 1. When 127 / m overflows binary32 (m below about 3.7e-37), scale2[1] is +infinity: the static
+ * quantiser then codes every zero value 0 and saturates every other value at +-127.
  */
 sq_status sq_static_scale(const float *amax, const float *factor, int64_t K, float *scale2, void *stream);
 
@@ -239,7 +244,9 @@ sq_status sq_layernorm_smooth_quant(const void *x, int64_t T, int64_t K, const f
  * Requirements: T >= 0, N >= 8, N % 8 == 0, K >= 16, K % 16 == 0, K <= 131072; xq, wq, y 16-byte
  * aligned; acc_out 16-byte aligned. The GEMM runs on the tensor cores (tcgen05, TMEM accumulators,
  * TMA-fed shared-memory pipeline); its device-side waits are bounded and report SQ_ERR_TIMEOUT
- * through sq_device_status() instead of hanging.
+ * through sq_device_status() instead of hanging. Output tiles are 128 tokens x 256, 192 or 64
+ * channels (whichever fills the SMs best), or, for T <= 128, 128 channels x 16..128 tokens; every
+ * form computes the same bits.
  */
 sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, const int8_t *wq,
                          const float *w_scale, int64_t N, int64_t K, const void *bias, void *y,
@@ -291,8 +298,9 @@ size_t sq_w8a8_linear_workspace_size(int64_t T, int64_t N, int64_t K);
  * SQ_OK, SQ_ERR_TIMEOUT (a bounded wait in a kernel ran out; the kernel stopped its work and
  * returned, the context stays usable), SQ_ERR_BOUNDS (libsq_checked.so only: a device-side bounds
  * check failed and the access it guards was skipped) or SQ_ERR_CUDA (an asynchronous CUDA error).
- * The first error recorded is kept. Reading the word clears it. The word is shared by every stream
- * on the device.
+ * The first error recorded is kept. The word is shared by every stream on the device; it is read and
+ * cleared in one atomic exchange ordered on `stream` (a one-thread kernel), so an error that a kernel
+ * on another stream records meanwhile is either reported by this call or kept for the next one.
  */
 sq_status sq_device_status(void *stream);
 

@@ -67,10 +67,13 @@ uint16_t orc_f32_to_bf16(float f) { return f32_to_bf16_rne(f); }
 float orc_bf16_to_f32(uint16_t h) { return bf16_to_f32(h); }
 
 /* Symmetric INT8 code of one value, [TAMING] "Why Outliers Break Quantization" (quantisation
- * equation): v / delta rounded to the nearest integer. roundf is C99's round-half-away-from-zero. */
+ * equation): v / delta rounded to the nearest integer. roundf is C99's round-half-away-from-zero.
+ * An infinite inv_delta (a static scale whose 127 / m overflowed) makes t = 0 * inf = NaN for a zero
+ * value: the code of a zero value is 0 whatever the scale. */
 static int8_t quantize_one(float v, float inv_delta)
 {
     float t = v * inv_delta;
+    if (isnan(t)) return 0;
     float r = roundf(t);
     if (r > (float)ORC_QMAX) r = (float)ORC_QMAX;
     if (r < -(float)ORC_QMAX) r = -(float)ORC_QMAX;
@@ -79,7 +82,10 @@ static int8_t quantize_one(float v, float inv_delta)
 
 /* Quantise one row of already-smoothed binary32 values with one symmetric scale:
  * m = max|v|, delta = m / 127, codes = round(v * (127 / m)). A zero row gives delta 0, codes 0.
- * [MIGRATE] section 7 (one scale per output row / per token), [W8A8] "One layer, measured". */
+ * [MIGRATE] section 7 (one scale per output row / per token), [W8A8] "One layer, measured".
+ * When 127 / m overflows binary32 (m below 127 / FLT_MAX, about 3.7e-37), the row is first scaled by
+ * 2^64 -- exact, and the quantiser is scale-free -- so that the reciprocal is finite:
+ * codes = round((v * 2^64) * (127 / (m * 2^64))); delta stays m / 127. */
 static void quantize_row(const float *v, int64_t n, int8_t *q, float *delta_out)
 {
     float m = 0.0f;
@@ -94,7 +100,12 @@ static void quantize_row(const float *v, int64_t n, int8_t *q, float *delta_out)
     }
     float delta = m / (float)ORC_QMAX;
     float inv = (float)ORC_QMAX / m;
-    for (int64_t k = 0; k < n; ++k) q[k] = quantize_one(v[k], inv);
+    float pre = 1.0f;
+    if (isinf(inv)) {
+        pre = 0x1p64f;
+        inv = (float)ORC_QMAX / (m * pre);
+    }
+    for (int64_t k = 0; k < n; ++k) q[k] = quantize_one(v[k] * pre, inv);
     *delta_out = delta;
 }
 
@@ -391,7 +402,8 @@ uint8_t orc_e4m3_encode(float v) { return e4m3_encode(v); }
 float orc_e4m3_decode(uint8_t c) { return e4m3_decode(c); }
 
 /* One row of smoothed binary32 values to E4M3 with one scale: m = max|v|, delta = m / 448,
- * codes e4m3(v * fl32(448 / m)); a zero row gives delta 0 and codes 0. */
+ * codes e4m3(v * fl32(448 / m)); a zero row gives delta 0 and codes 0. When 448 / m overflows
+ * binary32 (m below 448 / FLT_MAX), the row is first scaled by 2^64 (exact), as in the INT8 quantiser. */
 static void quantize_row_f8(const float *v, int64_t n, uint8_t *q, float *delta_out)
 {
     float m = 0.0f;
@@ -405,7 +417,12 @@ static void quantize_row_f8(const float *v, int64_t n, uint8_t *q, float *delta_
         return;
     }
     float inv = ORC_F8MAX / m;
-    for (int64_t k = 0; k < n; ++k) q[k] = e4m3_encode(v[k] * inv);
+    float pre = 1.0f;
+    if (isinf(inv)) {
+        pre = 0x1p64f;
+        inv = ORC_F8MAX / (m * pre);
+    }
+    for (int64_t k = 0; k < n; ++k) q[k] = e4m3_encode((v[k] * pre) * inv);
     *delta_out = m / ORC_F8MAX;
 }
 

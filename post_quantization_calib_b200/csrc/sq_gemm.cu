@@ -47,6 +47,8 @@ namespace {
 
 // Device-side status word: 0 or the first sq_status a kernel recorded.
 __device__ unsigned int g_sq_status;
+// The status word's value at the moment sq_device_status read and cleared it.
+__device__ unsigned int g_sq_status_read;
 
 // Host-side choice of the GEMM form (sq_set_gemm_cta_pair).
 std::atomic<int> g_cta_pair{0};
@@ -102,8 +104,10 @@ struct Tile {
     static constexpr int B_SLOT = KS * B_SLICE;
     static constexpr int SPARE = 232448 - 1024 - EPI_WARPS * 2 * OUT_BOX - 2 * COL_TAB - 512;
     static constexpr int STAGES = SWAP ? (SPARE / (A_SLOT + B_SLOT) > 11 ? 11 : SPARE / (A_SLOT + B_SLOT))
-                                       : TN == 256 ? 4 : 8;
-    static constexpr uint32_t TMEM_COLS = 2 * TN;          // two accumulators; a power of two >= 32
+                                       : (SPARE / (A_SLOT + B_SLOT) > 8 ? 8 : SPARE / (A_SLOT + B_SLOT));   // 256: 4, 192: 5, 64: 8
+    // two accumulators ACC_STRIDE columns apart; the allocation is a power of two >= 32 columns
+    static constexpr uint32_t TMEM_COLS = TN == 192 ? 512u : 2u * TN;
+    static constexpr uint32_t ACC_STRIDE = TMEM_COLS / 2;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_SLOT;
     static constexpr int OFF_OUT = OFF_B + STAGES * B_SLOT;
@@ -116,7 +120,7 @@ struct Tile {
     static constexpr uint32_t IDESC_F8 = make_idesc_f8(BM, TN);
     static_assert(SMEM_TOTAL <= 232448, "shared memory budget of one sm_100 CTA");
     static_assert(SWAP ? (TN >= 16 && TN <= 128 && (TN & (TN - 1)) == 0)
-                       : (TN % OUT_COLS == 0 && TN >= 32 && TN <= 256 && (TN & (TN - 1)) == 0), "tile width");
+                       : (TN % OUT_COLS == 0 && TN >= 32 && TN <= 256 && ((TN & (TN - 1)) == 0 || TN == 192)), "tile width");
 };
 
 // ------------------------------------------------------------------------------------------------
@@ -240,6 +244,17 @@ __device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) 
         : "r"(bar), "r"(parity)
         : "memory");
     return ok != 0;
+}
+// Lowers the pending transaction count of the current phase of `bar` by `bytes` (bytes that were
+// expected but will never arrive).
+__device__ __forceinline__ void mbar_complete_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// 64-bit load from shared memory of a CTA of the cluster (a shared::cluster address).
+__device__ __forceinline__ long long ld_cluster_s64(uint32_t addr) {
+    long long v;
+    asm volatile("ld.shared::cluster.b64 %0, [%1];" : "=l"(v) : "r"(addr) : "memory");
+    return v;
 }
 // Bounded wait with cluster-scope acquire (the barrier is completed from the peer CTA).
 __device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, uint64_t limit_ns,
@@ -567,7 +582,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 const uint32_t use = static_cast<uint32_t>(lt >> 1);
                 if (!mbar_wait(tempty(buf), (use & 1u) ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * TN);
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf) * L::ACC_STRIDE;
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait(full(stage), phase, limit_ns, abort_flag)) { ok = false; break; }
                     tc_fence_after();
@@ -611,7 +626,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             tc_fence_after();
             int m, n;
             tile_coords(t, m_tiles, n_tiles, m, n);
-            epilogue_swap<TN, F8>(tmem_base, quad, lane, static_cast<uint32_t>(buf * TN), m * BM, n * TN, x_scale, w_scale,
+            epilogue_swap<TN, F8>(tmem_base, quad, lane, static_cast<uint32_t>(buf) * L::ACC_STRIDE, m * BM, n * TN, x_scale, w_scale,
                               bias, y, acc_out, T, N);
             tc_fence_before();
             mbar_arrive(tempty(buf));
@@ -646,7 +661,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             tile_coords(t, m_tiles, n_tiles, m, n);
             const float xs_t = xs;
             prefetch(t + gridDim.x);
-            epilogue_rows<TN, F8>(tmem_base, quad, lane, static_cast<uint32_t>(buf * TN), m * BM + quad * 32, n * TN, xs_t, tab,
+            epilogue_rows<TN, F8>(tmem_base, quad, lane, static_cast<uint32_t>(buf) * L::ACC_STRIDE, m * BM + quad * 32, n * TN, xs_t, tab,
                           bias != nullptr, acc_out, T, N, &tmY, stage_buf, nstores);
             tc_fence_before();
             mbar_arrive(tempty(buf));
@@ -706,6 +721,7 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     const uint32_t done_bar = bar0 + 8u * (2 * P_STAGES + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + P_OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + P_OFF_MISC + 4);
+    long long *s_fills = reinterpret_cast<long long *>(smem + P_OFF_MISC + 8);   // ring fills this CTA issued
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -718,6 +734,7 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         for (int b = 0; b < 2; ++b) { mbar_init(tfull(b), 1); mbar_init(tempty(b), 2 * EPI_WARPS); }
         mbar_init(done_bar, 1);
         *abort_flag = 0;
+        *s_fills = 0;
         mbar_init_fence();
         fence_async_smem();
     }
@@ -755,16 +772,7 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                 }
             }
             if (!ok) give_up(abort_flag);
-            // The even CTA's full barriers count the bytes of both CTAs: once the last fill of every
-            // stage has completed there, no copy of either CTA is in flight.
-            if (rank == 0) {
-                for (int st = 0; st < P_STAGES; ++st) {
-                    if (fills <= st) break;
-                    const long long last = st + ((fills - 1 - st) / P_STAGES) * P_STAGES;
-                    if (!mbar_wait(full(st), static_cast<uint32_t>((last / P_STAGES) & 1), limit_ns, nullptr))
-                        record_status(SQ_ERR_TIMEOUT);
-                }
-            }
+            *s_fills = fills;     // the pair's copies are drained at the end, once both counts are known
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer (even CTA only) ----------------
@@ -848,16 +856,37 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
 
     tc_fence_before();
     __syncthreads();
-    if (*abort_flag) {
-        // After a timeout the peer may still have copies in flight towards this pair's barriers;
-        // give them time to land (they need microseconds) before the pair leaves.
-        const uint64_t t0 = global_ns();
-        while (global_ns() - t0 < 50000ull) {}
+    // Drain: every TMA copy of either CTA completes on the even CTA's full barriers, so the pair may
+    // leave once the last fill of every stage has completed there. Without a timeout both CTAs issued
+    // the same fills. After one, their counts f0 (even) and f1 (odd) may differ by at most a ring's
+    // depth (neither producer can run more than one ring ahead of the MMAs, which need both halves):
+    // a fill only the odd CTA issued still lacks the even CTA's arrival, posted here with the odd
+    // CTA's bytes; a fill only the even CTA issued expects bytes the odd CTA will never send, taken
+    // off its count here. Every wait is bounded; one that runs out records SQ_ERR_TIMEOUT.
+    cluster_sync_all();                                 // both fill counts are written
+    if (rank == 0 && threadIdx.x == 0) {
+        const long long f0 = *s_fills;
+        const long long f1 = ld_cluster_s64(mapa_rank(smem_u32(s_fills), 1));
+        const long long lo = f0 < f1 ? f0 : f1, hi = f0 < f1 ? f1 : f0;
+        for (long long j = lo; j < hi; ++j) {
+            const int st = static_cast<int>(j % P_STAGES);
+            if (f1 > f0) mbar_expect_tx(full(st), static_cast<uint32_t>(P_A_STAGE + P_B_STAGE));
+            else mbar_complete_tx(full(st), static_cast<uint32_t>(P_A_STAGE + P_B_STAGE));
+        }
+        for (int st = 0; st < P_STAGES; ++st) {
+            if (hi <= st) break;
+            const long long last = st + ((hi - 1 - st) / P_STAGES) * P_STAGES;
+            if (!mbar_wait(full(st), static_cast<uint32_t>((last / P_STAGES) & 1), limit_ns, nullptr))
+                record_status(SQ_ERR_TIMEOUT);
+        }
     }
-    cluster_sync_all();
+    cluster_sync_all();                                 // the odd CTA leaves only after the drain
     tc_fence_after();
     if (warp == 1) tmem_dealloc2(tmem_base, P_TMEM_COLS);
 }
+
+// Reads and clears the status word in one atomic exchange, ordered on the caller's stream.
+__global__ void k_status_exchange() { g_sq_status_read = atomicExch(&g_sq_status, 0u); }
 
 // One thread waits, with the same bounded wait as the GEMM, on a barrier nothing completes.
 __global__ void k_selftest_wait(uint64_t limit_ns) {
@@ -970,8 +999,17 @@ sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const voi
     const bool pair = !F8 && g_cta_pair.load(std::memory_order_relaxed) != 0 && T >= 2 * BM;   // 256-row tiles on CTA pairs
     // 64-channel tiles when 256-channel tiles would leave SMs idle (few tokens: the weight stream
     // then bounds the call, and more tiles spread it over more SMs)
-    const int64_t wide_tiles = ((T + BM - 1) / BM) * ((N + BN - 1) / BN);
-    const bool narrow = !pair && wide_tiles < sq::sm_count(dev);
+    const int64_t sms = sq::sm_count(dev);
+    const int64_t m_tiles = (T + BM - 1) / BM;
+    const int64_t wide_tiles = m_tiles * ((N + BN - 1) / BN);
+    const bool narrow = !pair && wide_tiles < sms;
+    // 192-channel tiles when the 256-channel tiles leave much of their last wave idle: a tile's main
+    // loop takes time in proportion to its width, so the call takes about waves x width. (The query,
+    // key and value projections of a 4096-wide block, N = 6144 at T = 4096: 768 tiles of 256 are 5.2
+    // waves on 148 SMs, 1024 tiles of 192 are 6.9.) Only a gain of 3 % or more switches.
+    const int64_t waves256 = (wide_tiles + sms - 1) / sms;
+    const int64_t waves192 = (m_tiles * ((N + 191) / 192) + sms - 1) / sms;
+    const bool mid = !pair && !narrow && waves192 * 192 * 100 < waves256 * 256 * 97;
     CUtensorMap mA, mB, mY;
     if (!pair && T <= BM) {
         // Decode form: the weight streams as the 128-row operand, the tokens (padded to 16 .. 128
@@ -988,7 +1026,7 @@ sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const voi
         }
     }
     st = encode_2d(enc, &mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, T, K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B, "xq");
-    if (st == SQ_OK) st = encode_2d(enc, &mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, K, N, K, BK, pair ? 128 : narrow ? 64 : BN, CU_TENSOR_MAP_SWIZZLE_128B, "wq");
+    if (st == SQ_OK) st = encode_2d(enc, &mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, K, N, K, BK, pair ? 128 : narrow ? 64 : mid ? 192 : BN, CU_TENSOR_MAP_SWIZZLE_128B, "wq");
     if (st == SQ_OK) st = encode_2d(enc, &mY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, T, N * 2, OUT_COLS, OUT_ROWS, CU_TENSOR_MAP_SWIZZLE_64B, "y");
     if (st != SQ_OK) return st;
     if (pair) {
@@ -1029,8 +1067,9 @@ sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const voi
             "launch(w8a8_linear_pair)");
     }
 
-    return narrow ? launch_single<64, false, F8>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream)
-                  : launch_single<BN, false, F8>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+    if (narrow) return launch_single<64, false, F8>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+    if (mid) return launch_single<192, false, F8>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+    return launch_single<BN, false, F8>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
 }
 
 
@@ -1089,17 +1128,20 @@ size_t sq_w8a8_linear_workspace_size(int64_t T, int64_t N, int64_t K) {
 sq_status sq_device_status(void *stream) {
     int dev = 0;
     SQ_TRY_ARCH(dev);
-    cudaError_t e = cudaStreamSynchronize(sq::as_stream(stream));
+    cudaStream_t st = sq::as_stream(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return sq::cuda_status(e, "cudaStreamSynchronize");
+    // read and clear in one atomic exchange: an error a kernel on another stream records meanwhile is
+    // either reported now or stays in the word for the next call, never lost
+    k_status_exchange<<<1, 1, 0, st>>>();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return sq::cuda_status(e, "launch(status_exchange)");
     unsigned int word = 0;
-    e = cudaMemcpyFromSymbol(&word, g_sq_status, sizeof word);
-    if (e != cudaSuccess) return sq::cuda_status(e, "cudaMemcpyFromSymbol(status)");
-    if (word != 0) {
-        const unsigned int zero = 0;
-        e = cudaMemcpyToSymbol(g_sq_status, &zero, sizeof zero);
-        if (e != cudaSuccess) return sq::cuda_status(e, "cudaMemcpyToSymbol(status)");
+    e = cudaMemcpyFromSymbolAsync(&word, g_sq_status_read, sizeof word, 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return sq::cuda_status(e, "reading the status word");
+    if (word != 0)
         return sq::fail(static_cast<sq_status>(word), "device status word reported %s", sq_status_string(static_cast<int>(word)));
-    }
     return SQ_OK;
 }
 

@@ -236,13 +236,22 @@ __device__ __forceinline__ uint32_t f8codes2(uint64_t t) {
     return d;
 }
 
+// Clamp of x to [-q, q] that keeps a NaN a NaN (min/max with the .NaN modifier).
+__device__ __forceinline__ float clamp_keep_nan(float x, float q) {
+    float d;
+    asm("{\n\t.reg .f32 t;\n\tmax.NaN.f32 t, %1, %2;\n\tmin.NaN.f32 %0, t, %3;\n\t}" : "=f"(d) : "f"(x), "f"(-q), "f"(q));
+    return d;
+}
+
 // codes2 for values that may lie beyond the calibrated range (static scale): t is clamped to
-// [-127, 127] first, so a code saturates at +-127.
+// [-127, 127] first, so a code saturates at +-127. When the static reciprocal 127/m overflowed to
+// infinity (a calibrated maximum below 127 / FLT_MAX), a zero value gives t = 0 * inf = NaN: the clamp
+// keeps it, and the truncating conversion turns a NaN into the code 0.
 __device__ __forceinline__ uint32_t codes2_clamped(uint64_t t) {
     uint32_t tl, th;
     unpack2(t, tl, th);
-    const float a = fminf(fmaxf(__uint_as_float(tl), -kQmax), kQmax);
-    const float b = fminf(fmaxf(__uint_as_float(th), -kQmax), kQmax);
+    const float a = clamp_keep_nan(__uint_as_float(tl), kQmax);
+    const float b = clamp_keep_nan(__uint_as_float(th), kQmax);
     return codes2(pack2(a, b));
 }
 
@@ -324,11 +333,6 @@ __device__ __forceinline__ void rows_body(const RowArgs p, unsigned cta, unsigne
     const bool has_vec = p.vec != nullptr;
     float sdelta = 0.0f;
     uint64_t sinv2 = 0;
-    if (MODE == MODE_QSTATIC) {
-        sdelta = __ldg(p.scale2);
-        const float si = __ldg(p.scale2 + 1);
-        sinv2 = pack2(si, si);
-    }
 
     const int64_t units = (p.rows + R - 1) / R;
     const int64_t g0 = static_cast<int64_t>(cta) * G + group;
@@ -346,6 +350,12 @@ __device__ __forceinline__ void rows_body(const RowArgs p, unsigned cta, unsigne
     // only amax waits for the fill (below).
     if (!(ABS && p.early)) pdl_wait();
     pdl_trigger();
+    if (MODE == MODE_QSTATIC) {
+        // the static scale is written by the kernel before this one (after the wait: never stale)
+        sdelta = __ldg(p.scale2);
+        const float si = __ldg(p.scale2 + 1);
+        sinv2 = pack2(si, si);
+    }
     if (MODE != MODE_ABSMAX && has_vec) {
         const float4 *cv = reinterpret_cast<const float4 *>(p.vec);
         for (int v = tid; v < nvec; v += kThreads) { c_lo[v] = __ldg(cv + 2 * v); c_hi[v] = __ldg(cv + 2 * v + 1); }
@@ -641,13 +651,25 @@ __device__ __forceinline__ void rows_body(const RowArgs p, unsigned cta, unsigne
                 // step and reciprocal of the row this lane holds; one lane per row stores the step
                 constexpr float qmax = MODE == MODE_QF8 ? kF8Max : kQmax;
                 const float delta = mrow > 0.0f ? __fdiv_rn(mrow, qmax) : 0.0f;
-                const float inv_m = mrow > 0.0f ? __fdiv_rn(qmax, mrow) : 0.0f;
+                float inv_m = mrow > 0.0f ? __fdiv_rn(qmax, mrow) : 0.0f;
+                // A row maximum below qmax / FLT_MAX (about 3.7e-37 for INT8): qmax / m overflows binary32.
+                // Such a row is scaled by 2^64 first (exact: its values are far below the top of the
+                // range) and coded as t = fl(fl(y * 2^64) * fl(qmax / fl(m * 2^64))); the step stays m / qmax.
+                const bool tiny = isinf(inv_m);
+                if (tiny) inv_m = __fdiv_rn(qmax, __fmul_rn(mrow, 0x1p64f));
                 if (wig == 0 && (lane % SUB) == 0 && lane / SUB < nr && SQ_CHECK(r0 + lane / SUB < p.rows, p.status))
                     p.scale[r0 + lane / SUB] = delta;
                 // ---- pass C: codes
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     const float iv = __shfl_sync(kAll, inv_m, r * SUB);
+                    if (__shfl_sync(kAll, tiny ? 1 : 0, r * SUB) != 0) {      // uniform across the row's lanes
+                        const uint64_t up2 = pack2(0x1p64f, 0x1p64f);
+#pragma unroll
+                        for (int i = 0; i < VPL; ++i)
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) y[r][i][k] = mul2_rn(y[r][i][k], up2);
+                    }
                     if (r < nr) {
                         const uint64_t inv2 = pack2(iv, iv);
                         uint2 *qrow = reinterpret_cast<uint2 *>(p.q + (r0 + r) * static_cast<int64_t>(K));

@@ -205,6 +205,60 @@ def test_quantiser_invariants_random(orc):
     assert np.allclose(xs, np.abs(y).max(axis=1) / 127, rtol=3e-7, atol=0)
 
 
+def _tiny_rows(rows, K, seed):
+    """bf16 rows whose largest magnitude lies between the bf16 subnormals and ~1e-37, where 127 / m
+    (and 448 / m) overflows binary32; one row is all zero except one subnormal, one is all zero."""
+    rng = np.random.default_rng(seed)
+    mag = 2.0 ** rng.uniform(-133, -123, size=(rows, K))
+    v = (mag * rng.choice([-1.0, 1.0], size=(rows, K))).astype(np.float32)
+    v[1, :] = 0.0
+    v[1, 3] = -2.0 ** -133                       # the smallest bf16 subnormal
+    v[2, :] = 0.0
+    v[3, 5] = 0.0
+    return bf16_bits(torch.from_numpy(v).to(torch.bfloat16))
+
+
+def test_tiny_rows_quantise_like_their_scaled_copies(orc):
+    """A row whose maximum m is so small that 127 / m overflows binary32 is quantised as the same row
+    scaled by a power of two into the normal range: the quantiser is scale-free, and a power-of-two
+    scaling is exact in every step (so the codes must be identical), while the step is still
+    fl(m / 127) of the unscaled m. Per-token (direct input), weight rows (s = 1) and FP8."""
+    x = _tiny_rows(6, 64, 90)
+    xf = bits_to_f64(x)
+    one = np.ones(64, np.float32)
+    big = bf16_bits(torch.from_numpy((xf * 2.0 ** 80).astype(np.float32)).to(torch.bfloat16))
+    assert np.array_equal(bits_to_f64(big), xf * 2.0 ** 80)        # the scaling itself is exact
+    q, d = orc.rmsnorm_smooth_quant(x, one, apply_norm=False)
+    qb, db = orc.rmsnorm_smooth_quant(big, one, apply_norm=False)
+    assert np.array_equal(q, qb)
+    m = np.abs(xf).max(axis=1).astype(np.float32)
+    assert np.array_equal(d, np.where(m > 0, m / np.float32(127), 0).astype(np.float32))
+    nz = m > 0
+    assert np.all(np.abs(q[nz]).max(axis=1) == 127) and np.all(q[~nz] == 0)
+    # codes within half a level of the exact v / delta (exact rational arithmetic in binary64 is
+    # exact here: the scaled values have 8 significant bits)
+    t = xf[nz] * 2.0 ** 80 * 127 / (m[nz].astype(np.float64)[:, None] * 2.0 ** 80)
+    assert np.all(np.abs(q[nz] - t) <= 0.5 + 1e-5)
+    wq, ws = orc.smooth_quantize_weight(x)
+    assert np.array_equal(wq, q) and np.array_equal(ws, d)
+    f8, d8 = orc.rmsnorm_smooth_quant_f8(x, one, apply_norm=False)
+    f8b, _ = orc.rmsnorm_smooth_quant_f8(big, one, apply_norm=False)
+    assert np.array_equal(f8, f8b)
+    assert np.array_equal(d8, np.where(m > 0, m / np.float32(448), 0).astype(np.float32))
+
+
+def test_static_scale_with_overflowing_reciprocal(orc):
+    """A static maximum below 127 / FLT_MAX: fl(127 / m) is +inf. Every nonzero value lies beyond the
+    representable step and saturates at +-127; a zero value still codes 0 (not the NaN of 0 * inf)."""
+    s2 = orc.static_scale(np.array([1e-38, 3e-38], np.float32))
+    assert s2[0] == np.float32(3e-38) / np.float32(127) and np.isinf(s2[1])
+    x = _tiny_rows(4, 32, 91)
+    q, xs = orc.rmsnorm_smooth_quant_static(x, np.ones(32, np.float32), s2, apply_norm=False)
+    xf = bits_to_f64(x)
+    assert np.array_equal(q, (np.sign(xf) * 127).astype(np.int8))
+    assert np.all(xs == s2[0])
+
+
 def test_rmsnorm_constant_rows_and_scale_invariance(orc):
     K = 128
     x = np.zeros((3, K), np.float32)
@@ -309,6 +363,45 @@ def test_fold_into_prev_linear_rounding_and_w_scale(orc):
     assert np.all(np.abs(bits_to_f64(wo) - exact) <= np.abs(exact) * 2.0 ** -8 + 1e-30)
     ws = (np.random.default_rng(62).random(K) * 1e-2).astype(np.float32)
     assert np.array_equal(orc.fold_into_w_scale(ws, fold), ws * fold)     # one binary32 product each
+
+
+@pytest.mark.parametrize("pow2", [True, False])
+def test_fold_into_w_scale_divides_the_int8_layer_output_by_s(orc, pow2):
+    """"06 -- SmoothQuant...", section 7: folding 1/s into an INT8 previous layer must make that layer's
+    dequantised output arrive divided by s, column by column. The previous layer's output is taken
+    through the oracle's own INT8 GEMM and dequantisation, once with the folded scale and once
+    without: with power-of-two s every step scales exactly (bit-exact bf16 outputs); otherwise the
+    folded scale is the exact ws / s within two binary32 roundings (fl(1/s), then the product), and the
+    bf16 outputs agree within one bf16 rounding of that."""
+    T, K, Kp = 24, 40, 64                  # previous layer: [T, Kp] x [K, Kp]^T -> [T, K]
+    rng = np.random.default_rng(63)
+    xq = rng.integers(-127, 128, size=(T, Kp), dtype=np.int8)
+    wq = rng.integers(-127, 128, size=(K, Kp), dtype=np.int8)
+    xs = (rng.random(T) * 1e-2 + 1e-3).astype(np.float32)
+    ws = (rng.random(K) * 1e-2 + 1e-3).astype(np.float32)
+    if pow2:
+        s = (2.0 ** rng.integers(-6, 7, size=K)).astype(np.float32)
+    else:
+        s = (0.05 + 20 * rng.random(K)).astype(np.float32)
+    fold = (np.float32(1.0) / s).astype(np.float32)               # fl32(1/s): the fold without gamma
+    ws_f = orc.fold_into_w_scale(ws, fold)
+    rel = np.abs(ws_f.astype(np.float64) * s.astype(np.float64) / ws.astype(np.float64) - 1.0)
+    assert np.all(rel <= 2.0 ** -23 + 2.0 ** -46), "folded scale is not ws / s within two roundings"
+    y0, acc = orc.w8a8_linear(xq, xs, wq, ws)                      # unfolded layer (bf16 bits)
+    y1, acc1 = orc.w8a8_linear(xq, xs, wq, ws_f)                   # folded layer
+    assert np.array_equal(acc, acc1)
+    v0, v1 = bits_to_f64(y0), bits_to_f64(y1)
+    target = v0 / s[None, :].astype(np.float64)
+    if pow2:
+        assert np.array_equal(v1, target), "a power-of-two fold must divide the output exactly"
+    else:
+        # |y1 - y0 / s| <= bf16 rounding of both outputs plus the scale's two binary32 roundings
+        tol = (np.abs(target) + np.abs(v1)) * (2.0 ** -8 + 2.0 ** -22) + 1e-30
+        assert np.all(np.abs(v1 - target) <= tol)
+    # a wrong index (the fold applied to the wrong channel) moves some output column by far more
+    wrong = orc.fold_into_w_scale(ws, np.roll(fold, 1))
+    yw, _ = orc.w8a8_linear(xq, xs, wq, wrong)
+    assert not np.allclose(bits_to_f64(yw), target, rtol=1e-2)
 
 
 # --------------------------------------------------------------------------------------------

@@ -188,8 +188,11 @@ EDGE = [
     (128, 256, 128, True, False),
     (255, 512, 4096, False, False),
     (777, 1288, 2064, True, True),
-    # enough 256-channel tiles to take the wide form, with ragged T, N and K
+    # 192-channel tiles (the 256-wide ones would leave most of a second wave idle), ragged T, N and K
     (2000, 2312, 1040, True, True),
+    (1100, 5000, 1040, False, True),
+    # enough 256-channel tiles to take the wide form, with ragged T, N and K
+    (2000, 4104, 1040, True, True),
     (64, 37888, 64, False, True),
 ]
 
@@ -441,6 +444,78 @@ def test_static_scale_path(sq, orc, K, norm):
     acc = torch.empty(T, N, dtype=torch.int32, device=dev)
     y = sq.sq_w8a8_linear(xq, xs, wq, ws, acc_out=acc)
     check_linear(sq, orc, xq, xs, wq, ws, None, y, acc)
+    ok_status(sq)
+
+
+# Rows whose maximum m is so small that 127 / m (448 / m for FP8) overflows binary32: the library
+# and the oracle both scale such a row by 2^64 before coding it (exact), and with an overflowing static
+# reciprocal a zero value codes 0 and every other value saturates. Tiny rows sit next to ordinary rows
+# in the same units (one-warp units of several rows, two- and eight-warp row groups), and include a
+# row of one subnormal, a zero row and zeros inside tiny rows. Per-token, weight, FP8 and static.
+TINY_SHAPES = [(37, 64), (700, 1024), (37, 4096), (700, 4096), (40, 8192)]
+
+
+def _tiny_rows_dev(T, K, seed):
+    rng = np.random.default_rng(seed)
+    mag = 2.0 ** rng.uniform(-133, -123, size=(T, K))
+    v = (mag * rng.choice([-1.0, 1.0], size=(T, K))).astype(np.float32)
+    normal = rng.random(T) < 0.3                       # ordinary rows in between
+    normal[:5] = False
+    v[normal] = rng.standard_normal((int(normal.sum()), K)).astype(np.float32)
+    v[1, :] = 0.0
+    v[1, 3] = -2.0 ** -133
+    v[2, :] = 0.0
+    v[3, 5] = 0.0
+    return torch.from_numpy(v).to(torch.bfloat16).cuda()
+
+
+@pytest.mark.parametrize("T,K", TINY_SHAPES)
+def test_tiny_rows_every_quantiser(sq, orc, T, K):
+    x = _tiny_rows_dev(T, K, 17 * T + K)
+    one = torch.ones(K, dtype=torch.float32, device="cuda")
+    xh, oh = h16(x), np.ones(K, np.float32)
+    xq, xs = sq.sq_rmsnorm_smooth_quant(x, one, apply_norm=False)
+    xq_o, xs_o = orc.rmsnorm_smooth_quant(xh, oh, apply_norm=False)
+    assert np.array_equal(hnp(xs), xs_o), "token scales of tiny rows differ"
+    assert np.array_equal(hnp(xq), xq_o), f"{int((hnp(xq) != xq_o).sum())} codes of tiny rows differ"
+    wq, ws = sq.sq_smooth_quantize_weight(x, None)
+    wq_o, ws_o = orc.smooth_quantize_weight(xh)
+    assert np.array_equal(hnp(ws), ws_o) and np.array_equal(hnp(wq), wq_o), "weight codes of tiny rows differ"
+    fq, fs = sq.sq_rmsnorm_smooth_quant_fp8(x, one, apply_norm=False)
+    fq_o, fs_o = orc.rmsnorm_smooth_quant_f8(xh, oh, apply_norm=False)
+    assert np.array_equal(hnp(fs), fs_o) and np.array_equal(hnp(fq), fq_o), "fp8 codes of tiny rows differ"
+    # a static scale calibrated on tiny values only: 127 / m overflows to +inf
+    amax = sq.sq_calibrate_absmax(x[4:5])
+    s2 = sq.sq_static_scale(amax)
+    s2_o = orc.static_scale(orc.calibrate_absmax(xh[4:5]))
+    assert np.array_equal(hnp(s2), s2_o) and np.isinf(s2_o[1])
+    sq_q, sq_s = sq.sq_rmsnorm_smooth_quant_static(x, one, s2, apply_norm=False)
+    st_o, ss_o = orc.rmsnorm_smooth_quant_static(xh, oh, s2_o, apply_norm=False)
+    assert np.array_equal(hnp(sq_s), ss_o) and np.array_equal(hnp(sq_q), st_o), "static codes of tiny rows differ"
+    assert np.array_equal(st_o, (np.sign(f64(xh)) * 127).astype(np.int8))
+    ok_status(sq)
+
+
+# The static quantiser reads the scale that the kernel launched just before it writes (a dependent
+# launch: it may start while that kernel still runs). The buffer is refilled with a wrong scale before
+# every pair of calls, so a read that does not wait for its producer shows up as wrong codes.
+def test_static_scale_read_after_its_producer(sq, orc):
+    dev = "cuda"
+    T, K = 256, 4096
+    ch = synth.outlier_channels(K, synth.OutlierSpec(16, 10.0, 25.0), 5)
+    X = synth.outlier_tokens(T, K, ch, 6, dev)
+    fold = synth.norm_gamma(K, 7, dev)
+    Xh, fh = h16(X), hnp(fold)
+    s2 = torch.empty(2, dtype=torch.float32, device=dev)
+    for i in range(12):
+        amax = (torch.rand(K, device=dev) + 0.5) * (1 + i)
+        s2.fill_(1e-30)                                # the wrong scale a stale read would see
+        sq.sq_static_scale(amax, scale2=s2)
+        xq, xs = sq.sq_rmsnorm_smooth_quant_static(X, fold, s2)
+        s2_o = orc.static_scale(hnp(amax))
+        xq_o, xs_o = orc.rmsnorm_smooth_quant_static(Xh, fh, s2_o)
+        assert np.array_equal(hnp(s2), s2_o)
+        assert np.array_equal(hnp(xs), xs_o) and np.array_equal(hnp(xq), xq_o), f"stale static scale at call {i}"
     ok_status(sq)
 
 
