@@ -43,3 +43,25 @@ def test_perf_lines_for_the_smallest_and_the_decode_workload():
         assert r["us"] > 0 and r["gbs"] > 0 and r["peaks"] in ("measured", "fallback")
         if r["stage"] == "gemm":
             assert r["tops"] > 0
+
+
+@pytest.mark.gpu
+def test_parity_report_lines_for_the_single_linear():
+    """The per-workload report: every stage of the single linear layer with its GPU rate, its parity
+    against the oracle (all bit-exact, the scale and bf16 bars met) and the oracle's time."""
+    import os
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+    import parity_report
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        rc = parity_report.main(["--workload", "single_linear_t256_k1024_n1024", "--reps", "3", "--gemm-sample", "8"])
+    assert rc == 0
+    rows = {r["stage"]: r for r in (json.loads(l) for l in buf.getvalue().splitlines() if l.strip())}
+    assert set(rows) == {"calib_absmax_pair", "scales", "weight_quant", "act_quant", "gemm"}
+    for st in ("calib_absmax_pair", "weight_quant", "act_quant"):
+        assert rows[st]["mismatches"] == 0 and rows[st]["oracle_s"] > 0 and rows[st]["us"] > 0
+    assert rows["scales"]["max_rel_err"] <= 1e-6
+    g = rows["gemm"]
+    assert g["acc_mismatches"] == 0 and g["y_mismatches"] == 0 and g["max_rel_err"] <= 1e-2
+    assert g["oracle_extrapolated"] is True and g["tops"] > 0 and g["oracle_threads"] >= 1
