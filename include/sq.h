@@ -244,9 +244,9 @@ sq_status sq_layernorm_smooth_quant(const void *x, int64_t T, int64_t K, const f
  * Requirements: T >= 0, N >= 8, N % 8 == 0, K >= 16, K % 16 == 0, K <= 131072; xq, wq, y 16-byte
  * aligned; acc_out 16-byte aligned. The GEMM runs on the tensor cores (tcgen05, TMEM accumulators,
  * TMA-fed shared-memory pipeline); its device-side waits are bounded and report SQ_ERR_TIMEOUT
- * through sq_device_status() instead of hanging. Output tiles are 128 tokens x 256, 192 or 64
- * channels (whichever fills the SMs best), or, for T <= 128, 128 channels x 16..128 tokens; every
- * form computes the same bits.
+ * through sq_device_status() instead of hanging. Output tiles are 128 tokens x 256 channels (64
+ * channels when 256-wide tiles would leave SMs idle), or, for T <= 128, 128 channels x 16..128
+ * tokens; every form computes the same bits.
  */
 sq_status sq_w8a8_linear(const int8_t *xq, const float *x_scale, int64_t T, const int8_t *wq,
                          const float *w_scale, int64_t N, int64_t K, const void *bias, void *y,

@@ -16,7 +16,8 @@
  *   - Quantiser: symmetric, delta = max|v| / 127, code = round-half-away-from-zero(v * (127/max|v|)),
  *     clamped to [-127, 127]. The pages leave the tie rule open ([TAMING], "Why Outliers Break
  *     Quantization") or use half-to-even in a listing; half-away is the fixed reading. The
- *     reciprocal-multiply form (v * fl32(127/m)) is the fixed reading of dividing v by delta.
+ *     reciprocal-multiply form (v * fl32(127/m)) is the fixed reading of dividing v by delta, and
+ *     the product is rounded once, to the integer (not first to binary32).
  *   - All per-element arithmetic is binary32 with each operation rounded (compile with
  *     -ffp-contract=off, no fast-math); the RMSNorm sum of squares is accumulated in binary64.
  *   - RMSNorm is the standard x / sqrt(mean(x^2) + eps) * gamma (the pages name RMSNorm but do not
@@ -67,16 +68,18 @@ uint16_t orc_f32_to_bf16(float f) { return f32_to_bf16_rne(f); }
 float orc_bf16_to_f32(uint16_t h) { return bf16_to_f32(h); }
 
 /* Symmetric INT8 code of one value, [TAMING] "Why Outliers Break Quantization" (quantisation
- * equation): v / delta rounded to the nearest integer. roundf is C99's round-half-away-from-zero.
+ * equation): v / delta rounded to the nearest integer, with v / delta taken as v * fl32(127 / m).
+ * The product of two binary32 values is exact in binary64 (48 significant bits), so the integer
+ * rounding is applied to the exact product, once; C99's round() is round-half-away-from-zero.
  * An infinite inv_delta (a static scale whose 127 / m overflowed) makes t = 0 * inf = NaN for a zero
  * value: the code of a zero value is 0 whatever the scale. */
 static int8_t quantize_one(float v, float inv_delta)
 {
-    float t = v * inv_delta;
+    double t = (double)v * (double)inv_delta;
     if (isnan(t)) return 0;
-    float r = roundf(t);
-    if (r > (float)ORC_QMAX) r = (float)ORC_QMAX;
-    if (r < -(float)ORC_QMAX) r = -(float)ORC_QMAX;
+    double r = round(t);
+    if (r > (double)ORC_QMAX) r = (double)ORC_QMAX;
+    if (r < -(double)ORC_QMAX) r = -(double)ORC_QMAX;
     return (int8_t)r;
 }
 

@@ -104,9 +104,9 @@ struct Tile {
     static constexpr int B_SLOT = KS * B_SLICE;
     static constexpr int SPARE = 232448 - 1024 - EPI_WARPS * 2 * OUT_BOX - 2 * COL_TAB - 512;
     static constexpr int STAGES = SWAP ? (SPARE / (A_SLOT + B_SLOT) > 11 ? 11 : SPARE / (A_SLOT + B_SLOT))
-                                       : (SPARE / (A_SLOT + B_SLOT) > 8 ? 8 : SPARE / (A_SLOT + B_SLOT));   // 256: 4, 192: 5, 64: 8
+                                       : (SPARE / (A_SLOT + B_SLOT) > 8 ? 8 : SPARE / (A_SLOT + B_SLOT));   // 256: 4, 64: 8
     // two accumulators ACC_STRIDE columns apart; the allocation is a power of two >= 32 columns
-    static constexpr uint32_t TMEM_COLS = TN == 192 ? 512u : 2u * TN;
+    static constexpr uint32_t TMEM_COLS = 2u * TN;
     static constexpr uint32_t ACC_STRIDE = TMEM_COLS / 2;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_SLOT;
@@ -120,7 +120,7 @@ struct Tile {
     static constexpr uint32_t IDESC_F8 = make_idesc_f8(BM, TN);
     static_assert(SMEM_TOTAL <= 232448, "shared memory budget of one sm_100 CTA");
     static_assert(SWAP ? (TN >= 16 && TN <= 128 && (TN & (TN - 1)) == 0)
-                       : (TN % OUT_COLS == 0 && TN >= 32 && TN <= 256 && ((TN & (TN - 1)) == 0 || TN == 192)), "tile width");
+                       : (TN % OUT_COLS == 0 && TN >= 32 && TN <= 256 && (TN & (TN - 1)) == 0), "tile width");
 };
 
 // ------------------------------------------------------------------------------------------------
@@ -999,17 +999,12 @@ sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const voi
     const bool pair = !F8 && g_cta_pair.load(std::memory_order_relaxed) != 0 && T >= 2 * BM;   // 256-row tiles on CTA pairs
     // 64-channel tiles when 256-channel tiles would leave SMs idle (few tokens: the weight stream
     // then bounds the call, and more tiles spread it over more SMs)
-    const int64_t sms = sq::sm_count(dev);
-    const int64_t m_tiles = (T + BM - 1) / BM;
-    const int64_t wide_tiles = m_tiles * ((N + BN - 1) / BN);
-    const bool narrow = !pair && wide_tiles < sms;
-    // 192-channel tiles when the 256-channel tiles leave much of their last wave idle: a tile's main
-    // loop takes time in proportion to its width, so the call takes about waves x width. (The query,
-    // key and value projections of a 4096-wide block, N = 6144 at T = 4096: 768 tiles of 256 are 5.2
-    // waves on 148 SMs, 1024 tiles of 192 are 6.9.) Only a gain of 3 % or more switches.
-    const int64_t waves256 = (wide_tiles + sms - 1) / sms;
-    const int64_t waves192 = (m_tiles * ((N + 191) / 192) + sms - 1) / sms;
-    const bool mid = !pair && !narrow && waves192 * 192 * 100 < waves256 * 256 * 97;
+    // (192-channel tiles, which would fill the last wave better for some shapes, were measured slower:
+    // with 40 KB of operands per 128 x 192 x 128 block against 48 KB per 128 x 256 x 128 the main loop
+    // does not shrink with the tile width, so 1024 tiles of 192 took 92.3 us where 768 tiles of 256
+    // took 84.0 us for the N = 6144, T = 4096, K = 4096 query-key-value projection.)
+    const int64_t wide_tiles = ((T + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const bool narrow = !pair && wide_tiles < sq::sm_count(dev);
     CUtensorMap mA, mB, mY;
     if (!pair && T <= BM) {
         // Decode form: the weight streams as the 128-row operand, the tokens (padded to 16 .. 128
@@ -1026,7 +1021,7 @@ sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const voi
         }
     }
     st = encode_2d(enc, &mA, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K, T, K, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B, "xq");
-    if (st == SQ_OK) st = encode_2d(enc, &mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, K, N, K, BK, pair ? 128 : narrow ? 64 : mid ? 192 : BN, CU_TENSOR_MAP_SWIZZLE_128B, "wq");
+    if (st == SQ_OK) st = encode_2d(enc, &mB, CU_TENSOR_MAP_DATA_TYPE_UINT8, wq, K, N, K, BK, pair ? 128 : narrow ? 64 : BN, CU_TENSOR_MAP_SWIZZLE_128B, "wq");
     if (st == SQ_OK) st = encode_2d(enc, &mY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, N, T, N * 2, OUT_COLS, OUT_ROWS, CU_TENSOR_MAP_SWIZZLE_64B, "y");
     if (st != SQ_OK) return st;
     if (pair) {
@@ -1067,9 +1062,8 @@ sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const voi
             "launch(w8a8_linear_pair)");
     }
 
-    if (narrow) return launch_single<64, false, F8>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
-    if (mid) return launch_single<192, false, F8>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
-    return launch_single<BN, false, F8>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
+    return narrow ? launch_single<64, false, F8>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream)
+                  : launch_single<BN, false, F8>(mA, mB, mY, x_scale, w_scale, bias, acc_out, y, T, N, K, dev, stream);
 }
 
 

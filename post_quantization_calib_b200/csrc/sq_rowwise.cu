@@ -40,10 +40,12 @@
 //     2^-1076 rounds away inside the fused multiply-add); the binary64 accumulator is rescaled by
 //     2^822 at the end. Squares of |x| < 2^-100 (and of subnormal bf16) are not exact; they are
 //     below 2^-200 and cannot move a binary32 result unless the whole row is that small.
-//   * INT8 codes: v = rz(t + copysign(1/2, t)) (round toward zero cannot carry the sum across an
-//     integer), then a truncating conversion gives round_half_away(t); |t| <= fl(m * fl(127/m))
-//     <= 127.00001, so the code never leaves [-127, 127].
-//   * pairs of binary32 values use the packed f32x2 instructions of sm_100.
+//   * INT8 codes: v = rz(y * iv + copysign(1/2, y)) in one fused multiply-add (round toward zero
+//     cannot carry the sum across an integer), then a truncating conversion gives
+//     round_half_away(y * iv) of the exact product; |y * iv| <= m * fl(127/m) <= 127.00001, so the
+//     code never leaves [-127, 127]; four codes are packed with two saturating conversions.
+//   * the quantisers' per-element arithmetic is scalar binary32 (the packed f32x2 forms cost more
+//     register moves than they save there); the abs-max keeps the packed forms.
 // Arithmetic otherwise follows the RMSNorm / quantiser definitions step by step with explicit
 // round-to-nearest operations (nothing is contracted into fused multiply-adds), so results are
 // bit-identical to the definitions.
@@ -213,27 +215,14 @@ __device__ __forceinline__ void add_centred_squares(uint32_t w, uint64_t nm2, do
     b = __fma_rn(dh, dh, b);
 }
 
-// Signed INT8 codes of the two values of t: round half away from zero. v = rz(t + copysign(1/2, t))
-// has the integer part of the exactly rounded value, and the conversion truncates it.
-__device__ __forceinline__ uint32_t codes2(uint64_t t) {
-    uint32_t tl, th;
-    unpack2(t, tl, th);
-    const uint64_t half = pack2u((tl & 0x80000000u) | 0x3F000000u, (th & 0x80000000u) | 0x3F000000u);
-    uint32_t vl, vh;
-    unpack2(add2_rz(t, half), vl, vh);
-    const int ql = __float2int_rz(__uint_as_float(vl));
-    const int qh = __float2int_rz(__uint_as_float(vh));
-    return __byte_perm(static_cast<uint32_t>(ql), static_cast<uint32_t>(qh), 0x0040);   // bytes: ql, qh in 0, 1
-}
-
-// E4M3 codes of the two values of t (round to nearest, ties to even, saturating at +-448, the sign
-// kept on a zero): the low element's code in the low byte.
-__device__ __forceinline__ uint32_t f8codes2(uint64_t t) {
-    uint32_t tl, th;
-    unpack2(t, tl, th);
-    uint16_t d;
-    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(__uint_as_float(th)), "f"(__uint_as_float(tl)));
-    return d;
+// INT8 code of y with the reciprocal step iv: round half away from zero of the exact product y * iv.
+// v = rz(y * iv + copysign(1/2, y)) in one fused multiply-add rounded toward zero cannot carry the
+// sum across an integer (an integer is representable), so the truncating conversion of v gives
+// round_half_away(y * iv) (iv > 0, so y * iv has the sign of y); |y * iv| <= 127.00001 on the
+// dynamic path, so its code never leaves [-127, 127].
+__device__ __forceinline__ int code_of(float y, float iv) {
+    const float h = __uint_as_float((__float_as_uint(y) & 0x80000000u) | 0x3F000000u);
+    return __float2int_rz(__fmaf_rz(y, iv, h));
 }
 
 // Clamp of x to [-q, q] that keeps a NaN a NaN (min/max with the .NaN modifier).
@@ -243,16 +232,29 @@ __device__ __forceinline__ float clamp_keep_nan(float x, float q) {
     return d;
 }
 
-// codes2 for values that may lie beyond the calibrated range (static scale): t is clamped to
-// [-127, 127] first, so a code saturates at +-127. When the static reciprocal 127/m overflowed to
-// infinity (a calibrated maximum below 127 / FLT_MAX), a zero value gives t = 0 * inf = NaN: the clamp
-// keeps it, and the truncating conversion turns a NaN into the code 0.
-__device__ __forceinline__ uint32_t codes2_clamped(uint64_t t) {
-    uint32_t tl, th;
-    unpack2(t, tl, th);
-    const float a = clamp_keep_nan(__uint_as_float(tl), kQmax);
-    const float b = clamp_keep_nan(__uint_as_float(th), kQmax);
-    return codes2(pack2(a, b));
+// code_of for values that may lie beyond the calibrated range (static scale): v is clamped to
+// [-127, 127] before the truncation, so a code saturates at +-127 (truncation is monotone). When the
+// static reciprocal 127/m overflowed to infinity (a calibrated maximum below 127 / FLT_MAX), a zero
+// value gives 0 * inf = NaN: the clamp keeps it and the conversion turns a NaN into the code 0.
+__device__ __forceinline__ int code_of_clamped(float y, float iv) {
+    const float h = __uint_as_float((__float_as_uint(y) & 0x80000000u) | 0x3F000000u);
+    return __float2int_rz(clamp_keep_nan(__fmaf_rz(y, iv, h), kQmax));
+}
+
+// Four INT8 codes in one word, q0 in the low byte (saturating packs of two values each).
+__device__ __forceinline__ uint32_t pack4_s8(int q0, int q1, int q2, int q3) {
+    uint32_t t, d;
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(t) : "r"(q3), "r"(q2));
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(q1), "r"(q0), "r"(t));
+    return d;
+}
+
+// E4M3 codes of two values (round to nearest, ties to even, saturating at +-448, the sign kept on a
+// zero): the first value's code in the low byte.
+__device__ __forceinline__ uint32_t f8codes2(float lo, float hi) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
 }
 
 // LayerNorm parameters of vector v (8 columns) as binary32 pairs: g from the shared-memory table,
@@ -331,8 +333,7 @@ __device__ __forceinline__ void rows_body(const RowArgs p, unsigned cta, unsigne
     float4 *c_lo = reinterpret_cast<float4 *>(smem + (ring_bytes > red_bytes ? ring_bytes : red_bytes));   // c[8v .. 8v+3]
     float4 *c_hi = c_lo + nvec;                                                                              // c[8v+4 .. 8v+7]
     const bool has_vec = p.vec != nullptr;
-    float sdelta = 0.0f;
-    uint64_t sinv2 = 0;
+    float sdelta = 0.0f, sinv = 0.0f;
 
     const int64_t units = (p.rows + R - 1) / R;
     const int64_t g0 = static_cast<int64_t>(cta) * G + group;
@@ -353,8 +354,7 @@ __device__ __forceinline__ void rows_body(const RowArgs p, unsigned cta, unsigne
     if (MODE == MODE_QSTATIC) {
         // the static scale is written by the kernel before this one (after the wait: never stale)
         sdelta = __ldg(p.scale2);
-        const float si = __ldg(p.scale2 + 1);
-        sinv2 = pack2(si, si);
+        sinv = __ldg(p.scale2 + 1);
     }
     if (MODE != MODE_ABSMAX && has_vec) {
         const float4 *cv = reinterpret_cast<const float4 *>(p.vec);
@@ -582,7 +582,6 @@ __device__ __forceinline__ void rows_body(const RowArgs p, unsigned cta, unsigne
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     if (r < nr) {
-                        const uint64_t ir2 = pack2(ir[r], ir[r]);
                         uint2 *qrow = reinterpret_cast<uint2 *>(p.q + (r0 + r) * static_cast<int64_t>(K));
 #pragma unroll
                         for (int i = 0; i < VPL; ++i) {
@@ -590,16 +589,17 @@ __device__ __forceinline__ void rows_body(const RowArgs p, unsigned cta, unsigne
                             if (!SQ_COL_IN(v)) continue;
                             float4 cl = make_float4(1.f, 1.f, 1.f, 1.f), ch = cl;
                             if (has_vec) { cl = c_lo[v]; ch = c_hi[v]; }
-                            const uint64_t c2[4] = {pack2(cl.x, cl.y), pack2(cl.z, cl.w), pack2(ch.x, ch.y), pack2(ch.z, ch.w)};
-                            uint32_t cc[4];
+                            const float cf[8] = {cl.x, cl.y, cl.z, cl.w, ch.x, ch.y, ch.z, ch.w};
+                            int q[8];
 #pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const uint64_t x2 = bf2_to_f2(word_of(xr[r][i], k));
-                                const uint64_t yy = NORM ? mul2_rn(mul2_rn(x2, ir2), c2[k]) : (has_vec ? mul2_rn(x2, c2[k]) : x2);
-                                cc[k] = codes2_clamped(mul2_rn(yy, sinv2));
+                            for (int e = 0; e < 8; ++e) {
+                                const uint32_t w = word_of(xr[r][i], e >> 1);
+                                const float x = __uint_as_float((e & 1) ? (w & 0xFFFF0000u) : (w << 16));
+                                const float y = NORM ? __fmul_rn(__fmul_rn(x, ir[r]), cf[e]) : (has_vec ? __fmul_rn(x, cf[e]) : x);
+                                q[e] = code_of_clamped(y, sinv);
                             }
                             if (SQ_CHECK(r0 + r < p.rows, p.status))
-                                qrow[v] = make_uint2(__byte_perm(cc[0], cc[1], 0x5410), __byte_perm(cc[2], cc[3], 0x5410));
+                                qrow[v] = make_uint2(pack4_s8(q[0], q[1], q[2], q[3]), pack4_s8(q[4], q[5], q[6], q[7]));
                         }
                     }
                 }
@@ -609,8 +609,9 @@ __device__ __forceinline__ void rows_body(const RowArgs p, unsigned cta, unsigne
                         if (r < nr && SQ_CHECK(r0 + r < p.rows, p.status)) p.scale[r0 + r] = sdelta;
                 }
             } else {
-                // ---- pass B: y = (x * inv_rms) * c  (or x * c, or x) as element pairs, row maxima
-                uint64_t y[R][VPL][4];
+                // ---- pass B: y = (x * inv_rms) * c  (or x * c, or x; LayerNorm: its own form), row maxima.
+                // Binary32 scalars: each value is rounded exactly as the definition orders it.
+                float yv[R][VPL][8];
                 float m[R];
 #pragma unroll
                 for (int r = 0; r < R; ++r) m[r] = 0.0f;
@@ -620,23 +621,29 @@ __device__ __forceinline__ void rows_body(const RowArgs p, unsigned cta, unsigne
                     const bool in = SQ_COL_IN(v);
                     float4 cl = make_float4(1.f, 1.f, 1.f, 1.f), ch = cl;
                     if (has_vec && in) { cl = c_lo[v]; ch = c_hi[v]; }
-                    uint64_t c2[4] = {pack2(cl.x, cl.y), pack2(cl.z, cl.w), pack2(ch.x, ch.y), pack2(ch.z, ch.w)};
-                    uint64_t b2[4];                             // LayerNorm: beta pairs
-                    if (LN && in) ln_params(c_lo, c_hi, p.vec2, v, c2, b2);
+                    const float cf[8] = {cl.x, cl.y, cl.z, cl.w, ch.x, ch.y, ch.z, ch.w};
+                    uint64_t g2[4], b2[4];                      // LayerNorm: gamma and beta pairs
+                    if (LN && in) ln_params(c_lo, c_hi, p.vec2, v, g2, b2);
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
-                        const uint64_t ir2 = pack2(ir[r], ir[r]);
-                        const uint64_t nm2 = LN ? pack2(-mu[r], -mu[r]) : 0ull;
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            const uint64_t x2 = bf2_to_f2(word_of(xr[r][i], k));
-                            // LayerNorm: an absent vector must not reach the row maximum (its y is not 0)
-                            const uint64_t yy = LN ? (in ? ln_y2(word_of(xr[r][i], k), nm2, ir2, c2[k], b2[k]) : 0ull)
-                                              : NORM ? mul2_rn(mul2_rn(x2, ir2), c2[k]) : (has_vec ? mul2_rn(x2, c2[k]) : x2);
-                            y[r][i][k] = yy;
-                            uint32_t yl, yh;
-                            unpack2(yy, yl, yh);
-                            m[r] = max3f(m[r], fabsf(__uint_as_float(yl)), fabsf(__uint_as_float(yh)));
+                            const uint32_t w = word_of(xr[r][i], k);
+                            float yl, yh;
+                            if (LN) {
+                                // an absent vector must not reach the row maximum (its y is not 0)
+                                uint32_t l = 0u, h = 0u;
+                                if (in) unpack2(ln_y2(w, pack2(-mu[r], -mu[r]), pack2(ir[r], ir[r]), g2[k], b2[k]), l, h);
+                                yl = __uint_as_float(l);
+                                yh = __uint_as_float(h);
+                            } else {
+                                const float xl = __uint_as_float(w << 16), xh = __uint_as_float(w & 0xFFFF0000u);
+                                yl = NORM ? __fmul_rn(__fmul_rn(xl, ir[r]), cf[2 * k]) : (has_vec ? __fmul_rn(xl, cf[2 * k]) : xl);
+                                yh = NORM ? __fmul_rn(__fmul_rn(xh, ir[r]), cf[2 * k + 1]) : (has_vec ? __fmul_rn(xh, cf[2 * k + 1]) : xh);
+                            }
+                            yv[r][i][2 * k] = yl;
+                            yv[r][i][2 * k + 1] = yh;
+                            m[r] = max3f(m[r], fabsf(yl), fabsf(yh));
                         }
                     }
                 }
@@ -654,39 +661,42 @@ __device__ __forceinline__ void rows_body(const RowArgs p, unsigned cta, unsigne
                 float inv_m = mrow > 0.0f ? __fdiv_rn(qmax, mrow) : 0.0f;
                 // A row maximum below qmax / FLT_MAX (about 3.7e-37 for INT8): qmax / m overflows binary32.
                 // Such a row is scaled by 2^64 first (exact: its values are far below the top of the
-                // range) and coded as t = fl(fl(y * 2^64) * fl(qmax / fl(m * 2^64))); the step stays m / qmax.
+                // range) and coded with fl(qmax / fl(m * 2^64)); the step stays m / qmax.
                 const bool tiny = isinf(inv_m);
                 if (tiny) inv_m = __fdiv_rn(qmax, __fmul_rn(mrow, 0x1p64f));
                 if (wig == 0 && (lane % SUB) == 0 && lane / SUB < nr && SQ_CHECK(r0 + lane / SUB < p.rows, p.status))
                     p.scale[r0 + lane / SUB] = delta;
-                // ---- pass C: codes
+                // ---- pass C: codes (INT8: round half away from zero of y * 127/m, exact product;
+                // FP8: e4m3 of fl(y * 448/m))
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
                     const float iv = __shfl_sync(kAll, inv_m, r * SUB);
                     if (__shfl_sync(kAll, tiny ? 1 : 0, r * SUB) != 0) {      // uniform across the row's lanes
-                        const uint64_t up2 = pack2(0x1p64f, 0x1p64f);
 #pragma unroll
                         for (int i = 0; i < VPL; ++i)
 #pragma unroll
-                            for (int k = 0; k < 4; ++k) y[r][i][k] = mul2_rn(y[r][i][k], up2);
+                            for (int e = 0; e < 8; ++e) yv[r][i][e] = __fmul_rn(yv[r][i][e], 0x1p64f);
                     }
                     if (r < nr) {
-                        const uint64_t inv2 = pack2(iv, iv);
                         uint2 *qrow = reinterpret_cast<uint2 *>(p.q + (r0 + r) * static_cast<int64_t>(K));
 #pragma unroll
                         for (int i = 0; i < VPL; ++i) {
                             const int v = i * GT + gtid;
                             if (SQ_COL_IN(v)) {
-                                uint32_t c01, c23, c45, c67;
+                                uint2 out;
                                 if (MODE == MODE_QF8) {
-                                    c01 = f8codes2(mul2_rn(y[r][i][0], inv2)); c23 = f8codes2(mul2_rn(y[r][i][1], inv2));
-                                    c45 = f8codes2(mul2_rn(y[r][i][2], inv2)); c67 = f8codes2(mul2_rn(y[r][i][3], inv2));
+                                    uint32_t c[4];
+#pragma unroll
+                                    for (int k = 0; k < 4; ++k)
+                                        c[k] = f8codes2(__fmul_rn(yv[r][i][2 * k], iv), __fmul_rn(yv[r][i][2 * k + 1], iv));
+                                    out = make_uint2(__byte_perm(c[0], c[1], 0x5410), __byte_perm(c[2], c[3], 0x5410));
+                                    if (iv == 0.0f) out = make_uint2(0u, 0u);   // a zero row: codes +0
                                 } else {
-                                    c01 = codes2(mul2_rn(y[r][i][0], inv2)); c23 = codes2(mul2_rn(y[r][i][1], inv2));
-                                    c45 = codes2(mul2_rn(y[r][i][2], inv2)); c67 = codes2(mul2_rn(y[r][i][3], inv2));
+                                    int q[8];
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) q[e] = code_of(yv[r][i][e], iv);
+                                    out = make_uint2(pack4_s8(q[0], q[1], q[2], q[3]), pack4_s8(q[4], q[5], q[6], q[7]));
                                 }
-                                uint2 out = make_uint2(__byte_perm(c01, c23, 0x5410), __byte_perm(c45, c67, 0x5410));
-                                if (MODE == MODE_QF8 && iv == 0.0f) out = make_uint2(0u, 0u);   // a zero row: codes +0
                                 if (SQ_CHECK(r0 + r < p.rows, p.status)) qrow[v] = out;
                             }
                         }

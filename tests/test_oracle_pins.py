@@ -205,6 +205,37 @@ def test_quantiser_invariants_random(orc):
     assert np.allclose(xs, np.abs(y).max(axis=1) / 127, rtol=3e-7, atol=0)
 
 
+def _near_tie_row():
+    """A row of binary32 values whose products with fl32(127/m) lie within a rounding of k + 1/2:
+    y_k = fl32((k + 1/2) / fl32(127/m)) for k = 0..126, both signs, the row maximum m itself, zeros to 256."""
+    m = np.float32(37.123)
+    inv = np.float32(127.0) / m
+    y = ((np.arange(127) + 0.5) / np.float64(inv)).astype(np.float32)
+    row = np.zeros(256, np.float32)
+    row[0], row[1:128], row[128:255] = m, y, -y
+    return row, m, inv
+
+
+def test_codes_round_the_exact_product(orc):
+    """The INT8 code is round-half-away-from-zero of the exact product v * fl32(127/m), rounded once:
+    checked element by element with exact rational arithmetic on values placed next to the ties
+    k + 1/2, where rounding the product to binary32 first would move a third of them by one code.
+    The values enter as the smoothing factors of a weight row of ones (w' = 1 * s = s exactly)."""
+    from fractions import Fraction
+    row, m, inv = _near_tie_row()
+    ones = bf16_bits(torch.ones(1, 256, dtype=torch.bfloat16))
+    wq, ws = orc.smooth_quantize_weight(ones, row)
+    assert ws[0] == m / np.float32(127) and abs(int(wq[0, 0])) == 127
+
+    def rha(fr):
+        f = int(abs(fr) + Fraction(1, 2))         # floor(|p| + 1/2) for p >= 0
+        return f if fr >= 0 else -f
+    exact = np.array([rha(Fraction(float(v)) * Fraction(float(inv))) for v in row])
+    assert np.array_equal(wq[0].astype(np.int64), np.clip(exact, -127, 127))
+    twice = np.array([rha(Fraction(float(np.float32(np.float64(v) * np.float64(inv))))) for v in row])
+    assert (twice != exact).sum() > 20                # the fixture does tell the two readings apart
+
+
 def _tiny_rows(rows, K, seed):
     """bf16 rows whose largest magnitude lies between the bf16 subnormals and ~1e-37, where 127 / m
     (and 448 / m) overflows binary32; one row is all zero except one subnormal, one is all zero."""

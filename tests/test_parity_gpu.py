@@ -188,10 +188,9 @@ EDGE = [
     (128, 256, 128, True, False),
     (255, 512, 4096, False, False),
     (777, 1288, 2064, True, True),
-    # 192-channel tiles (the 256-wide ones would leave most of a second wave idle), ragged T, N and K
+    # enough 256-channel tiles to take the wide form, with ragged T, N and K
     (2000, 2312, 1040, True, True),
     (1100, 5000, 1040, False, True),
-    # enough 256-channel tiles to take the wide form, with ragged T, N and K
     (2000, 4104, 1040, True, True),
     (64, 37888, 64, False, True),
 ]
@@ -493,6 +492,34 @@ def test_tiny_rows_every_quantiser(sq, orc, T, K):
     st_o, ss_o = orc.rmsnorm_smooth_quant_static(xh, oh, s2_o, apply_norm=False)
     assert np.array_equal(hnp(sq_s), ss_o) and np.array_equal(hnp(sq_q), st_o), "static codes of tiny rows differ"
     assert np.array_equal(st_o, (np.sign(f64(xh)) * 127).astype(np.int8))
+    ok_status(sq)
+
+
+# Values placed next to the ties k + 1/2 of v * fl32(127/m): the codes round the exact product once
+# (a third of these values would move by one code if the product were rounded to binary32 first).
+# They enter as the smoothing factors of weight rows of ones, and as the fold of tokens of ones (no
+# norm), so y = the designed values exactly; 300 rows reach every row geometry's unit layout.
+def test_near_tie_codes_match_the_oracle(sq, orc):
+    dev = "cuda"
+    m = np.float32(37.123)
+    inv = np.float32(127.0) / m
+    y = ((np.arange(127) + 0.5) / np.float64(inv)).astype(np.float32)
+    row = np.zeros(256, np.float32)
+    row[0], row[1:128], row[128:255] = m, y, -y
+    for K in (256, 4096):
+        f = np.tile(row, K // 256)
+        ones = torch.ones(300, K, dtype=torch.bfloat16, device=dev)
+        fd = torch.from_numpy(f).to(dev)
+        wq, ws = sq.sq_smooth_quantize_weight(ones, fd)
+        wq_o, ws_o = orc.smooth_quantize_weight(h16(ones), f)
+        assert np.array_equal(hnp(ws), ws_o) and np.array_equal(hnp(wq), wq_o), f"near-tie weight codes differ (K={K})"
+        xq, xs = sq.sq_rmsnorm_smooth_quant(ones, fd, apply_norm=False)
+        xq_o, xs_o = orc.rmsnorm_smooth_quant(h16(ones), f, apply_norm=False)
+        assert np.array_equal(hnp(xs), xs_o) and np.array_equal(hnp(xq), xq_o), f"near-tie token codes differ (K={K})"
+        s2 = sq.sq_static_scale(torch.full((K,), float(m), dtype=torch.float32, device=dev))
+        sq_q, _ = sq.sq_rmsnorm_smooth_quant_static(ones, fd, s2, apply_norm=False)
+        st_o, _ = orc.rmsnorm_smooth_quant_static(h16(ones), f, hnp(s2), apply_norm=False)
+        assert np.array_equal(hnp(sq_q), st_o), f"near-tie static codes differ (K={K})"
     ok_status(sq)
 
 
