@@ -447,24 +447,37 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t *r) {
         : "r"(taddr));
 }
 
+// Per-channel constants of the swapped (decode) form's epilogue for output channel n (w_scale and the
+// bias widened to binary32; zeros beyond N). Fetched before the tile's accumulator is ready, so their
+// memory latency overlaps the weight stream instead of following it.
+struct SwapCol {
+    float ws, b;
+};
+__device__ __forceinline__ SwapCol swap_col(int n, int N, const float *__restrict__ w_scale,
+                                            const __nv_bfloat16 *__restrict__ bias) {
+    SwapCol c = {0.0f, 0.0f};
+    if (n < N) {
+        c.ws = __ldg(w_scale + n);
+        if (bias != nullptr) c.b = __uint_as_float(static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short *>(bias) + n)) << 16);
+    }
+    return c;
+}
+
 // Epilogue of the swapped (decode) form for one tile: thread (quad, lane) owns output channel
-// n = n_base + 32 quad + lane and writes y[t][n] = bf16(float(acc) * (x_scale[t] * w_scale[n]) + bias[n])
-// (each operation rounded once, the same steps as the other forms) for the tile's tokens t < T; a warp
-// writes 32 consecutive channels of a token per store. Optionally writes the raw accumulators.
+// n = n_base + 32 quad + lane (constants `col`, fetched ahead) and writes
+// y[t][n] = bf16(float(acc) * (x_scale[t] * w_scale[n]) + bias[n]) (each operation rounded once, the same
+// steps as the other forms) for the tile's tokens t < T, with x_scale read from the shared-memory copy
+// `xs` (all T <= 128 tokens); a warp writes 32 consecutive channels of a token per store. Optionally
+// writes the raw accumulators.
 template <int TN, bool F8>
 __device__ __forceinline__ void epilogue_swap(uint32_t tmem_base, int quad, int lane, uint32_t tcol, int n_base, int t0,
-                                              const float *__restrict__ x_scale, const float *__restrict__ w_scale,
-                                              const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ y,
+                                              const float *xs, SwapCol col, bool has_bias, __nv_bfloat16 *__restrict__ y,
                                               int32_t *__restrict__ acc_out, int T, int N)
 {
     const int nq = n_base + quad * 32;
     if (nq >= N) return;                    // the whole quarter lies beyond N
     const int n = nq + lane;
     const bool okn = n < N;
-    const float ws = okn ? __ldg(w_scale + n) : 0.0f;
-    float b = 0.0f;
-    if (bias != nullptr && okn)
-        b = __uint_as_float(static_cast<uint32_t>(__ldg(reinterpret_cast<const unsigned short *>(bias) + n)) << 16);
     const uint32_t tl = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + tcol;
 #pragma unroll
     for (int c = 0; c < TN; c += 16) {
@@ -480,10 +493,10 @@ __device__ __forceinline__ void epilogue_swap(uint32_t tmem_base, int quad, int 
             if (t < T && okn) {
                 const int acc = static_cast<int>(r[j]);
                 const int64_t o = static_cast<int64_t>(t) * N + n;
-                if (!SQ_CHECK(t >= 0 && n >= 0 && o < static_cast<int64_t>(T) * N, &g_sq_status)) continue;
+                if (!SQ_CHECK(t >= 0 && t < BM && n >= 0 && o < static_cast<int64_t>(T) * N, &g_sq_status)) continue;
                 if (acc_out != nullptr) acc_out[o] = acc;
-                float v = __fmul_rn(acc_value<F8>(r[j]), __fmul_rn(__ldg(x_scale + t), ws));
-                if (bias != nullptr) v = __fadd_rn(v, b);
+                float v = __fmul_rn(acc_value<F8>(r[j]), __fmul_rn(xs[t], col.ws));
+                if (has_bias) v = __fadd_rn(v, col.b);
                 y[o] = __float2bfloat16_rn(v);
             }
         }
@@ -623,7 +636,18 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         // ---------------- epilogue ----------------
         const int quad = warp & 3;                  // TMEM lanes this warp may read: 32*quad .. +31
       if constexpr (SWAP) {
+        // the tokens' x_scale (T <= 128) into shared memory (the column-table area, unused by this
+        // form) while the weight streams; the first tile's channel constants likewise
+        const int ep = threadIdx.x - 64;
+        if (ep < T && SQ_CHECK(ep < BM, &g_sq_status)) sCol[ep] = __ldg(x_scale + ep);
+        named_sync(EPI_BAR, EPI_THREADS);
         int lt = 0;
+        SwapCol col = {0.0f, 0.0f};
+        if (static_cast<int>(blockIdx.x) < num_tiles) {
+            int m, n;
+            tile_coords(blockIdx.x, m_tiles, n_tiles, m, n);
+            col = swap_col(m * BM + quad * 32 + lane, N, w_scale, bias);
+        }
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++lt) {
             const int buf = lt & 1;
             const uint32_t use = static_cast<uint32_t>(lt >> 1);
@@ -631,8 +655,15 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             tc_fence_after();
             int m, n;
             tile_coords(t, m_tiles, n_tiles, m, n);
-            epilogue_swap<TN, F8>(tmem_base, quad, lane, static_cast<uint32_t>(buf) * L::ACC_STRIDE, m * BM, n * TN, x_scale, w_scale,
-                              bias, y, acc_out, T, N);
+            const SwapCol cur = col;
+            const int tn = t + static_cast<int>(gridDim.x);
+            if (tn < num_tiles) {                   // the next tile's constants, ahead of its accumulator
+                int m2, n2;
+                tile_coords(tn, m_tiles, n_tiles, m2, n2);
+                col = swap_col(m2 * BM + quad * 32 + lane, N, w_scale, bias);
+            }
+            epilogue_swap<TN, F8>(tmem_base, quad, lane, static_cast<uint32_t>(buf) * L::ACC_STRIDE, m * BM, n * TN, sCol, cur,
+                                  bias != nullptr, y, acc_out, T, N);
             tc_fence_before();
             mbar_arrive(tempty(buf));
         }

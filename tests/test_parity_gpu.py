@@ -193,6 +193,9 @@ EDGE = [
     (1100, 5000, 1040, False, True),
     (2000, 4104, 1040, True, True),
     (64, 37888, 64, False, True),
+    # decode form with ragged N (a partial last weight tile) and T just below its 16 / 128 buckets
+    (33, 14344, 1040, True, True),
+    (128, 1000, 272, False, False),
 ]
 
 
