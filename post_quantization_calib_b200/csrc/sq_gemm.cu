@@ -11,7 +11,7 @@
 // The pages name the operation, not a kernel design (their INT8 kernels target earlier tensor-core
 // generations). This kernel is written for B200:
 //   * persistent: one CTA per SM (the shared-memory footprint admits exactly one), tiles
-//     128 tokens x 256 output channels handed out round-robin in bands of 32 M tiles for L2 reuse;
+//     128 tokens x 256 output channels handed out round-robin in bands of 16 or 32 M tiles for L2 reuse;
 //   * warp 0 (one lane) streams 128-byte K slices of both operands into a 4-stage shared-memory
 //     ring with TMA (128-byte swizzle), completion tracked by mbarrier transaction counts;
 //   * warp 1 (one lane) issues tcgen05.mma.kind::i8 (M=128, N=256, K=32, signed x signed -> s32)
@@ -63,12 +63,16 @@ constexpr int OUT_COLS = 32;       // bf16 columns per TMA store box (64 bytes, 
 constexpr int OUT_ROWS = 32;       // rows per box: one warp's TMEM lane quarter
 constexpr int OUT_BOX = OUT_COLS * 2 * OUT_ROWS;
 constexpr int THREADS = 64 + 32 * EPI_WARPS;
-// M tiles per raster band. Every band streams the whole weight from DRAM, so wider bands read less
-// (the 70B-shaped MLP up-projection, T 16384, K 8192, N 28672: 2.02 GB read per call with bands of
-// 16, 1.14 GB with 32); the GEMM runs at the power limit, and the DRAM power saved raised the
-// sustained clock (1462 -> 1485 MHz, 2713 -> 2766 TOPS on one B200). Bands of 64 token tiles (67 MB of
-// tokens at K = 8192) no longer stay in the L2 and read 6.6 GB.
-constexpr int BAND = 32;
+// M tiles per raster band, chosen per call (band_for below). Every band streams the whole weight,
+// so when the weight does not fit the L2 wider bands read less from DRAM (the 70B-shaped MLP
+// up-projection, T 16384, K 8192, N 28672: 2.02 GB read per call with bands of 16, 1.16 GB with 32).
+// The GEMM runs at the power limit, and the DRAM power saved raised the sustained clock and rate
+// (1440 -> 1466 MHz, 2674 -> 2733 TOPS; gate+up N 28672, K 4096: 2494 -> 2567 TOPS). With a weight that
+// the L2 holds, 16 is slightly better (query projection N = K = 4096: 2450 against 2427 TOPS). Bands of
+// 64 token tiles (67 MB of tokens at K = 8192) no longer stay in the L2 and read 6.6 GB.
+constexpr int BAND_SMALL = 16;
+constexpr int BAND_LARGE = 32;
+int band_for(int64_t N, int64_t K) { return N * K > (int64_t(64) << 20) ? BAND_LARGE : BAND_SMALL; }
 constexpr int COL_TAB = 2 * BN * 4;   // w_scale and bias (binary32) of up to 256 columns
 
 // Instruction descriptor of tcgen05.mma.kind::i8: D = s32, A and B signed 8-bit, both K-major,
@@ -204,7 +208,7 @@ __device__ __forceinline__ uint64_t kmajor_sw128_desc(uint32_t saddr) {
            (static_cast<uint64_t>(2u) << 61);
 }
 
-__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int &m, int &n) {
+__device__ __forceinline__ void tile_coords(int t, int m_tiles, int n_tiles, int BAND, int &m, int &n) {
     const int per_band = BAND * n_tiles;
     const int band = t / per_band;
     const int within = t - band * per_band;
@@ -511,7 +515,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
               const __grid_constant__ CUtensorMap tmY, const float *__restrict__ x_scale,
               const float *__restrict__ w_scale, const __nv_bfloat16 *__restrict__ bias,
               int32_t *__restrict__ acc_out, __nv_bfloat16 *__restrict__ y, int T, int N, int K, int m_tiles,
-              int n_tiles, uint64_t limit_ns)
+              int n_tiles, int band, uint64_t limit_ns)
 {
     using L = Tile<TN, SWAP>;
     constexpr int STAGES = L::STAGES;
@@ -565,7 +569,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             bool ok = true;
             for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
                 int m, n;
-                tile_coords(t, m_tiles, n_tiles, m, n);
+                tile_coords(t, m_tiles, n_tiles, band, m, n);
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait(empty(stage), phase ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
                     mbar_expect_tx(full(stage), stage_tx);
@@ -645,7 +649,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         SwapCol col = {0.0f, 0.0f};
         if (static_cast<int>(blockIdx.x) < num_tiles) {
             int m, n;
-            tile_coords(blockIdx.x, m_tiles, n_tiles, m, n);
+            tile_coords(blockIdx.x, m_tiles, n_tiles, band, m, n);
             col = swap_col(m * BM + quad * 32 + lane, N, w_scale, bias);
         }
         for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++lt) {
@@ -654,12 +658,12 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             if (!mbar_wait(tfull(buf), use & 1u, limit_ns, abort_flag)) { give_up(abort_flag); break; }
             tc_fence_after();
             int m, n;
-            tile_coords(t, m_tiles, n_tiles, m, n);
+            tile_coords(t, m_tiles, n_tiles, band, m, n);
             const SwapCol cur = col;
             const int tn = t + static_cast<int>(gridDim.x);
             if (tn < num_tiles) {                   // the next tile's constants, ahead of its accumulator
                 int m2, n2;
-                tile_coords(tn, m_tiles, n_tiles, m2, n2);
+                tile_coords(tn, m_tiles, n_tiles, band, m2, n2);
                 col = swap_col(m2 * BM + quad * 32 + lane, N, w_scale, bias);
             }
             epilogue_swap<TN, F8>(tmem_base, quad, lane, static_cast<uint32_t>(buf) * L::ACC_STRIDE, m * BM, n * TN, sCol, cur,
@@ -678,7 +682,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         auto prefetch = [&](int t) {
             if (t >= num_tiles) return;
             int m, n;
-            tile_coords(t, m_tiles, n_tiles, m, n);
+            tile_coords(t, m_tiles, n_tiles, band, m, n);
             cols_fetch<TN>(cols, n * TN, ep, w_scale, bias, N);
             const int row = m * BM + quad * 32 + lane;
             xs = row < T ? __ldg(x_scale + row) : 0.0f;
@@ -694,7 +698,7 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             if (named_sync_or(EPI_BAR, EPI_THREADS, !ok)) { give_up(abort_flag); break; }
             tc_fence_after();
             int m, n;
-            tile_coords(t, m_tiles, n_tiles, m, n);
+            tile_coords(t, m_tiles, n_tiles, band, m, n);
             const float xs_t = xs;
             prefetch(t + gridDim.x);
             epilogue_rows<TN, F8>(tmem_base, quad, lane, static_cast<uint32_t>(buf) * L::ACC_STRIDE, m * BM + quad * 32, n * TN, xs_t, tab,
@@ -740,7 +744,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmY, const float *__restrict__ x_scale,
                    const float *__restrict__ w_scale, const __nv_bfloat16 *__restrict__ bias,
-                   int32_t *__restrict__ acc_out, int T, int N, int K, int m_tiles, int n_tiles,
+                   int32_t *__restrict__ acc_out, int T, int N, int K, int m_tiles, int n_tiles, int band,
                    uint64_t limit_ns)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -796,7 +800,7 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             bool ok = true;
             for (int t = cid; t < num_tiles && ok; t += ncl) {
                 int m, n;
-                tile_coords(t, m_tiles, n_tiles, m, n);
+                tile_coords(t, m_tiles, n_tiles, band, m, n);
                 for (int kb = 0; kb < k_blocks; ++kb) {
                     if (!mbar_wait_cluster(empty(stage), phase ^ 1u, limit_ns, abort_flag)) { ok = false; break; }
                     if (rank == 0) mbar_expect_tx(full(stage), 2u * (P_A_STAGE + P_B_STAGE));
@@ -861,7 +865,7 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         auto prefetch = [&](int t) {
             if (t >= num_tiles) return;
             int m, n;
-            tile_coords(t, m_tiles, n_tiles, m, n);
+            tile_coords(t, m_tiles, n_tiles, band, m, n);
             cols_fetch<BN>(cols, n * BN, ep, w_scale, bias, N);
             const int row = m * 2 * BM + static_cast<int>(rank) * BM + quad * 32 + lane;
             xs = row < T ? __ldg(x_scale + row) : 0.0f;
@@ -876,7 +880,7 @@ k_w8a8_linear_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constan
             if (named_sync_or(EPI_BAR, EPI_THREADS, !ok)) { give_up(abort_flag); break; }
             tc_fence_after();
             int m, n;
-            tile_coords(t, m_tiles, n_tiles, m, n);
+            tile_coords(t, m_tiles, n_tiles, band, m, n);
             const float xs_t = xs;
             prefetch(t + ncl);
             epilogue_rows<BN, false>(tmem_base, quad, lane, static_cast<uint32_t>(buf * BN),
@@ -1005,7 +1009,7 @@ sq_status launch_single(const CUtensorMap &mA, const CUtensorMap &mB, const CUte
         sq::launch_pdl(k_w8a8_linear<TN, SWAP, F8>, dim3(grid), dim3(THREADS), L::SMEM_TOTAL, sq::as_stream(stream), nullptr,
                        mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out,
                        static_cast<__nv_bfloat16 *>(y), static_cast<int>(T), static_cast<int>(N), static_cast<int>(K), m_tiles,
-                       n_tiles, sq::wait_timeout_ns(dev)),
+                       n_tiles, band_for(N, K), sq::wait_timeout_ns(dev)),
         "launch(w8a8_linear)");
 }
 
@@ -1094,7 +1098,7 @@ sq_status linear_impl(const void *xq, const float *x_scale, int64_t T, const voi
             sq::launch_pdl(k_w8a8_linear_pair, dim3(2 * clusters), dim3(THREADS), P_SMEM_TOTAL, sq::as_stream(stream), &attr[0],
                            mA, mB, mY, x_scale, w_scale, reinterpret_cast<const __nv_bfloat16 *>(bias), acc_out,
                            static_cast<int>(T), static_cast<int>(N), static_cast<int>(K), m_tiles, n_tiles,
-                           sq::wait_timeout_ns(dev)),
+                           band_for(N, K), sq::wait_timeout_ns(dev)),
             "launch(w8a8_linear_pair)");
     }
 
