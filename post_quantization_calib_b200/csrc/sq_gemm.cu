@@ -165,6 +165,14 @@ __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.a
 __device__ __forceinline__ void prefetch_map(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
+// L2 prefetch of one 8-bit tensor box (a hint: no shared memory is written and nothing completes on a
+// barrier). The innermost coordinate c0 must be a multiple of 16 elements, as for the loads.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int c0, int c1) {
+    if (!SQ_CHECK(c0 >= 0 && (c0 & 15) == 0, &g_sq_status)) return;
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1)
+                 : "memory");
+}
 
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(ncols) : "memory");
@@ -545,13 +553,29 @@ k_w8a8_linear(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         mbar_init_fence();
         fence_async_smem();
     }
-    if (warp == 0 && lane == 0) { prefetch_map(&tmA); prefetch_map(&tmB); prefetch_map(&tmY); }
+    if (warp == 0 && lane == 0) {
+        prefetch_map(&tmA); prefetch_map(&tmB); prefetch_map(&tmY);
+        if (SWAP && static_cast<int>(blockIdx.x) < m_tiles * n_tiles) {
+            // Decode form: the first two stages of this CTA's weight rows (64 KB) are requested into
+            // the L2 while the previous kernel of the stream finishes, so the first loads after the
+            // dependency wait find them there (a whole ring's worth, most of the weight, competed with
+            // the previous call's own stream). Only a cache hint: the loads themselves still follow the wait, and
+            // the L2 is where every writer's data meets, so a weight written by that kernel is still
+            // read as written.
+            int m, n;
+            tile_coords(blockIdx.x, m_tiles, n_tiles, band, m, n);
+            const int kbs = (K + L::KS * BK - 1) / (L::KS * BK);
+            for (int kb = 0; kb < 2 && kb < kbs; ++kb)
+                for (int ks = 0; ks < L::KS; ++ks) tma_prefetch_l2_2d(&tmA, (kb * L::KS + ks) * BK, m * BM);
+        }
+    }
     if (warp == 1) { tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS); tmem_relinquish(); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
-    // dependent launch: the set-up above touched shared and tensor memory only
+    // dependent launch: the set-up above touched shared and tensor memory only (and, in the decode
+    // form, sent L2 prefetch hints)
     pdl_wait();
     pdl_trigger();
 
