@@ -10,6 +10,10 @@ Each stage runs through the C ABI on the workload's seeded synthetic inputs (``s
   weight_quant       S4: diag(s) W quantised to INT8 per output channel
   act_quant          S5: fused RMSNorm(gamma / s) + per-token INT8 of the workload's T tokens
   gemm               S6 + S7: INT8 GEMM with the dequant epilogue to bf16
+The variant paths are timed only when named with --stage: act_quant_static (static per-tensor scale),
+act_quant_fp8 and weight_quant_fp8 (E4M3 codes), gemm_fp8 (kind::f8f6f4 GEMM), act_quant_layernorm
+(LayerNorm with gamma / s and beta / s folded), calib_absmax_layernorm (abs-max of the calibration set's
+LayerNorm output) and fold_prev_linear (1/s folded into a previous [K, N] linear layer and its bias).
 Decode workloads add act_quant and gemm at each decode token count, once as a single call and once per
 call in a chain of 8 back-to-back calls captured in a CUDA graph (the way a decoder runs one layer after
 another, without the host's per-call cost; the 8 GEMMs read 8 distinct copies of the weight, which
@@ -129,6 +133,14 @@ def line(peaks: Dict, workload: str, group: int, stage: str, us: float, nbytes: 
 
 
 STAGES = ("calib_absmax_pair", "scales", "weight_quant", "act_quant", "gemm")
+# Variant paths, timed only when asked for (--stage): the static per-tensor activation quantiser (its
+# scale from the calibration abs-max of the quantiser's own y), the FP8 E4M3 per-token quantiser, the
+# LayerNorm-fed quantiser (gamma and beta folded; the tokens' own LayerNorm stands in for the RMSNorm),
+# the FP8 weight quantiser and the FP8 GEMM; the LayerNorm calibration abs-max and the fold of 1/s into
+# a previous linear layer (a [K, N] weight and bias: the layer whose output feeds this one), both timed
+# once per group.
+VARIANTS = ("act_quant_static", "act_quant_fp8", "act_quant_layernorm", "weight_quant_fp8", "gemm_fp8",
+            "calib_absmax_layernorm", "fold_prev_linear")
 
 
 def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device, stages=STAGES,
@@ -184,6 +196,8 @@ def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device, stages=ST
                 quant()
             if "gemm" in stages:
                 rows.append(line(peaks, w.name, g, "gemm", timer.single(gemm), gbytes, ops, T=T, N=N, K=K))
+            if any(v in stages for v in VARIANTS):
+                rows.extend(run_variants(w, g, peaks, timer, stages, x, fold, W, s, calib, bias, gamma, T, N, K, device))
             if T in w.decode_T and "gemm" in stages and "act_quant" in stages:
                 # a decoder's consecutive layers: each GEMM streams its own weight (8 together exceed
                 # the L2); the activations are small and stay in L2 either way
@@ -202,10 +216,77 @@ def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device, stages=ST
     return rows
 
 
+def run_variants(w, g, peaks, timer, stages, x, fold, W, s, calib, bias, gamma, T, N, K, device) -> List[Dict]:
+    """The variant paths at the workload's shapes (the stages named in VARIANTS that `stages` asks for)."""
+    rows: List[Dict] = []
+    qbytes = 3 * T * K + 4 * K + 4 * T
+    xq = torch.empty(T, K, dtype=torch.int8, device=device)
+    xs = torch.empty(T, dtype=torch.float32, device=device)
+    if "act_quant_static" in stages:
+        amax_y = torch.empty(K, dtype=torch.float32, device=device)
+        if w.norm:
+            sq.sq_calibrate_absmax(calib, norm_gamma=fold, eps=w.eps, amax=amax_y)
+            s2 = sq.sq_static_scale(amax_y)
+        else:
+            sq.sq_calibrate_absmax(calib, amax=amax_y)
+            s2 = sq.sq_static_scale(amax_y, factor=fold)
+        f = lambda: sq.sq_rmsnorm_smooth_quant_static(x, fold, s2, eps=w.eps, apply_norm=w.norm, xq=xq, x_scale=xs)
+        rows.append(line(peaks, w.name, g, "act_quant_static", timer.single(f), qbytes, T=T, K=K))
+    if "act_quant_fp8" in stages or "gemm_fp8" in stages:
+        xq8 = torch.empty(T, K, dtype=torch.uint8, device=device)
+        xs8 = torch.empty(T, dtype=torch.float32, device=device)
+        f = lambda: sq.sq_rmsnorm_smooth_quant_fp8(x, fold, eps=w.eps, apply_norm=w.norm, xq=xq8, x_scale=xs8)
+        us = timer.single(f)
+        if "act_quant_fp8" in stages:
+            rows.append(line(peaks, w.name, g, "act_quant_fp8", us, qbytes, T=T, K=K))
+    if "act_quant_layernorm" in stages:
+        beta = 0.05 * torch.randn(K, generator=torch.Generator(device=device).manual_seed(7), device=device)
+        g_ln = gamma if gamma is not None else torch.ones(K, dtype=torch.float32, device=device)
+        f_ln = torch.empty(K, dtype=torch.float32, device=device)
+        s_ln = torch.empty(K, dtype=torch.float32, device=device)
+        amax_ln = sq.sq_calibrate_absmax_layernorm(calib, g_ln, beta)
+        sq.sq_compute_scales(amax_ln, sq.sq_calibrate_absmax(W), w.alpha, gamma=g_ln, s=s_ln, fold=f_ln)
+        bf = sq.sq_fold_layernorm_bias(beta, s_ln)
+        f = lambda: sq.sq_layernorm_smooth_quant(x, f_ln, bf, xq=xq, x_scale=xs)
+        rows.append(line(peaks, w.name, g, "act_quant_layernorm", timer.single(f), qbytes + 4 * K, T=T, K=K))
+    if "weight_quant_fp8" in stages or "gemm_fp8" in stages:
+        wq8 = torch.empty(N, K, dtype=torch.uint8, device=device)
+        ws8 = torch.empty(N, dtype=torch.float32, device=device)
+        f = lambda: sq.sq_smooth_quantize_weight_fp8(W, s, wq=wq8, w_scale=ws8)
+        us = timer.single(f)
+        if "weight_quant_fp8" in stages:
+            rows.append(line(peaks, w.name, g, "weight_quant_fp8", us, 3 * N * K + 4 * K + 4 * N, N=N, K=K))
+    if "gemm_fp8" in stages:
+        y = torch.empty(T, N, dtype=torch.bfloat16, device=device)
+        f = lambda: sq.sq_w8a8_linear_fp8(xq8, xs8, wq8, ws8, bias=bias, y=y)
+        gbytes = T * K + N * K + 2 * T * N + 4 * T + 4 * N + (2 * N if bias is not None else 0)
+        rows.append(line(peaks, w.name, g, "gemm_fp8", timer.single(f), gbytes, 2 * T * N * K, T=T, N=N, K=K))
+    if T == w.T and "calib_absmax_layernorm" in stages:
+        g_ln = gamma if gamma is not None else torch.ones(K, dtype=torch.float32, device=device)
+        beta = torch.zeros(K, dtype=torch.float32, device=device)
+        amax_ln = torch.empty(K, dtype=torch.float32, device=device)
+        f = lambda: sq.sq_calibrate_absmax_layernorm(calib, g_ln, beta, amax=amax_ln)
+        R = calib.shape[0]
+        rows.append(line(peaks, w.name, g, "calib_absmax_layernorm", timer.single(f), 2 * R * K + 12 * K,
+                         rows=R, K=K))
+    if T == w.T and "fold_prev_linear" in stages:
+        gen = torch.Generator(device=device).manual_seed(11)
+        wp = (0.02 * torch.randn(K, N, generator=gen, device=device)).to(torch.bfloat16)
+        bp = (0.01 * torch.randn(K, generator=gen, device=device)).to(torch.bfloat16)
+        wp_out = torch.empty_like(wp)
+        bp_out = torch.empty_like(bp)
+        f = lambda: sq.sq_fold_into_prev_linear(wp, fold, bp, w_out=wp_out, b_out=bp_out)
+        rows.append(line(peaks, w.name, g, "fold_prev_linear", timer.single(f), 4 * K * N + 8 * K,
+                         rows=K, cols=N))
+        del wp, wp_out
+    return rows
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--workload", action="append", help="workload name (repeatable; default: all five)")
-    ap.add_argument("--stage", action="append", choices=STAGES, help="stage to time (repeatable; default: all)")
+    ap.add_argument("--stage", action="append", choices=STAGES + VARIANTS,
+                    help="stage to time (repeatable; default: the five stages of the path; the variants only when named)")
     ap.add_argument("--tokens", action="append", type=int, help="token count (repeatable; default: the workload's)")
     ap.add_argument("--reps", type=int, default=20)
     args = ap.parse_args(argv)
