@@ -18,7 +18,9 @@ Decode workloads add act_quant and gemm at each decode token count, once as a si
 call in a chain of 8 back-to-back calls captured in a CUDA graph (the way a decoder runs one layer after
 another, without the host's per-call cost; the 8 GEMMs read 8 distinct copies of the weight, which
 together exceed the L2). The GEMM chain is also timed issued call by call on the stream ("chain_form":
-"stream"), where each call's dependent launch overlaps the previous call's end.
+"stream"), where each call's dependent launch overlaps the previous call's end. The HBM-bound stages
+(calib_absmax_pair, weight_quant, act_quant) are likewise timed per call in a CUDA graph of 8 calls on 8
+copies of their inputs ("chain": 8), unless --no-chain is given.
 
 Times are medians of CUDA-event intervals on the launching stream, with the L2 flushed (a 256 MB read)
 before every repetition. Rates are algorithmic bytes (or 2 x multiply-adds) over that
@@ -54,15 +56,24 @@ def load_peaks() -> Dict:
 
 class Timer:
     """CUDA-event medians on the current stream, L2 flushed before each repetition by reading a 256 MB
-    buffer (a read leaves clean lines, so no write-back of the flush lands inside the timed call)."""
+    buffer (a read leaves clean lines, so no write-back of the flush lands inside the timed call).
 
-    def __init__(self, device, reps: int):
+    With `hold` (the default) a spin kernel of about 100 us follows the flush, so that the host has
+    queued the timed call before the first event fires: the interval is then the call's device time
+    (its launch on the device included), not the host's marshalling and launch cost."""
+
+    HOLD_CYCLES = 200_000
+
+    def __init__(self, device, reps: int, hold: bool = True):
         self.reps = reps
+        self.hold = hold
         self.flush = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
         self.sink = torch.empty((), dtype=torch.float32, device=device)
 
     def clear_l2(self) -> None:
         torch.sum(self.flush, dim=0, out=self.sink)
+        if self.hold:
+            torch.cuda._sleep(self.HOLD_CYCLES)
 
     def single(self, fn: Callable[[], None]) -> float:
         fn()
@@ -143,11 +154,16 @@ VARIANTS = ("act_quant_static", "act_quant_fp8", "act_quant_layernorm", "weight_
             "calib_absmax_layernorm", "fold_prev_linear")
 
 
+CHAIN = 8   # calls per timed chain (each on its own copy of the inputs, together beyond the L2)
+
+
 def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device, stages=STAGES,
-                 tokens: Optional[List[int]] = None) -> List[Dict]:
+                 tokens: Optional[List[int]] = None, chain: bool = True) -> List[Dict]:
     """The workload's stages (those in `stages`; the others still run once, untimed, where a later
     stage needs their output), at the workload's token count and its decode token counts (or at
-    `tokens`)."""
+    `tokens`). With `chain`, the HBM-bound stages at the workload's own token count are also timed per
+    call in a CUDA graph of CHAIN calls on distinct copies of their inputs ("chain": CHAIN): the way
+    they run inside a model, without the fixed cost of one event-timed launch."""
     rows: List[Dict] = []
     K = w.K
     for g in range(w.groups):
@@ -160,10 +176,17 @@ def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device, stages=ST
         aw = torch.empty(K, dtype=torch.float32, device=device)
         pair = lambda: sq.sq_calibrate_absmax_pair(calib, W, norm_gamma=gamma, eps=w.eps, amax=amax, amax_w=aw)
         if "calib_absmax_pair" in stages:
-            rows.append(line(peaks, w.name, g, "calib_absmax_pair", timer.single(pair),
-                             2 * R * K + 2 * N * K + 12 * K, rows=R, N=N, K=K))
-        else:
-            pair()
+            pbytes = 2 * R * K + 2 * N * K + 12 * K
+            rows.append(line(peaks, w.name, g, "calib_absmax_pair", timer.single(pair), pbytes, rows=R, N=N, K=K))
+            if chain:
+                copies = [(calib, W)] + [(calib.clone(), W.clone()) for _ in range(CHAIN - 1)]
+                fns = [lambda c=c, m=m: sq.sq_calibrate_absmax_pair(c, m, norm_gamma=gamma, eps=w.eps, amax=amax, amax_w=aw)
+                       for c, m in copies]
+                rows.append(line(peaks, w.name, g, "calib_absmax_pair", timer.chained(fns), pbytes, rows=R, N=N, K=K,
+                                 chain=CHAIN))
+                del copies, fns
+                torch.cuda.empty_cache()
+        pair()
         s = torch.empty(K, dtype=torch.float32, device=device)
         fold = torch.empty(K, dtype=torch.float32, device=device)
         scales = lambda: sq.sq_compute_scales(amax, aw, w.alpha, gamma=gamma, s=s, fold=fold)
@@ -175,10 +198,15 @@ def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device, stages=ST
         ws = torch.empty(N, dtype=torch.float32, device=device)
         wquant = lambda: sq.sq_smooth_quantize_weight(W, s, wq=wq, w_scale=ws)
         if "weight_quant" in stages:
-            rows.append(line(peaks, w.name, g, "weight_quant", timer.single(wquant), 3 * N * K + 4 * K + 4 * N,
-                             N=N, K=K))
-        else:
-            wquant()
+            wbytes = 3 * N * K + 4 * K + 4 * N
+            rows.append(line(peaks, w.name, g, "weight_quant", timer.single(wquant), wbytes, N=N, K=K))
+            if chain:
+                copies = [W] + [W.clone() for _ in range(CHAIN - 1)]
+                fns = [lambda m=m: sq.sq_smooth_quantize_weight(m, s, wq=wq, w_scale=ws) for m in copies]
+                rows.append(line(peaks, w.name, g, "weight_quant", timer.chained(fns), wbytes, N=N, K=K, chain=CHAIN))
+                del copies, fns
+                torch.cuda.empty_cache()
+        wquant()
         token_counts = tokens if tokens else [w.T] + [t for t in w.decode_T if t != w.T]
         for T in token_counts:
             x = X[:T] if T <= X.shape[0] else synth.outlier_tokens(T, K, d["channels"], synth.seed_for(w.index, "x", g), device)
@@ -192,8 +220,13 @@ def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device, stages=ST
             ops = 2 * T * N * K
             if "act_quant" in stages:
                 rows.append(line(peaks, w.name, g, "act_quant", timer.single(quant), qbytes, T=T, K=K))
-            else:
-                quant()
+                if chain and T == w.T and T not in w.decode_T:
+                    copies = [x] + [x.clone() for _ in range(CHAIN - 1)]
+                    fns = [lambda c=c: sq.sq_rmsnorm_smooth_quant(c, fold, eps=w.eps, apply_norm=w.norm, xq=xq, x_scale=xs)
+                           for c in copies]
+                    rows.append(line(peaks, w.name, g, "act_quant", timer.chained(fns), qbytes, T=T, K=K, chain=CHAIN))
+                    del copies, fns
+            quant()
             if "gemm" in stages:
                 rows.append(line(peaks, w.name, g, "gemm", timer.single(gemm), gbytes, ops, T=T, N=N, K=K))
             if any(v in stages for v in VARIANTS):
@@ -289,17 +322,21 @@ def main(argv=None) -> int:
                     help="stage to time (repeatable; default: the five stages of the path; the variants only when named)")
     ap.add_argument("--tokens", action="append", type=int, help="token count (repeatable; default: the workload's)")
     ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--no-chain", action="store_true", help="single calls only (no chains of calls in a CUDA graph)")
+    ap.add_argument("--no-hold", action="store_true",
+                    help="no spin kernel between the flush and the timed call (the host's launch cost may then enter)")
     args = ap.parse_args(argv)
     if not torch.cuda.is_available():
         print("perf: needs a CUDA device", file=sys.stderr)
         return 2
     device = torch.device("cuda", torch.cuda.current_device())
     peaks = load_peaks()
-    timer = Timer(device, args.reps)
+    timer = Timer(device, args.reps, hold=not args.no_hold)
     names = args.workload or [w.name for w in synth.WORKLOADS]
     for n in names:
         for r in run_workload(synth.workload(n), timer, peaks, device, stages=tuple(args.stage or STAGES),
-                              tokens=args.tokens):
+                              tokens=args.tokens, chain=not args.no_chain):
+            r["host_ahead"] = timer.hold
             print(json.dumps(r), flush=True)
     return 0
 

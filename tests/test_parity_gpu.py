@@ -328,10 +328,27 @@ FEW_ROWS = [(1, 4096), (7, 2568), (64, 8192), (300, 6144), (592, 4096), (593, 40
 
 @pytest.mark.parametrize("T,K", FEW_ROWS)
 def test_quantisers_over_few_rows(sq, orc, T, K):
+    every_quantiser(sq, orc, T, K, 21)
+
+
+# The quantisers at the ends of their width range: the narrowest rows (one lane vector, eight rows to a
+# warp) and the widest the row kernels hold (16384 elements), full and one vector short of full, at
+# token counts that leave a ragged last unit.
+WIDTHS = [(1, 8), (333, 8), (3001, 16), (37, 24), (5, 16384), (300, 16384), (129, 16376)]
+
+
+@pytest.mark.parametrize("T,K", WIDTHS)
+def test_quantisers_at_the_width_limits(sq, orc, T, K):
+    every_quantiser(sq, orc, T, K, 31)
+
+
+def every_quantiser(sq, orc, T, K, seed):
+    """Dynamic INT8 and FP8, static INT8 (with clipping), LayerNorm INT8 and the weight quantiser on
+    T rows of K elements, each against the oracle (codes and scales bit-exact)."""
     dev = "cuda"
-    ch = synth.outlier_channels(K, synth.OutlierSpec(max(1, K // 256), 10, 40), 21)
-    x = synth.outlier_tokens(T, K, ch, 22, dev)
-    fold = synth.norm_gamma(K, 23, dev)
+    ch = synth.outlier_channels(K, synth.OutlierSpec(max(1, K // 256), 10, 40), seed)
+    x = synth.outlier_tokens(T, K, ch, seed + 1, dev)
+    fold = synth.norm_gamma(K, seed + 2, dev)
     x_h, f_h = h16(x), hnp(fold)
     for norm in (True, False):
         q, sc = sq.sq_rmsnorm_smooth_quant(x, fold, apply_norm=norm)
@@ -347,11 +364,11 @@ def test_quantisers_over_few_rows(sq, orc, T, K):
         q, sc = sq.sq_rmsnorm_smooth_quant_static(x, fold, torch.from_numpy(s2).to(dev), apply_norm=norm)
         rq, rs = orc.rmsnorm_smooth_quant_static(x_h, f_h, s2, apply_norm=norm)
         assert np.array_equal(hnp(q), rq) and np.array_equal(hnp(sc), rs)
-    beta = synth.norm_gamma(K, 24, dev) - 1.0
+    beta = synth.norm_gamma(K, seed + 3, dev) - 1.0
     q, sc = sq.sq_layernorm_smooth_quant(x + 3, fold, beta)
     rq, rs = orc.layernorm_smooth_quant(h16(x + 3), f_h, hnp(beta))
     assert np.array_equal(hnp(q), rq) and np.array_equal(hnp(sc), rs)
-    w = synth.normal_weight(T, K, 25, dev)              # a weight with as few output channels
+    w = synth.normal_weight(T, K, seed + 4, dev)        # a weight with as few output channels
     q, sc = sq.sq_smooth_quantize_weight(w, fold)
     rq, rs = orc.smooth_quantize_weight(h16(w), f_h)
     assert np.array_equal(hnp(q), rq) and np.array_equal(hnp(sc), rs)
