@@ -107,6 +107,8 @@ struct RowArgs {
     int stream_once;        // input larger than half the L2: its lines are evicted first
     int early;              // ABSMAX modes launched right after this library's zero-fill of amax: the
                             // rows may be read before pdl_wait(); amax is touched only after it
+    int group_major;        // unit numbering across the grid: 1 = group by group over all CTAs (few units
+                            // per group: each SM gets an equal share), 0 = CTA by CTA
 };
 
 // 1 / sqrt(ss / K + eps) with each step rounded as the RMSNorm definition orders it. When K is a
@@ -336,7 +338,8 @@ __device__ __forceinline__ void rows_body(const RowArgs p, unsigned cta, unsigne
     float sdelta = 0.0f, sinv = 0.0f;
 
     const int64_t units = (p.rows + R - 1) / R;
-    const int64_t g0 = static_cast<int64_t>(cta) * G + group;
+    // first unit of this group; the group then takes every gstride-th unit
+    const int64_t g0 = p.group_major ? static_cast<int64_t>(group) * nctas + cta : static_cast<int64_t>(cta) * G + group;
     const int64_t gstride = static_cast<int64_t>(nctas) * G;
     const int64_t nunits = g0 < units ? (units - 1 - g0) / gstride + 1 : 0;
 
@@ -950,7 +953,14 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
     if (a.status == nullptr) return sq::fail(SQ_ERR_CUDA, "device status word unavailable");
     const int64_t units = (a.rows + R - 1) / R;
     if (!ABS) {
-        int64_t ctas = (units + G - 1) / G;
+        // Up to 4 units per row group: units are numbered group by group across the CTAs, so every SM
+        // gets an equal share (CTA by CTA, a third of the SMs would take a whole extra unit per group
+        // at 4096 rows), and below one unit per SM each unit gets an SM of its own. Measured in CUDA
+        // graphs of 8 calls: weight quantiser 4096 x 4096, 12.3 us per call against 13.1; activation
+        // quantiser 4096 x 4096, 14.6 against 15.1; 8 / 64 tokens of 4096, 3.6 / 3.8 against 3.9 /
+        // 4.1. With more units per group the CTA-by-CTA numbering measured up to 3 % faster.
+        a.group_major = units <= 4 * G * full ? 1 : 0;
+        int64_t ctas = a.group_major ? units : (units + G - 1) / G;
         if (ctas > full) ctas = full;
         return sq::cuda_status(sq::launch_pdl(kern, dim3(static_cast<unsigned>(ctas)), dim3(kThreads), smem, st, nullptr, a),
                                "launch(rowquant)");
