@@ -342,6 +342,17 @@ def test_quantisers_at_the_width_limits(sq, orc, T, K):
     every_quantiser(sq, orc, T, K, 31)
 
 
+# Row counts on both sides of the switch between the two unit numberings of the quantisers (group by group
+# across the CTAs up to 4 units per row group, CTA by CTA beyond): 4 x 8 groups x 148 SMs = 4736 rows of
+# 4096 elements, 4 x 4 x 148 = 2368 rows of 8192.
+NUMBERING = [(4736, 4096), (4737, 4096), (2368, 8192), (2369, 8192)]
+
+
+@pytest.mark.parametrize("T,K", NUMBERING)
+def test_quantisers_across_the_unit_numberings(sq, orc, T, K):
+    every_quantiser(sq, orc, T, K, 41)
+
+
 def every_quantiser(sq, orc, T, K, seed):
     """Dynamic INT8 and FP8, static INT8 (with clipping), LayerNorm INT8 and the weight quantiser on
     T rows of K elements, each against the oracle (codes and scales bit-exact)."""
