@@ -319,6 +319,28 @@ def test_absmax_pair_matches_two_calls_at_every_split(sq):
     ok_status(sq)
 
 
+def test_empty_inputs_are_no_ops(sq):
+    """No tokens (T = 0) for every activation quantiser and the GEMM, no output channels (N = 0) for the
+    weight quantisers: each call returns success without a launch, and the device status stays clean."""
+    dev = "cuda"
+    K, N = 4096, 264
+    fold = torch.ones(K, device=dev)
+    x0 = torch.empty(0, K, dtype=torch.bfloat16, device=dev)
+    for q, sc in (sq.sq_rmsnorm_smooth_quant(x0, fold), sq.sq_rmsnorm_smooth_quant(x0, fold, apply_norm=False),
+                  sq.sq_rmsnorm_smooth_quant_fp8(x0, fold),
+                  sq.sq_rmsnorm_smooth_quant_static(x0, fold, sq.sq_static_scale(torch.ones(K, device=dev))),
+                  sq.sq_layernorm_smooth_quant(x0, fold, torch.zeros(K, device=dev))):
+        assert q.shape == (0, K) and sc.shape == (0,)
+    w0 = torch.empty(0, K, dtype=torch.bfloat16, device=dev)
+    for wq0, ws0 in (sq.sq_smooth_quantize_weight(w0, fold), sq.sq_smooth_quantize_weight_fp8(w0, fold)):
+        assert wq0.shape == (0, K) and ws0.shape == (0,)
+    wq = torch.zeros(N, K, dtype=torch.int8, device=dev)
+    ws = torch.ones(N, device=dev)
+    y = sq.sq_w8a8_linear(torch.empty(0, K, dtype=torch.int8, device=dev), torch.empty(0, device=dev), wq, ws)
+    assert y.shape == (0, N)
+    ok_status(sq)
+
+
 # Quantisers over few rows (decode-sized token counts) take one row per group of eight warps, up to 4
 # rows per SM; every quantiser mode against the oracle at token counts on both sides of that bound
 # (592 rows on 148 SMs), at widths whose rows fill the eight-warp group exactly (4096, 8192) or not
