@@ -12,7 +12,7 @@
  *   [W8A8]    "SmoothQuant and W8A8: Quantizing Activations Too"
  *   [WOVS]    "SmoothQuant: Weight-Only vs W8A8"
  *
- * Readings where the pages are silent or disagree (each is also listed in the design notes):
+ * Readings where the pages are silent or disagree:
  *   - Quantiser: symmetric, delta = max|v| / 127, code = round-half-away-from-zero(v * (127/max|v|)),
  *     clamped to [-127, 127]. The pages leave the tie rule open ([TAMING], "Why Outliers Break
  *     Quantization") or use half-to-even in a listing; half-away is the fixed reading. The
