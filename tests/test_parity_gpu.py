@@ -229,10 +229,11 @@ def test_edge_shapes(sq, orc, T, N, K, norm, bias):
     ok_status(sq)
 
 
-def test_extreme_codes_accumulate_exactly(sq, orc):
-    # all +-127 codes at K = 8192: |acc| = 8192 * 16129, the largest magnitude the path produces
+# all +-127 codes: |acc| = K * 16129; K = 8192 is the widest configuration, K = 131072 the widest the GEMM
+# accepts (131072 * 16129 = 2114060288 < 2^31), in the token-tile form and in the decode form (T <= 128)
+@pytest.mark.parametrize("T,N,K", [(130, 264, 8192), (130, 264, 131072), (16, 264, 131072)])
+def test_extreme_codes_accumulate_exactly(sq, orc, T, N, K):
     dev = "cuda"
-    T, N, K = 130, 264, 8192
     xq = torch.full((T, K), 127, dtype=torch.int8, device=dev)
     xq[1::2] = -127
     wq = torch.full((N, K), -127, dtype=torch.int8, device=dev)
