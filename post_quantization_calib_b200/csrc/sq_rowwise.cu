@@ -976,8 +976,8 @@ sq_status launch_rows_t(RowArgs a, const Geo &geo, int dev, cudaStream_t st) {
     const int64_t units = (a.rows + R - 1) / R;
     if (!ABS) {
         // Up to 4 units per row group: units are numbered group by group across the CTAs, so every SM
-        // gets an equal share (CTA by CTA, a third of the SMs would take a whole extra unit per group
-        // at 4096 rows), and below one unit per SM each unit gets an SM of its own. Measured in CUDA
+        // gets an equal share (CTA by CTA, 4096 rows on 148 x 8 groups give 68 SMs 32 rows and the
+        // other 80 SMs 24), and below one unit per SM each unit gets an SM of its own. Measured in CUDA
         // graphs of 8 calls: weight quantiser 4096 x 4096, 12.3 us per call against 13.1; activation
         // quantiser 4096 x 4096, 14.6 against 15.1; 8 / 64 tokens of 4096, 3.6 / 3.8 against 3.9 /
         // 4.1. With more units per group the CTA-by-CTA numbering measured up to 3 % faster.
