@@ -27,6 +27,24 @@ def test_reference_arm_prints_its_line():
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
+def test_reference_arm_under_two_ranks():
+    """Launched as the multi-GPU runs are (torchrun, two processes on 127.0.0.1): rank 0 alone times the
+    oracle and prints the line (n_gpus 2, parallelism dp2); the other rank exits 0 without work."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+                        "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "1", "--ref-seconds", "4"],
+                       cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["config"]["parallelism"] == "dp2" and d["value"] > 0
+
+
 def test_clock_summary_keeps_to_the_timed_window_and_names_reasons():
     """The clock record summarises the samples inside the timed steps (falling back to the whole run,
     and saying so, when that window holds fewer than three) and names every active slowdown reason."""
