@@ -18,7 +18,8 @@ Decode workloads add act_quant and gemm at each decode token count, once as a si
 call in a chain of 8 back-to-back calls captured in a CUDA graph (the way a decoder runs one layer after
 another, without the host's per-call cost; the 8 GEMMs read 8 distinct copies of the weight, which
 together exceed the L2). The GEMM chain is also timed issued call by call on the stream ("chain_form":
-"stream"), where each call's dependent launch overlaps the previous call's end. The HBM-bound stages
+"stream"), where each call's dependent launch overlaps the previous call's end, and whole decode layers
+(the activation quantiser, then the GEMM, 8 layers in one graph: stage "layer", per layer). The HBM-bound stages
 (calib_absmax_pair, weight_quant, act_quant) are likewise timed per call in a CUDA graph of 8 calls on 8
 copies of their inputs ("chain": 8), unless --no-chain is given.
 
@@ -240,7 +241,14 @@ def run_workload(w: synth.Workload, timer: Timer, peaks: Dict, device, stages=ST
                 rows.append(line(peaks, w.name, g, "gemm", timer.chained(gemms), gbytes, ops, T=T, N=N, K=K, chain=8))
                 rows.append(line(peaks, w.name, g, "gemm", timer.stream_chained(gemms), gbytes, ops, T=T, N=N, K=K,
                                  chain=8, chain_form="stream"))
-                del wqs, gemms
+                # whole decode layers: each layer quantises its own tokens, then multiplies by its own weight
+                xs8 = [x] + [x.clone() for _ in range(7)]
+                quants = [lambda c=c: sq.sq_rmsnorm_smooth_quant(c, fold, eps=w.eps, apply_norm=w.norm, xq=xq, x_scale=xs)
+                          for c in xs8]
+                layer = [f for pair in zip(quants, gemms) for f in pair]
+                rows.append(line(peaks, w.name, g, "layer", 2 * timer.chained(layer), qbytes + gbytes, ops, T=T, N=N, K=K,
+                                 chain=8, chain_form="layer"))
+                del wqs, gemms, xs8, quants, layer
         del calib
         torch.cuda.empty_cache()
     st = sq.sq_device_status()

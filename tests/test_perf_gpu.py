@@ -39,6 +39,11 @@ def test_perf_lines_for_the_smallest_and_the_decode_workload():
         assert ("decode_k4096_n14336", "gemm", T, 8) in stages
         assert ("decode_k4096_n14336", "act_quant", T, 8) in stages
         assert ("gemm", T, "stream") in forms and ("gemm", T, None) in forms
+        assert ("layer", T, "layer") in forms
+    # the HBM-bound stages of the small workload also per call in a chain of 8
+    for st in ("calib_absmax_pair", "weight_quant", "act_quant"):
+        assert any(r["workload"] == "single_linear_t256_k1024_n1024" and r["stage"] == st and r.get("chain") == 8
+                   for r in rows)
     for r in rows:
         assert r["us"] > 0 and r["gbs"] > 0 and r["peaks"] in ("measured", "fallback")
         if r["stage"] == "gemm":
